@@ -1,0 +1,213 @@
+"""CPU oracle for the HiLS attention forward pass -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never calls it, and it
+imports nothing from the CUDA package: the two sides share only the seeded
+input generator.
+
+The arithmetic lives in ``hils_oracle.c`` (plain C, fp64, OpenMP over rows),
+which follows the pages on HiLS attention step by step:
+
+* model card "HiLS-Attention" (axforge.ai), section "What HiLS-Attention is":
+  landmark-key chunk-mass surrogate, inter-/intra-chunk softmax factorisation,
+  top-k chunk selection, and the naive exact-chunk-mass selector;
+* "HiLS Attention Extrapolates 64x at 90% Retrieval Accuracy" (aiweekly.co):
+  each retrieved chunk attended independently, outputs fused by chunk scores;
+* "HiLS Attention: ..." (molayo1419.me), section "Core idea": the two-step
+  factorisation (inter-chunk attention over landmarks, then standard attention
+  inside the selected chunks) and section "Hardware-efficient kernel": the
+  union of the chunks of M adjacent queries.
+
+Every entry point is pinned in ``tests/test_oracle_pins.py`` against closed
+forms, hand-derived values and brute force; none is "parity unpinned".
+
+This module compiles the C source with gcc on first use (``build()``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hils_oracle.c")
+_LIB = os.path.join(_HERE, "libhils_oracle.so")
+
+MODES = {"landmark": 0, "given": 1, "exact_mass": 2}
+
+
+def compile_source(src: str, lib: str) -> str:
+    """Compile one oracle C source into a shared library (gcc, -O2, OpenMP)."""
+    tmp = lib + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared",
+                           "-o", tmp, src, "-lm"])
+    os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False) -> str:
+    """Compile ``hils_oracle.c`` into ``libhils_oracle.so`` when it is stale."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        compile_source(_SRC, _LIB)
+    return _LIB
+
+
+def _bind(path):
+    lib = ctypes.CDLL(path)
+    P, I, I64, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
+    lib.hils_oracle_rows.argtypes = [I, I, I, I, I, I, I, D, I, P, P, P, P, I64, P, I, P, P,
+                                     P, P, P, P, P, P, I]
+    lib.hils_oracle_rows.restype = I
+    lib.hils_oracle_decode.argtypes = [I, I, I, I, I, I, I, D, I, P, P, P, P, I64, P, P, P, P,
+                                       P, P, P, I]
+    lib.hils_oracle_decode.restype = I
+    lib.hils_oracle_union.argtypes = [I, I, I, I, I64, I64, P, P, I64]
+    lib.hils_oracle_union.restype = I64
+    return lib
+
+
+@dataclass
+class Problem:
+    """Shapes of one HiLS problem (BHLD layout, chunk size C, top-k)."""
+    B: int
+    Hq: int
+    Hkv: int
+    L: int
+    d: int
+    C: int
+    topk: int
+    scale: float
+
+
+def _as_array(x):
+    """Accept numpy arrays or CPU torch tensors (fp32, or bf16 kept as raw bits).
+
+    Returns (contiguous numpy array, is_bf16)."""
+    if hasattr(x, "detach"):  # torch tensor, imported lazily
+        import torch
+        x = x.detach()
+        if x.device.type != "cpu":
+            raise ValueError("oracle inputs must live in host memory")
+        if x.dtype == torch.bfloat16:
+            return np.ascontiguousarray(x.contiguous().view(torch.int16).numpy().view(np.uint16)), True
+        if x.dtype == torch.float32:
+            return np.ascontiguousarray(x.contiguous().numpy()), False
+        raise TypeError(f"unsupported oracle input dtype {x.dtype}")
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return np.ascontiguousarray(x), True
+    if x.dtype == np.float32:
+        return np.ascontiguousarray(x), False
+    if x.dtype == np.float64:
+        # fp64 inputs are rounded to fp32 storage: the oracle reads fp32 or bf16.
+        return np.ascontiguousarray(x.astype(np.float32)), False
+    raise TypeError(f"unsupported oracle input dtype {x.dtype}")
+
+
+def _inputs(q, k, v, lmk):
+    arrs = [_as_array(a) for a in (q, k, v, lmk)]
+    fmts = {b for _, b in arrs}
+    if len(fmts) != 1:
+        raise TypeError("q, k, v and lmk must share one element format")
+    return [a for a, _ in arrs], fmts.pop()
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _outputs(n, p):
+    return {
+        "sel": np.empty((n, p.topk), np.int32),
+        "w": np.empty((n, p.topk), np.float64),
+        "lse_lmk": np.empty((n,), np.float64),
+        "out": np.empty((n, p.d), np.float64),
+        "lse": np.empty((n,), np.float64),
+        "wfin": np.empty((n, p.topk + 1), np.float64),
+    }
+
+
+class Oracle:
+    """The oracle bound to one compiled library (the default one, or a test's
+    deliberately broken copy)."""
+
+    def __init__(self, lib_path: str | None = None):
+        self.lib = _bind(lib_path or build())
+
+    def rows(self, p: Problem, q, k, v, lmk, rows, mode: str = "landmark", sel_in=None,
+             w_in=None, nthreads: int = 0) -> dict:
+        """Prefill rows (flat indices (b*Hq + hq)*L + t).
+
+        Returns numpy arrays: sel [n,k] int32 (ascending, -1 pad), w [n,k]
+        (selected logits, -inf pad), lse_lmk [n], out [n,d], lse [n],
+        wfin [n,k+1] (fusion weights in sel order, own chunk last)."""
+        (qa, ka, va, la), bf16 = _inputs(q, k, v, lmk)
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
+        n = r.shape[0]
+        res = _outputs(n, p)
+        si = wi = None
+        if mode == "given":
+            si = np.ascontiguousarray(np.asarray(sel_in, dtype=np.int32).reshape(n, p.topk))
+            wi = np.ascontiguousarray(np.asarray(w_in, dtype=np.float64).reshape(n, p.topk))
+        rc = self.lib.hils_oracle_rows(
+            p.B, p.Hq, p.Hkv, p.L, p.d, p.C, p.topk, p.scale, int(bf16), _ptr(qa), _ptr(ka),
+            _ptr(va), _ptr(la), n, _ptr(r), MODES[mode], _ptr(si), _ptr(wi), _ptr(res["sel"]),
+            _ptr(res["w"]), _ptr(res["lse_lmk"]), _ptr(res["out"]), _ptr(res["lse"]),
+            _ptr(res["wfin"]), int(nthreads))
+        if rc != 0:
+            raise ValueError("oracle rejected its arguments")
+        return res
+
+    def decode(self, p: Problem, q, k, v, lmk, heads=None, nthreads: int = 0) -> dict:
+        """Decode step: q is [B,Hq,d], the cache length is p.L and the query
+        position is p.L - 1.  heads: flat b*Hq + hq (default: all)."""
+        (qa, ka, va, la), bf16 = _inputs(q, k, v, lmk)
+        h = np.arange(p.B * p.Hq, dtype=np.int64) if heads is None else heads
+        h = np.ascontiguousarray(np.asarray(h, dtype=np.int64).reshape(-1))
+        n = h.shape[0]
+        res = _outputs(n, p)
+        rc = self.lib.hils_oracle_decode(
+            p.B, p.Hq, p.Hkv, p.L, p.d, p.C, p.topk, p.scale, int(bf16), _ptr(qa), _ptr(ka),
+            _ptr(va), _ptr(la), n, _ptr(h), _ptr(res["sel"]), _ptr(res["w"]),
+            _ptr(res["lse_lmk"]), _ptr(res["out"]), _ptr(res["lse"]), _ptr(res["wfin"]),
+            int(nthreads))
+        if rc != 0:
+            raise ValueError("oracle rejected its arguments")
+        return res
+
+    def union(self, L: int, C: int, topk: int, M: int, head: int, g: int, sel) -> np.ndarray:
+        """Sorted chunk union of query group g (rows [g*M, (g+1)*M)) of flat
+        head `head`, from a full selection array sel [B*Hq*L, topk]."""
+        s = np.ascontiguousarray(np.asarray(sel, dtype=np.int32))
+        cap = (L + C - 1) // C
+        u = np.empty((cap,), np.int32)
+        n = self.lib.hils_oracle_union(L, C, topk, M, head, g, _ptr(s), _ptr(u), cap)
+        if n < 0:
+            raise ValueError("union capacity exceeded")
+        return u[:n].copy()
+
+
+_default = None
+
+
+def default() -> Oracle:
+    """The oracle compiled from ``hils_oracle.c``."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default
+
+
+def rows(*a, **kw):
+    return default().rows(*a, **kw)
+
+
+def decode(*a, **kw):
+    return default().decode(*a, **kw)
+
+
+def union(*a, **kw):
+    return default().union(*a, **kw)
