@@ -1,0 +1,505 @@
+#!/usr/bin/env python3
+"""Benchmark of the HiLS attention forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--extra/--no-extra] [--no-cpu-baseline]
+
+One step = one pass of the whole prefill hot path over the workload's
+synthetic batch: landmark scoring + inter-chunk normaliser + top-k
+(hils_select), then the chunk union, intra-chunk attention and fusion
+(hils_attn_fwd, which builds each tile's union itself).  Default workload:
+the 512K-token 7B-shaped prefill (B=1, 32/8 heads, d=128, k=64, M=128).
+The 128K prefill and the B=16 x 512K decode step are timed as extra lines
+inside the same JSON object ("workloads").
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
+cuda synchronize, CUDA events on the launching stream, max over ranks.
+Inputs (q alone is 4.3 GB) are larger than the 126 MB L2, so no flush is
+needed between steps.  Multi-GPU (torchrun): every rank runs its own
+independent batch (different seed); value = all ranks' query tokens / the
+slowest rank's time ("weak" scaling, no collective on the data path).
+
+`--impl reference` times the CPU oracle (the reference implementation of
+this project, plain fp64 C) on the host cores for the same workload: a
+bounded sample of rows per step, scaled to query-tokens/s.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from chunk_wise_hierarchical_landmark_b200 import workloads as W  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+CSRC = os.path.join(ROOT, "chunk_wise_hierarchical_landmark_b200", "csrc")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work
+
+def prefill_work(w: W.Workload) -> dict:
+    """Algorithmic FLOPs of one prefill over all heads (exact sums over t).
+    Scoring: 2*d FLOP per (row, completed chunk).  Attention: 4*d FLOP per
+    (row, attended key) -- QK^T and PV -- over min(k, n_c) full chunks plus
+    the t mod C + 1 causal keys of the own chunk."""
+    t = np.arange(w.L, dtype=np.int64)
+    n_c = t // w.C
+    keys = np.minimum(w.topk, n_c) * w.C + (t % w.C) + 1
+    heads = w.B * w.Hq
+    return {"score_flop": float(2 * w.d * n_c.sum() * heads),
+            "attn_flop": float(4 * w.d * keys.sum() * heads),
+            "candidates": float(n_c.sum() * heads)}
+
+
+def decode_bytes(w: W.Workload, sel: torch.Tensor) -> float:
+    """Algorithmic HBM bytes of one decode step: every landmark key of every
+    (b, hkv), plus the K and V of the union of chunks the G query heads of a
+    KV head attend (selected chunks and the own chunk), each read once."""
+    esize = 2 if w.dtype == "bf16" else 4
+    G = w.Hq // w.Hkv
+    lmk = w.B * w.Hkv * (w.L // w.C) * w.d * esize
+    s = sel.reshape(w.B, w.Hkv, G * w.topk).cpu().numpy()
+    own = (w.L - 1) // w.C
+    chunks = 0
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            u = set(int(c) for c in s[b, h] if c >= 0)
+            u.add(own)
+            chunks += len(u)
+    last = w.L - own * w.C  # keys in the own chunk
+    kv = (chunks - w.B * w.Hkv) * w.C + w.B * w.Hkv * last
+    return float(lmk + 2 * kv * w.d * esize)
+
+
+def source_hash(files):
+    h = hashlib.sha256()
+    for f in sorted(files):
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def load_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu capture, or None when the
+    kernel's source changed since the capture."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("workload") != workload:
+        return None
+    if rec.get("source_hash") != source_hash(rec.get("sources", [])):
+        return None
+    return rec.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    Q = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.uuid = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            pass
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=10)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 10:
+                continue
+            if self.uuid and self.uuid.replace("GPU-", "") not in f[1]:
+                continue
+            rows.append(f)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][3]) if rows[0][3].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# distributed helpers
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+# ---------------------------------------------------------------------------
+# our arm
+
+def bench_prefill(hb, synth, w, steps, warmup, ws, rank, seed_offset, e2e=True, clocks=True):
+    dev = torch.device("cuda")
+    q, k, v, lmk = synth.make_inputs(w, "cuda", seed=w.seed + seed_offset)
+    p = hb.make_params(w.B, w.Hq, w.Hkv, w.L, w.d, w.topk, w.M, w.C, w.scale,
+                       q.dtype, False)
+    B, Hq, L, K = w.B, w.Hq, w.L, w.topk
+    sel = torch.empty((B, Hq, L, K), dtype=torch.int32, device=dev)
+    cw = torch.empty((B, Hq, L, K), dtype=torch.float32, device=dev)
+    lse_lmk = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        hb.hils_select(p, q, lmk, sel, cw, lse_lmk, None, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        hb.hils_attn_fwd(p, q, k, v, sel, cw, out, lse, None, None, stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    n0 = hb.launch_count()
+    sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
+    if sampler:
+        sampler.__enter__()
+    barrier(ws)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    if sampler:
+        sampler.__exit__(None, None, None)
+    launches = hb.launch_count() - n0
+    ms = t0.elapsed_time(t1) / steps
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    res = dict(ms=ms, sel_ms=sel_ms, attn_ms=attn_ms, launches=launches,
+               clocks=sampler.summary() if sampler else None)
+
+    if e2e:
+        hq, hk, hv, hl = (x.cpu().pin_memory() for x in (q, k, v, lmk))
+        ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        hlse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            lmk.copy_(hl, non_blocking=True)
+            hb.hils_prefill(p, q, k, v, lmk, sel, cw, lse_lmk, out, lse, None, stream)
+            ho.copy_(out, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(ws)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        n_e2e = max(1, min(steps, 3))
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+        res["e2e_ms"] = a.elapsed_time(b) / n_e2e
+        res["h2d"] = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hl))
+        res["d2h"] = ho.numel() * ho.element_size() + hlse.numel() * hlse.element_size()
+        res["host_inputs"] = (hq, hk, hv, hl)
+    res["sel"] = sel
+    return res
+
+
+def bench_decode(hb, synth, w, steps, warmup, seed_offset):
+    dev = torch.device("cuda")
+    q, k, v, lmk = synth.make_inputs(w, "cuda", seed=w.seed + seed_offset)
+    p = hb.make_params(w.B, w.Hq, w.Hkv, w.L, w.d, w.topk, w.M, w.C, w.scale, q.dtype, False)
+    sel = torch.empty((w.B, w.Hq, w.topk), dtype=torch.int32, device=dev)
+    cw = torch.empty_like(sel, dtype=torch.float32)
+    lse_lmk = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    ws_t = hb.workspace(p, hb.HILS_OP_DECODE, dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        hb.hils_decode_fwd(p, q, k, v, lmk, sel, cw, lse_lmk, out, lse, ws_t, stream)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        hb.hils_decode_fwd(p, q, k, v, lmk, sel, cw, lse_lmk, out, lse, ws_t, stream)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    nbytes = decode_bytes(w, sel)
+    return dict(ms=ms, bytes=nbytes)
+
+
+def union_stats(hb, sel, w):
+    """Chunk-union size per group of M rows and adjacent-query overlap."""
+    u_off, _ = hb.union(sel, M=w.M)
+    sizes = (u_off[1:] - u_off[:-1]).float()
+    s = sel.reshape(-1, w.L, w.topk)
+    h = min(4, s.shape[0])
+    ov = []
+    for i in range(h):
+        a = s[i, w.topk * w.C + 1:-1].cpu().numpy()
+        bb = s[i, w.topk * w.C + 2:].cpu().numpy()
+        inter = [(len(set(x) & set(y)) / w.topk) for x, y in zip(a[::97], bb[::97])]
+        ov.extend(inter)
+    return {"union_mean": round(sizes.mean().item(), 2),
+            "union_p50": float(sizes.median().item()),
+            "union_p99": float(torch.quantile(sizes, 0.99).item()),
+            "adjacent_overlap": round(float(np.mean(ov)) if ov else float("nan"), 4),
+            "pages_adjacent_overlap": 0.928}
+
+
+def cpu_baseline(w, host_inputs, budget_s=15.0):
+    """The oracle, as it stands, on all host cores over a bounded sample of
+    rows of the same workload; scaled to query-tokens/s."""
+    import oracle
+    q, k, v, lmk = host_inputs
+    p = oracle.Problem(w.B, w.Hq, w.Hkv, w.L, w.d, w.C, w.topk, w.scale)
+    cores = os.cpu_count() or 1
+    rng = np.random.default_rng(w.seed)
+    rows_per_try = max(cores, 8)
+    done = 0
+    t_total = 0.0
+    while t_total < budget_s and done < 1 << 20:
+        rows = rng.integers(0, w.B * w.Hq * w.L, size=rows_per_try)
+        t0 = time.perf_counter()
+        oracle.rows(p, q, k, v, lmk, rows, nthreads=cores)
+        t_total += time.perf_counter() - t0
+        done += rows_per_try
+        rows_per_try = min(rows_per_try * 2, 4096)
+    rows_per_s = done / t_total
+    return {"value": rows_per_s / w.Hq, "unit": "query-tokens/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{done} rows drawn uniformly over (b, head, position) of {w.name}; "
+                      f"{t_total:.1f} s on {cores} threads; value = rows/s / Hq"}
+
+
+def run_ours(args):
+    ws, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    from chunk_wise_hierarchical_landmark_b200 import binding as hb
+    from chunk_wise_hierarchical_landmark_b200 import synth
+    hb.lib()
+    w = W.BY_NAME[args.workload]
+    res = bench_prefill(hb, synth, w, args.steps, args.warmup, ws, rank, seed_offset=rank)
+    ms = max_over_ranks(res["ms"], ws)
+    e2e_ms = max_over_ranks(res["e2e_ms"], ws)
+    qtok = w.B * w.L * ws
+    work = prefill_work(w)
+    peaks, peak_src = load_peaks()
+    # dominant kernel by time share
+    kernels = {
+        "hils_select": {"ms": res["sel_ms"], "flop": work["score_flop"]},
+        "hils_attn_fwd": {"ms": res["attn_ms"], "flop": work["attn_flop"]},
+    }
+    dom = max(kernels, key=lambda kname: kernels[kname]["ms"])
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    achieved = kernels[dom]["flop"] / (kernels[dom]["ms"] * 1e-3) / 1e12
+    line = {
+        "metric": "HiLS fwd query-tokens/s (prefill, 512K tokens, 7B-shaped GQA 32/8, d=128)",
+        "value": qtok / (ms * 1e-3),
+        "unit": "query-tokens/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded; per-rank seed offset)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "d": w.d,
+                   "chunk": w.C, "topk": w.topk, "M": w.M,
+                   "l2": "inputs larger than L2 (q alone %.1f GB); no flush" %
+                         (w.B * w.Hq * w.L * w.d * 2 / 1e9),
+                   "parallelism": f"independent batch per GPU x{ws}"},
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_src} bf16 dense, sustained",
+                     "traffic": load_traffic(dom, w.name)},
+        "kernels": {kn: {"ms": round(kv["ms"], 3), "algorithmic_tflops": round(kv["flop"] / (kv["ms"] * 1e-3) / 1e12, 3),
+                         "share": round(kv["ms"] / (res["sel_ms"] + res["attn_ms"]), 3)}
+                    for kn, kv in kernels.items()},
+        "e2e": {"value": qtok / (e2e_ms * 1e-3), "unit": "query-tokens/s",
+                "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+        "gpu_launches": res["launches"],
+        "clocks": res["clocks"],
+    }
+    if args.extra:
+        extra = {}
+        try:
+            extra["union"] = union_stats(hb, res["sel"], w)
+        except Exception as e:  # statistics only
+            extra["union"] = {"error": str(e)[:200]}
+        del res["sel"]
+        w2 = W.PREFILL_128K
+        r2 = bench_prefill(hb, synth, w2, max(3, args.steps), 3, ws, rank, rank, e2e=False,
+                           clocks=False)
+        wk2 = prefill_work(w2)
+        extra[w2.name] = {"value": w2.B * w2.L * ws / (max_over_ranks(r2["ms"], ws) * 1e-3),
+                          "unit": "query-tokens/s", "ms_per_step": r2["ms"],
+                          "select_ms": r2["sel_ms"], "attn_ms": r2["attn_ms"],
+                          "attn_tflops": wk2["attn_flop"] / (r2["attn_ms"] * 1e-3) / 1e12,
+                          "select_tflops": wk2["score_flop"] / (r2["sel_ms"] * 1e-3) / 1e12}
+        del r2
+        torch.cuda.empty_cache()
+        w3 = W.DECODE_512K
+        r3 = bench_decode(hb, synth, w3, max(5, args.steps), 3, rank)
+        gbs = r3["bytes"] / (r3["ms"] * 1e-3) / 1e9
+        extra[w3.name] = {"value": w3.B * ws / (max_over_ranks(r3["ms"], ws) * 1e-3),
+                          "unit": "query-tokens/s", "ms_per_step": r3["ms"],
+                          "algorithmic_bytes": r3["bytes"], "achieved_gbs": gbs,
+                          "hbm_frac": gbs / peaks["hbm_gbs"]}
+        line["workloads"] = extra
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, res["host_inputs"])
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from chunk_wise_hierarchical_landmark_b200 import synth
+    w = W.BY_NAME[args.workload]
+    host = synth.make_inputs(w, "cuda" if torch.cuda.is_available() else "cpu")
+    host = tuple(x.cpu() for x in host)
+    p = oracle.Problem(w.B, w.Hq, w.Hkv, w.L, w.d, w.C, w.topk, w.scale)
+    cores = os.cpu_count() or 1
+    rng = np.random.default_rng(w.seed)
+    per_step = max(cores * 4, 64)
+    q, k, v, lmk = host
+    for _ in range(args.warmup):
+        oracle.rows(p, q, k, v, lmk, rng.integers(0, w.B * w.Hq * w.L, size=cores), nthreads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.rows(p, q, k, v, lmk, rng.integers(0, w.B * w.Hq * w.L, size=per_step),
+                    nthreads=cores)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = per_step / dt / w.Hq
+    sample = (f"{per_step} rows per step drawn uniformly over (b, head, position) of {w.name}; "
+              f"value = rows/s / Hq")
+    line = {
+        "impl": "reference",
+        "metric": "HiLS fwd query-tokens/s (prefill, 512K tokens, 7B-shaped GQA 32/8, d=128)",
+        "value": value, "unit": "query-tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "d": w.d,
+                   "chunk": w.C, "topk": w.topk, "M": w.M},
+        "cpu_baseline": {"value": value, "unit": "query-tokens/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "query-tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=W.PREFILL_512K.name, choices=sorted(W.BY_NAME))
+    ap.add_argument("--extra", dest="extra", action="store_true", default=True)
+    ap.add_argument("--no-extra", dest="extra", action="store_false")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

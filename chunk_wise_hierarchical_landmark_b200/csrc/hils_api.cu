@@ -1,0 +1,241 @@
+// C ABI of libhils.so (declared in include/hils.h): argument validation,
+// workspace sizing, kernel dispatch and status reporting.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/hils.h"
+#include "kernels.h"
+
+#define HILS_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+std::atomic<int64_t> g_launches{0};
+thread_local char g_msg[256] = "";
+
+hils_status fail(hils_status s, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+hils_status fail(hils_status s, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+hils_status cuda_fail(cudaError_t e, const char *where) {
+  return fail(HILS_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+constexpr int kMaxL = 1 << 24;
+constexpr size_t kDebugWs = 256;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+hils_status check_params(const hils_params *p) {
+  if (!p) return fail(HILS_ERR_INVALID_ARG, "params is NULL");
+  if (p->B < 1 || p->Hq < 1 || p->Hkv < 1 || p->L < 1 || p->d < 1 || p->chunk < 1 ||
+      p->topk < 1 || p->M < 1)
+    return fail(HILS_ERR_INVALID_ARG, "shape fields must be >= 1");
+  if (p->Hq % p->Hkv) return fail(HILS_ERR_INVALID_ARG, "Hq %% Hkv != 0");
+  if (!std::isfinite(p->scale)) return fail(HILS_ERR_INVALID_ARG, "scale is not finite");
+  if (p->dtype != HILS_F32 && p->dtype != HILS_BF16)
+    return fail(HILS_ERR_INVALID_ARG, "unknown dtype %d", p->dtype);
+  if (p->debug_checks != 0 && p->debug_checks != 1)
+    return fail(HILS_ERR_INVALID_ARG, "debug_checks must be 0 or 1");
+  if (p->d != 64 && p->d != 128) return fail(HILS_ERR_UNSUPPORTED, "d=%d (supported: 64, 128)", p->d);
+  if (p->chunk != 64) return fail(HILS_ERR_UNSUPPORTED, "chunk=%d (supported: 64)", p->chunk);
+  if (p->topk > 64) return fail(HILS_ERR_UNSUPPORTED, "topk=%d (supported: 1..64)", p->topk);
+  if (p->M != 16 && p->M != 32 && p->M != 64 && p->M != 128)
+    return fail(HILS_ERR_UNSUPPORTED, "M=%d (supported: 16, 32, 64, 128)", p->M);
+  if (p->L > kMaxL) return fail(HILS_ERR_UNSUPPORTED, "L=%d above %d", p->L, kMaxL);
+  if ((int64_t)p->B * p->Hq > (1 << 16) - 1)
+    return fail(HILS_ERR_UNSUPPORTED, "B*Hq above 65535");
+  return HILS_OK;
+}
+
+#define NEED(ptr)                                                              \
+  do {                                                                         \
+    if (!(ptr)) return fail(HILS_ERR_INVALID_ARG, #ptr " is NULL");            \
+    if (!aligned16(ptr)) return fail(HILS_ERR_INVALID_ARG, #ptr " is not 16-byte aligned"); \
+  } while (0)
+#define MAYBE(ptr)                                                             \
+  do {                                                                         \
+    if ((ptr) && !aligned16(ptr)) return fail(HILS_ERR_INVALID_ARG, #ptr " is not 16-byte aligned"); \
+  } while (0)
+
+hils::RowSpec prefill_rows(const hils_params *p) {
+  return hils::RowSpec{p->B, p->Hq, p->Hkv, p->L, p->d, p->chunk, p->topk, p->scale, 0, p->L};
+}
+hils::RowSpec decode_rows(const hils_params *p) {
+  return hils::RowSpec{p->B, p->Hq, p->Hkv, p->L, p->d, p->chunk, p->topk, p->scale, p->L - 1, 1};
+}
+
+// Debug mode: clear the device error word before the launches ...
+hils_status debug_begin(const hils_params *p, void *ws, size_t ws_bytes, uint32_t **err,
+                        cudaStream_t st) {
+  *err = nullptr;
+  if (!p->debug_checks) return HILS_OK;
+  if (!ws || ws_bytes < kDebugWs) return fail(HILS_ERR_WORKSPACE, "debug_checks needs %zu bytes of workspace", kDebugWs);
+  *err = static_cast<uint32_t *>(ws);
+  cudaError_t e = cudaMemsetAsync(*err, 0, sizeof(uint32_t), st);
+  return e == cudaSuccess ? HILS_OK : cuda_fail(e, "cudaMemsetAsync");
+}
+// ... and read it back (synchronising the stream) after them.
+hils_status debug_end(uint32_t *err, cudaStream_t st) {
+  if (!err) return HILS_OK;
+  uint32_t code = 0;
+  cudaError_t e = cudaMemcpyAsync(&code, err, sizeof code, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "debug read-back");
+  if (code == 5) return fail(HILS_ERR_DEVICE_CHECK, "a device-side check found an invalid chunk index");
+  if (code == 6) return fail(HILS_ERR_TIMEOUT, "a bounded device wait gave up");
+  if (code) return fail(HILS_ERR_DEVICE_CHECK, "device error word %u", code);
+  return HILS_OK;
+}
+
+hils_status do_select(const hils_params *p, const hils::RowSpec &rs, const void *q,
+                      const void *lmk, int32_t *sel, float *w, float *lse_lmk, cudaStream_t st) {
+  cudaError_t e = hils::select_simt(rs, p->dtype == HILS_BF16, q, lmk, sel, w, lse_lmk, st);
+  g_launches += 1;
+  return e == cudaSuccess ? HILS_OK : cuda_fail(e, "select launch");
+}
+
+hils_status do_attn(const hils_params *p, const hils::RowSpec &rs, const void *q, const void *k,
+                    const void *v, const int32_t *sel, const float *w, void *out, float *lse,
+                    float *wfin, uint32_t *err, cudaStream_t st) {
+  cudaError_t e =
+      hils::attn_simt(rs, p->dtype == HILS_BF16, q, k, v, sel, w, out, lse, wfin, err, st);
+  g_launches += 1;
+  return e == cudaSuccess ? HILS_OK : cuda_fail(e, "attention launch");
+}
+
+}  // namespace
+
+HILS_API size_t hils_workspace_size(const hils_params *p, int op) {
+  if (check_params(p) != HILS_OK) return 0;
+  if (op != HILS_OP_PREFILL && op != HILS_OP_DECODE) return 0;
+  return p->debug_checks ? kDebugWs : 0;
+}
+
+HILS_API hils_status hils_select(const hils_params *p, const void *q, const void *lmk_k,
+                                 int32_t *sel_idx, float *chunk_w, float *lse_lmk, void *ws,
+                                 size_t ws_bytes, void *stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  NEED(q);
+  NEED(sel_idx);
+  NEED(chunk_w);
+  MAYBE(lse_lmk);
+  if (p->L >= p->chunk) NEED(lmk_k);
+  (void)ws;
+  (void)ws_bytes;
+  return do_select(p, prefill_rows(p), q, lmk_k, sel_idx, chunk_w, lse_lmk,
+                   static_cast<cudaStream_t>(stream));
+}
+
+HILS_API int64_t hils_union_capacity(const hils_params *p) {
+  if (check_params(p) != HILS_OK) return -1;
+  const int64_t nchunks = (p->L + p->chunk - 1) / p->chunk;
+  const int64_t gph = (p->L + p->M - 1) / p->M;
+  const int64_t per = std::min<int64_t>(nchunks, (int64_t)p->M * p->topk + p->M / p->chunk + 2);
+  return (int64_t)p->B * p->Hq * gph * per;
+}
+
+HILS_API hils_status hils_union(const hils_params *p, const int32_t *sel_idx, int32_t *u_off,
+                                int32_t *u_idx, int64_t u_cap, void *ws, size_t ws_bytes,
+                                void *stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  NEED(sel_idx);
+  NEED(u_off);
+  NEED(u_idx);
+  if (u_cap < hils_union_capacity(p))
+    return fail(HILS_ERR_INVALID_ARG, "u_cap %lld below hils_union_capacity", (long long)u_cap);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t *err = nullptr;
+  if ((s = debug_begin(p, ws, ws_bytes, &err, st)) != HILS_OK) return s;
+  int n = 0;
+  cudaError_t e = hils::union_csr(p->B, p->Hq, p->L, p->chunk, p->topk, p->M, sel_idx, u_off,
+                                  u_idx, u_cap, err, st, &n);
+  g_launches += n;
+  if (e != cudaSuccess) return cuda_fail(e, "union launch");
+  return debug_end(err, st);
+}
+
+HILS_API hils_status hils_attn_fwd(const hils_params *p, const void *q, const void *k,
+                                   const void *v, const int32_t *sel_idx, const float *chunk_w,
+                                   void *out, float *lse, float *w_final, void *ws,
+                                   size_t ws_bytes, void *stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  NEED(q);
+  NEED(k);
+  NEED(v);
+  NEED(sel_idx);
+  NEED(chunk_w);
+  NEED(out);
+  NEED(lse);
+  MAYBE(w_final);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t *err = nullptr;
+  if ((s = debug_begin(p, ws, ws_bytes, &err, st)) != HILS_OK) return s;
+  s = do_attn(p, prefill_rows(p), q, k, v, sel_idx, chunk_w, out, lse, w_final, err, st);
+  if (s != HILS_OK) return s;
+  return debug_end(err, st);
+}
+
+HILS_API hils_status hils_prefill(const hils_params *p, const void *q, const void *k,
+                                  const void *v, const void *lmk_k, int32_t *sel_idx,
+                                  float *chunk_w, float *lse_lmk, void *out, float *lse, void *ws,
+                                  size_t ws_bytes, void *stream) {
+  hils_status s = hils_select(p, q, lmk_k, sel_idx, chunk_w, lse_lmk, ws, ws_bytes, stream);
+  if (s != HILS_OK) return s;
+  return hils_attn_fwd(p, q, k, v, sel_idx, chunk_w, out, lse, nullptr, ws, ws_bytes, stream);
+}
+
+HILS_API hils_status hils_decode_fwd(const hils_params *p, const void *q, const void *k_cache,
+                                     const void *v_cache, const void *lmk_k, int32_t *sel_idx,
+                                     float *chunk_w, float *lse_lmk, void *out, float *lse,
+                                     void *ws, size_t ws_bytes, void *stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  NEED(q);
+  NEED(k_cache);
+  NEED(v_cache);
+  NEED(sel_idx);
+  NEED(chunk_w);
+  NEED(out);
+  NEED(lse);
+  MAYBE(lse_lmk);
+  if (p->L > p->chunk) NEED(lmk_k);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t *err = nullptr;
+  if ((s = debug_begin(p, ws, ws_bytes, &err, st)) != HILS_OK) return s;
+  const hils::RowSpec rs = decode_rows(p);
+  if ((s = do_select(p, rs, q, lmk_k, sel_idx, chunk_w, lse_lmk, st)) != HILS_OK) return s;
+  if ((s = do_attn(p, rs, q, k_cache, v_cache, sel_idx, chunk_w, out, lse, nullptr, err, st)) !=
+      HILS_OK)
+    return s;
+  return debug_end(err, st);
+}
+
+HILS_API const char *hils_status_string(hils_status s) {
+  switch (s) {
+    case HILS_OK: return "ok";
+    case HILS_ERR_INVALID_ARG: return "invalid argument";
+    case HILS_ERR_UNSUPPORTED: return "unsupported configuration";
+    case HILS_ERR_WORKSPACE: return "workspace too small";
+    case HILS_ERR_CUDA: return "CUDA error";
+    case HILS_ERR_DEVICE_CHECK: return "device-side check failed";
+    case HILS_ERR_TIMEOUT: return "bounded device wait timed out";
+  }
+  return "unknown status";
+}
+
+HILS_API const char *hils_last_error(void) { return g_msg; }
+
+HILS_API int64_t hils_launch_count(void) { return g_launches.load(); }

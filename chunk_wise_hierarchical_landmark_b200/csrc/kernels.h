@@ -1,0 +1,33 @@
+// Internal launcher interface between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace hils {
+
+// Rows handled by a launch: positions [t_first, t_first + t_count) of every
+// (b, hq) head.  Query row (bh, t) lives at q + (bh * t_count + t - t_first) * d
+// and so do the per-row outputs (prefill: t_first = 0, t_count = L; decode:
+// t_first = N - 1, t_count = 1 with q laid out [B, Hq, d]).
+struct RowSpec {
+  int B, Hq, Hkv, L, d, C, topk;
+  float scale;
+  int t_first, t_count;
+};
+
+// SIMT kernels (hils_simt.cu)
+cudaError_t select_simt(const RowSpec &rs, bool bf16, const void *q, const void *lmk,
+                        int32_t *sel, float *w, float *lse_lmk, cudaStream_t st);
+cudaError_t attn_simt(const RowSpec &rs, bool bf16, const void *q, const void *k, const void *v,
+                      const int32_t *sel, const float *w, void *out, float *lse, float *wfin,
+                      uint32_t *err, cudaStream_t st);
+size_t simt_attn_smem(int d, int L, int C);
+
+// Chunk union in CSR form (hils_union.cu)
+cudaError_t union_csr(int B, int Hq, int L, int C, int topk, int M, const int32_t *sel,
+                      int32_t *u_off, int32_t *u_idx, int64_t u_cap, uint32_t *err,
+                      cudaStream_t st, int *launches);
+
+}  // namespace hils

@@ -1,0 +1,174 @@
+/*
+ * hils.h -- C ABI of libhils.so: the forward pass of HiLS (Hierarchical
+ * Landmark Sparse) attention on NVIDIA B200 (sm_100a).
+ *
+ * The method (pages on "Hierarchical Sparse Attention Done Right: Toward
+ * Infinite Context Modeling"):
+ *   - model card "HiLS-Attention" (axforge.ai), section "What HiLS-Attention
+ *     is": one compressed (landmark) key per chunk estimates the chunk's mass;
+ *     attention factorises into an inter-chunk and an intra-chunk softmax; the
+ *     top-k chunks are selected;
+ *   - molayo1419.me article, section "Core idea": step 1, inter-chunk
+ *     attention of the query over all landmark keys; step 2, standard
+ *     attention inside the selected chunks;
+ *   - aiweekly.co article, mechanism paragraph: each query attends to each
+ *     retrieved chunk independently and the outputs are fused by the chunk
+ *     retrieval scores;
+ *   - molayo1419.me article, section "Hardware-efficient kernel": M adjacent
+ *     queries share the union of their chunks, loaded once.
+ *
+ * Conventions shared by every call
+ *   Layout: BHLD, contiguous.  q [B,Hq,L,d], k and v [B,Hkv,L,d], landmark
+ *   keys lmk_k [B,Hkv,floor(L/C),d] (one per complete chunk).  Query head hq
+ *   reads KV head hq / (Hq/Hkv).  Element type of q, k, v, lmk_k and out is
+ *   params.dtype (fp32 or bf16); chunk_w, lse_lmk, lse and w_final are fp32;
+ *   sel_idx is int32.
+ *   Row t (0-based) has own chunk floor(t/C) and completed chunks
+ *   c < floor(t/C).  Its own chunk is always attended, causally (keys <= t),
+ *   with fusion logit equal to the log-sum-exp of its causal token logits;
+ *   it does not take a top-k slot.  Selection order is (landmark logit
+ *   descending, chunk index ascending); rows with fewer than k completed
+ *   chunks select all of them.  The fusion weights are a softmax over the
+ *   selected landmark logits plus the own-chunk logit.
+ *   Pointers: every array argument is a DEVICE pointer owned by the caller,
+ *   16-byte aligned.  The library allocates no device memory and keeps no
+ *   state other than cached device attributes and a launch counter.
+ *   Streams: every call is asynchronous on `stream` (a cudaStream_t passed as
+ *   void*; NULL = legacy default stream).  Argument and shape errors are
+ *   returned before anything is launched.  A launch failure returns
+ *   HILS_ERR_CUDA.  With params.debug_checks = 1 the call also validates its
+ *   selections on the device and synchronises the stream to report
+ *   HILS_ERR_DEVICE_CHECK (a bad index) or HILS_ERR_TIMEOUT (a bounded
+ *   device wait gave up); device code never traps.
+ *   Supported: dtype bf16 with d in {64, 128}, or fp32 with d in {64, 128};
+ *   chunk C = 64; 1 <= topk <= 64; Hq % Hkv == 0; M in {16, 32, 64, 128};
+ *   L >= 1 (a ragged last chunk is allowed; it is never complete).  Anything
+ *   else returns HILS_ERR_UNSUPPORTED.
+ */
+#ifndef HILS_H_
+#define HILS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HILS_OK = 0,
+  HILS_ERR_INVALID_ARG = 1, /* null pointer, misaligned pointer, bad shape */
+  HILS_ERR_UNSUPPORTED = 2, /* valid but not implemented (dtype, d, chunk...) */
+  HILS_ERR_WORKSPACE = 3,   /* ws too small (see hils_workspace_size) */
+  HILS_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  HILS_ERR_DEVICE_CHECK = 5,/* debug_checks: a device-side check failed */
+  HILS_ERR_TIMEOUT = 6      /* debug_checks: a bounded device wait gave up */
+} hils_status;
+
+typedef enum { HILS_F32 = 0, HILS_BF16 = 1 } hils_dtype;
+
+typedef struct {
+  int B, Hq, Hkv; /* batch, query heads, KV heads (Hq % Hkv == 0) */
+  int L;          /* prefill: sequence length; decode: KV-cache length N,
+                     which already includes the new token (query at N-1) */
+  int d;          /* head dimension */
+  int chunk;      /* C, tokens per chunk */
+  int topk;       /* k, chunks selected per query */
+  int M;          /* adjacent queries per group for the chunk union */
+  float scale;    /* softmax scale of token and landmark logits (1/sqrt(d)) */
+  int dtype;      /* hils_dtype of q, k, v, lmk_k and out */
+  int debug_checks; /* 0 or 1, see above */
+} hils_params;
+
+#define HILS_OP_PREFILL 0
+#define HILS_OP_DECODE 1
+
+/* Bytes of device workspace `op` needs for these params (0 is possible).
+ * Returns 0 for invalid params as well; the calls themselves validate. */
+size_t hils_workspace_size(const hils_params *p, int op);
+
+/*
+ * Landmark scoring, inter-chunk softmax normaliser and top-k selection
+ * (model card, "What HiLS-Attention is"; molayo1419.me, "Core idea", step 1).
+ *   q       [B,Hq,L,d]          in
+ *   lmk_k   [B,Hkv,L/C,d]       in
+ *   sel_idx [B,Hq,L,topk] int32 out: selected chunk ids, ascending, -1 pad
+ *   chunk_w [B,Hq,L,topk] fp32  out: their landmark logits
+ *                                    scale*<q_t, lmk_c>, -inf pad
+ *   lse_lmk [B,Hq,L] fp32       out, may be NULL: log-sum-exp of the logits of
+ *                                    all completed chunks (-inf if none); the
+ *                                    inter-chunk softmax is exp(chunk_w - lse_lmk)
+ */
+hils_status hils_select(const hils_params *p, const void *q, const void *lmk_k,
+                        int32_t *sel_idx, float *chunk_w, float *lse_lmk,
+                        void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Chunk union per group of M adjacent queries (molayo1419.me, "Hardware-
+ * efficient kernel"): for group g = [g*M, (g+1)*M) of head (b, hq), the
+ * ascending set of all chunk ids selected by its rows plus each row's own
+ * chunk, in CSR form.  Groups are ordered (b, hq, g); G = B*Hq*ceil(L/M).
+ *   sel_idx [B,Hq,L,topk] int32 in (as written by hils_select)
+ *   u_off   [G+1] int32         out: u_off[0] = 0, u_off[G] = total
+ *   u_idx   [u_cap] int32       out: concatenated sets
+ *   u_cap   capacity of u_idx; must be >= hils_union_capacity(p)
+ * hils_attn_fwd does not need this output: it builds each tile's union
+ * internally.  This call materialises it (union-size statistics, checks).
+ */
+int64_t hils_union_capacity(const hils_params *p);
+hils_status hils_union(const hils_params *p, const int32_t *sel_idx, int32_t *u_off,
+                       int32_t *u_idx, int64_t u_cap, void *ws, size_t ws_bytes,
+                       void *stream);
+
+/*
+ * Intra-chunk attention over the selected chunks and the own chunk, and
+ * score-weighted fusion (molayo1419.me, "Core idea", step 2; aiweekly.co,
+ * mechanism paragraph).
+ *   q, k, v  in (see layout)
+ *   sel_idx, chunk_w  in: a selection as written by hils_select (ascending
+ *            ids, -1 pad; logits of the selected chunks)
+ *   out      [B,Hq,L,d] dtype out
+ *   lse      [B,Hq,L] fp32 out: log-sum-exp of the fused chunk logits
+ *   w_final  [B,Hq,L,topk+1] fp32 out, may be NULL: fusion weights of the
+ *            selected chunks in sel_idx order (0 for padding), own chunk last
+ */
+hils_status hils_attn_fwd(const hils_params *p, const void *q, const void *k, const void *v,
+                          const int32_t *sel_idx, const float *chunk_w, void *out,
+                          float *lse, float *w_final, void *ws, size_t ws_bytes,
+                          void *stream);
+
+/* hils_select followed by hils_attn_fwd on the same stream. */
+hils_status hils_prefill(const hils_params *p, const void *q, const void *k, const void *v,
+                         const void *lmk_k, int32_t *sel_idx, float *chunk_w, float *lse_lmk,
+                         void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * One decode step for B sequences (prefill of a single row t = N-1 per head,
+ * with the KV cache already holding the new token).
+ *   q        [B,Hq,d]          in
+ *   k_cache, v_cache [B,Hkv,N,d] in (N = p->L)
+ *   lmk_k    [B,Hkv,N/C,d]     in
+ *   sel_idx  [B,Hq,topk] int32 out, chunk_w [B,Hq,topk] fp32 out,
+ *   lse_lmk  [B,Hq] fp32 out (may be NULL), out [B,Hq,d] dtype out,
+ *   lse      [B,Hq] fp32 out
+ * Needs hils_workspace_size(p, HILS_OP_DECODE) bytes of workspace.
+ */
+hils_status hils_decode_fwd(const hils_params *p, const void *q, const void *k_cache,
+                            const void *v_cache, const void *lmk_k, int32_t *sel_idx,
+                            float *chunk_w, float *lse_lmk, void *out, float *lse, void *ws,
+                            size_t ws_bytes, void *stream);
+
+/* Static description of a status code. */
+const char *hils_status_string(hils_status s);
+
+/* Human-readable detail of the last failure on the calling thread ("" if none). */
+const char *hils_last_error(void);
+
+/* Number of kernels this library has launched in this process so far. */
+int64_t hils_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HILS_H_ */

@@ -58,14 +58,13 @@ def build(force: bool = False) -> str:
 def _bind(path):
     lib = ctypes.CDLL(path)
     P, I, I64, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
-    lib.hils_oracle_rows.argtypes = [I, I, I, I, I, I, I, D, I, P, P, P, P, I64, P, I, P, P,
+    lib.hils_oracle_rows.argtypes = [I, I, I, I, I, I, I, D, I, I, P, P, P, P, I64, P, I, P, P,
                                      P, P, P, P, P, P, I]
     lib.hils_oracle_rows.restype = I
-    lib.hils_oracle_decode.argtypes = [I, I, I, I, I, I, I, D, I, P, P, P, P, I64, P, P, P, P,
-                                       P, P, P, I]
-    lib.hils_oracle_decode.restype = I
     lib.hils_oracle_union.argtypes = [I, I, I, I, I64, I64, P, P, I64]
     lib.hils_oracle_union.restype = I64
+    lib.hils_oracle_scores.argtypes = [I, I, I, I, I, I, D, I, I, P, P, I64, P, P, I, I]
+    lib.hils_oracle_scores.restype = I
     return lib
 
 
@@ -138,8 +137,9 @@ class Oracle:
         self.lib = _bind(lib_path or build())
 
     def rows(self, p: Problem, q, k, v, lmk, rows, mode: str = "landmark", sel_in=None,
-             w_in=None, nthreads: int = 0) -> dict:
-        """Prefill rows (flat indices (b*Hq + hq)*L + t).
+             w_in=None, nthreads: int = 0, decode: bool = False) -> dict:
+        """Prefill rows (flat indices (b*Hq + hq)*L + t), or with decode=True
+        decode heads (flat b*Hq + hq, q [B,Hq,d], position t = L-1).
 
         Returns numpy arrays: sel [n,k] int32 (ascending, -1 pad), w [n,k]
         (selected logits, -inf pad), lse_lmk [n], out [n,d], lse [n],
@@ -153,7 +153,7 @@ class Oracle:
             si = np.ascontiguousarray(np.asarray(sel_in, dtype=np.int32).reshape(n, p.topk))
             wi = np.ascontiguousarray(np.asarray(w_in, dtype=np.float64).reshape(n, p.topk))
         rc = self.lib.hils_oracle_rows(
-            p.B, p.Hq, p.Hkv, p.L, p.d, p.C, p.topk, p.scale, int(bf16), _ptr(qa), _ptr(ka),
+            p.B, p.Hq, p.Hkv, p.L, p.d, p.C, p.topk, p.scale, int(bf16), int(decode), _ptr(qa), _ptr(ka),
             _ptr(va), _ptr(la), n, _ptr(r), MODES[mode], _ptr(si), _ptr(wi), _ptr(res["sel"]),
             _ptr(res["w"]), _ptr(res["lse_lmk"]), _ptr(res["out"]), _ptr(res["lse"]),
             _ptr(res["wfin"]), int(nthreads))
@@ -164,19 +164,26 @@ class Oracle:
     def decode(self, p: Problem, q, k, v, lmk, heads=None, nthreads: int = 0) -> dict:
         """Decode step: q is [B,Hq,d], the cache length is p.L and the query
         position is p.L - 1.  heads: flat b*Hq + hq (default: all)."""
-        (qa, ka, va, la), bf16 = _inputs(q, k, v, lmk)
         h = np.arange(p.B * p.Hq, dtype=np.int64) if heads is None else heads
-        h = np.ascontiguousarray(np.asarray(h, dtype=np.int64).reshape(-1))
-        n = h.shape[0]
-        res = _outputs(n, p)
-        rc = self.lib.hils_oracle_decode(
-            p.B, p.Hq, p.Hkv, p.L, p.d, p.C, p.topk, p.scale, int(bf16), _ptr(qa), _ptr(ka),
-            _ptr(va), _ptr(la), n, _ptr(h), _ptr(res["sel"]), _ptr(res["w"]),
-            _ptr(res["lse_lmk"]), _ptr(res["out"]), _ptr(res["lse"]), _ptr(res["wfin"]),
-            int(nthreads))
+        return self.rows(p, q, k, v, lmk, h, nthreads=nthreads, decode=True)
+
+    def scores(self, p: Problem, q, lmk, rows, nthreads: int = 0,
+               decode: bool = False) -> np.ndarray:
+        """Landmark logits of every completed chunk for the rows (numbered as in
+        rows()): [n, L//C] fp64, -inf for chunks that are not completed."""
+        qa, bf16 = _as_array(q)
+        la, bf16_l = _as_array(lmk)
+        if bf16 != bf16_l:
+            raise TypeError("q and lmk must share one element format")
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
+        ncols = max(p.L // p.C, 1)
+        s = np.empty((r.shape[0], ncols), np.float64)
+        rc = self.lib.hils_oracle_scores(p.B, p.Hq, p.Hkv, p.L, p.d, p.C, p.scale, int(bf16),
+                                         int(decode), _ptr(qa), _ptr(la), r.shape[0], _ptr(r), _ptr(s), ncols,
+                                         int(nthreads))
         if rc != 0:
             raise ValueError("oracle rejected its arguments")
-        return res
+        return s[:, :p.L // p.C]
 
     def union(self, L: int, C: int, topk: int, M: int, head: int, g: int, sel) -> np.ndarray:
         """Sorted chunk union of query group g (rows [g*M, (g+1)*M)) of flat
@@ -211,3 +218,7 @@ def decode(*a, **kw):
 
 def union(*a, **kw):
     return default().union(*a, **kw)
+
+
+def scores(*a, **kw):
+    return default().scores(*a, **kw)

@@ -227,16 +227,36 @@ static void load_q(const problem *P, const void *q, int q_is_decode, int b, int 
   for (int i = 0; i < P->d; ++i) qt[i] = ld(q, row * (int64_t)P->d + i, P->bf16);
 }
 
+/* Decode a flat row index.  Prefill (q_decode = 0): rows are
+ * (b*Hq + hq)*L + t and q is [B,Hq,L,d].  Decode (q_decode = 1): rows are
+ * heads b*Hq + hq, q is [B,Hq,d], and the query sits at position t = L-1 of a
+ * cache of length L that already holds the new token. */
+static int row_of(const problem *P, int q_decode, int64_t flat, int *b, int *hq, int *t) {
+  if (q_decode) {
+    if (flat < 0 || flat >= (int64_t)P->B * P->Hq) return 0;
+    *hq = (int)(flat % P->Hq);
+    *b = (int)(flat / P->Hq);
+    *t = P->L - 1;
+  } else {
+    if (flat < 0 || flat >= (int64_t)P->B * P->Hq * P->L) return 0;
+    *t = (int)(flat % P->L);
+    *hq = (int)((flat / P->L) % P->Hq);
+    *b = (int)(flat / ((int64_t)P->L * P->Hq));
+  }
+  return 1;
+}
+
 /*
- * Prefill rows.  rows[r] is a flat query index (b*Hq + hq)*L + t.  Every
- * output pointer may be NULL; the per-row outputs are packed in the order of
- * rows[].  Returns 0, or -1 on an invalid argument.
+ * Rows of the forward pass (see row_of for the row numbering).  Every output
+ * pointer may be NULL; per-row outputs are packed in the order of rows[].
+ * Returns 0, or -1 on an invalid argument.
  */
 int hils_oracle_rows(int B, int Hq, int Hkv, int L, int d, int C, int topk, double scale,
-                     int bf16, const void *q, const void *k, const void *v, const void *lmk,
-                     int64_t nrows, const int64_t *rows, int mode, const int32_t *sel_in,
-                     const double *w_in, int32_t *sel_out, double *w_out, double *lse_lmk_out,
-                     double *out, double *lse_out, double *wfin_out, int nthreads) {
+                     int bf16, int q_decode, const void *q, const void *k, const void *v,
+                     const void *lmk, int64_t nrows, const int64_t *rows, int mode,
+                     const int32_t *sel_in, const double *w_in, int32_t *sel_out, double *w_out,
+                     double *lse_lmk_out, double *out, double *lse_out, double *wfin_out,
+                     int nthreads) {
   if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || L < 1 || d < 1 || C < 1 || topk < 1)
     return -1;
   if (mode == MODE_GIVEN && (!sel_in || !w_in)) return -1;
@@ -249,54 +269,15 @@ int hils_oracle_rows(int B, int Hq, int Hkv, int L, int d, int C, int topk, doub
   int bad = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
   for (int64_t r = 0; r < nrows; ++r) {
-    const int64_t flat = rows[r];
-    if (flat < 0 || flat >= (int64_t)B * Hq * L) { bad = 1; continue; }
-    const int t = (int)(flat % L);
-    const int hq = (int)((flat / L) % Hq);
-    const int b = (int)(flat / ((int64_t)L * Hq));
+    int b, hq, t;
+    if (!row_of(&P, q_decode, rows[r], &b, &hq, &t)) { bad = 1; continue; }
     double *qt = (double *)malloc(sizeof(double) * (size_t)d);
-    load_q(&P, q, 0, b, hq, t, qt);
+    load_q(&P, q, q_decode, b, hq, t, qt);
     ref_row(&P, qt, b, hq, t, mode, sel_in ? sel_in + r * topk : NULL,
             w_in ? w_in + r * topk : NULL, sel_out ? sel_out + r * topk : NULL,
             w_out ? w_out + r * topk : NULL, lse_lmk_out ? lse_lmk_out + r : NULL,
             out ? out + r * d : NULL, lse_out ? lse_out + r : NULL,
             wfin_out ? wfin_out + r * (topk + 1) : NULL);
-    free(qt);
-  }
-  return bad ? -1 : 0;
-}
-
-/*
- * Decode: one new query per (b, hq), q laid out [B,Hq,d]; the cache of length
- * N = L already holds the new token, so the query position is t = N-1.
- * Rows are the B*Hq heads in order; nheads selects the first nheads of them
- * through heads[] (flat b*Hq + hq).
- */
-int hils_oracle_decode(int B, int Hq, int Hkv, int N, int d, int C, int topk, double scale,
-                       int bf16, const void *q, const void *k, const void *v, const void *lmk,
-                       int64_t nheads, const int64_t *heads, int32_t *sel_out, double *w_out,
-                       double *lse_lmk_out, double *out, double *lse_out, double *wfin_out,
-                       int nthreads) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || N < 1 || d < 1 || C < 1 || topk < 1)
-    return -1;
-  problem P = {B, Hq, Hkv, N, d, C, topk, scale, bf16, k, v, lmk};
-#ifdef _OPENMP
-  if (nthreads > 0) omp_set_num_threads(nthreads);
-#else
-  (void)nthreads;
-#endif
-  int bad = 0;
-#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
-  for (int64_t r = 0; r < nheads; ++r) {
-    const int64_t flat = heads[r];
-    if (flat < 0 || flat >= (int64_t)B * Hq) { bad = 1; continue; }
-    const int hq = (int)(flat % Hq), b = (int)(flat / Hq);
-    double *qt = (double *)malloc(sizeof(double) * (size_t)d);
-    load_q(&P, q, 1, b, hq, N - 1, qt);
-    ref_row(&P, qt, b, hq, N - 1, MODE_LANDMARK, NULL, NULL,
-            sel_out ? sel_out + r * topk : NULL, w_out ? w_out + r * topk : NULL,
-            lse_lmk_out ? lse_lmk_out + r : NULL, out ? out + r * d : NULL,
-            lse_out ? lse_out + r : NULL, wfin_out ? wfin_out + r * (topk + 1) : NULL);
     free(qt);
   }
   return bad ? -1 : 0;
@@ -328,4 +309,38 @@ int64_t hils_oracle_union(int L, int C, int topk, int M, int64_t head, int64_t g
     }
   free(mark);
   return n <= cap ? n : -1;
+}
+
+/*
+ * Landmark logits of every completed chunk of each row [KR step 1]:
+ * s[r][c] = scale * <q_t, lmk_c> for c < floor(t/C); entries c >= floor(t/C)
+ * are set to -inf.  s is [nrows, ncols]; ncols must be >= floor(L/C).
+ * Row numbering as in hils_oracle_rows.  The tests use these logits to
+ * enumerate the selections admissible at a near-tie.
+ */
+int hils_oracle_scores(int B, int Hq, int Hkv, int L, int d, int C, double scale, int bf16,
+                       int q_decode, const void *q, const void *lmk, int64_t nrows,
+                       const int64_t *rows, double *s, int ncols, int nthreads) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || L < 1 || d < 1 || C < 1 || ncols < L / C)
+    return -1;
+  problem P = {B, Hq, Hkv, L, d, C, 1, scale, bf16, NULL, NULL, lmk};
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t r = 0; r < nrows; ++r) {
+    int b, hq, t;
+    if (!row_of(&P, q_decode, rows[r], &b, &hq, &t)) { bad = 1; continue; }
+    const int hkv = hq / (Hq / Hkv);
+    double *qt = (double *)malloc(sizeof(double) * (size_t)d);
+    load_q(&P, q, q_decode, b, hq, t, qt);
+    const int64_t lmk_head = ((int64_t)b * Hkv + hkv) * (L / C);
+    for (int c = 0; c < ncols; ++c)
+      s[r * ncols + c] = c < t / C ? scale * dot(qt, lmk, lmk_head + c, d, bf16) : -INFINITY;
+    free(qt);
+  }
+  return bad ? -1 : 0;
 }

@@ -127,6 +127,9 @@ def pin_landmark_logit_and_normaliser(orc):
     assert r["sel"][0].tolist() == g["expect_sel"], r["sel"]
     assert np.allclose(r["w"][0], g["expect_logits"], rtol=0, atol=1e-15), r["w"]
     assert abs(r["lse_lmk"][0] - g["expect_lse_lmk"]) < 1e-14, r["lse_lmk"]
+    s = orc.scores(p, q, lmk, [t])
+    assert s.shape == (1, L // C)
+    assert np.allclose(s[0, :2], g["expect_logits"], rtol=0, atol=1e-15) and s[0, 2] == -np.inf, s
 
 
 def pin_topk_planted_ties(orc):

@@ -1,0 +1,91 @@
+"""The C-ABI library loads, exports every symbol include/hils.h declares, and
+rejects bad arguments before launching anything (runs without a GPU: no call
+here reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from chunk_wise_hierarchical_landmark_b200 import binding as hb
+from chunk_wise_hierarchical_landmark_b200 import build as hbuild
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "hils.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    hbuild.build()
+    return hb.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hils_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in hils.h but not exported"
+    assert set(hb.EXPORTS) <= set(names)
+
+
+def _params(**kw):
+    base = dict(B=1, Hq=4, Hkv=2, L=1024, d=128, topk=8, M=64)
+    base.update(kw)
+    return hb.make_params(**base)
+
+
+FAKE = ctypes.c_void_p(1 << 20)       # aligned, never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p((1 << 20) + 4)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), 2), (dict(topk=65), 2), (dict(topk=0), 1), (dict(Hq=3, Hkv=2), 1),
+    (dict(M=48), 2), (dict(L=0), 1), (dict(L=(1 << 24) + 1), 2), (dict(chunk=32), 2),
+])
+def test_bad_params_rejected(lib, kw, status):
+    p = _params(**kw)
+    rc = lib.hils_select(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, None, 0, None)
+    assert rc == status, hb.lib().hils_last_error()
+    assert lib.hils_last_error().decode()
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    p = _params()
+    assert lib.hils_select(None, FAKE, FAKE, FAKE, FAKE, None, None, 0, None) == 1
+    assert lib.hils_select(ctypes.byref(p), None, FAKE, FAKE, FAKE, None, None, 0, None) == 1
+    assert lib.hils_select(ctypes.byref(p), MISALIGNED, FAKE, FAKE, FAKE, None, None, 0, None) == 1
+    assert b"aligned" in lib.hils_last_error()
+    assert lib.hils_attn_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None,
+                             None, 0, None) == 1
+    assert lib.hils_decode_fwd(ctypes.byref(p), FAKE, FAKE, None, FAKE, FAKE, FAKE, None, FAKE,
+                               FAKE, None, 0, None) == 1
+
+
+def test_debug_mode_needs_workspace(lib):
+    p = _params(debug_checks=True)
+    assert lib.hils_workspace_size(ctypes.byref(p), hb.HILS_OP_PREFILL) >= 4
+    rc = lib.hils_attn_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None,
+                           0, None)
+    assert rc == 3
+
+
+def test_workspace_and_capacity(lib):
+    p = _params()
+    assert lib.hils_workspace_size(ctypes.byref(p), hb.HILS_OP_PREFILL) == 0
+    assert lib.hils_workspace_size(ctypes.byref(p), 7) == 0
+    cap = lib.hils_union_capacity(ctypes.byref(p))
+    assert cap == 1 * 4 * (1024 // 64) * min(16, 64 * 8 + 1 + 2)
+    bad = _params(d=96)
+    assert lib.hils_union_capacity(ctypes.byref(bad)) == -1
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.hils_status_string(s)
+    assert lib.hils_status_string(0) == b"ok"
+    assert lib.hils_launch_count() >= 0
