@@ -1,0 +1,500 @@
+// Intra-chunk attention + score-weighted fusion on the 5th-generation tensor
+// cores (tcgen05, accumulators in tensor memory, operands staged by TMA).
+//
+// Method (molayo1419.me, "Core idea" step 2 and "Hardware-efficient kernel";
+// aiweekly.co mechanism paragraph): each query attends, with an ordinary
+// softmax, to each of its selected chunks and to its own chunk (causally);
+// the per-chunk outputs are fused with weights softmax(chunk logits), the
+// own chunk's logit being the log-sum-exp of its causal token logits.  A tile
+// of 128 adjacent queries of one head loads the union of their chunks once.
+//
+// One CTA = one tile of 128 query rows (positions [t0, t0+128) of one
+// (b, hq)); 6 warps:
+//   warp 0     TMA producer: Q tile once, then K_c / V_c of every union chunk
+//              into an NS-stage ring;
+//   warp 1     TMEM owner and MMA issuer (one thread): S = Q K_c^T into one of
+//              two TMEM buffers, then O += P_c V_c into the TMEM accumulator;
+//   warps 2-5  one thread per row (TMEM lane): chunk softmax, P -> shared
+//              memory (bf16, 128B-swizzled K-major), epilogue.
+// Processing order: the tile's own chunks first (later one first), then the
+// rest of the union ascending.  After its own chunk a row knows its largest
+// fusion logit M = max(lse_own, max selected logit), so every chunk's
+// probabilities are written directly against M:
+//   P_j = exp(x_j - m_c) / l_c * exp(s_c - M)       (selected chunk c)
+//   P_j = exp(x_j - M)                               (own chunk)
+// and O = sum_c P_c V_c needs no rescaling.  P is rounded to bf16 for the
+// tensor core; the output is normalised by the sum of the ROUNDED
+// probabilities, which the tensor core accumulates alongside O (P times an
+// all-ones 64x16 tile into a 16-column TMEM sum), so the weights applied to V
+// sum to one exactly: out = O / sum_j bf16(P_j).  lse stays the fp32 value
+// M + log(sum_c exp(s_c - M)).
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace hils {
+namespace {
+
+using namespace sm100;
+
+constexpr int kRows = 128;   // query rows per tile (UMMA M)
+constexpr int kChunk = 64;   // keys per chunk (UMMA N of QK^T, K of PV)
+constexpr int kStages = 3;   // K/V ring depth
+constexpr int kThreads = 192;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D>
+struct Layout {
+  static constexpr int kQBytes = kRows * D * 2;
+  static constexpr int kKVBytes = kChunk * D * 2;  // one of K or V for one chunk
+  static constexpr int kPBytes = kRows * kChunk * 2;
+  static constexpr int q = 0;
+  static constexpr int k0 = q + kQBytes;
+  static constexpr int v0 = k0 + kStages * kKVBytes;
+  static constexpr int p0 = v0 + kStages * kKVBytes;
+  static constexpr int ones = p0 + 2 * kPBytes;   // 16 x 64 bf16 ones (B of the row-sum MMA)
+  static constexpr int bars = ones + 16 * 128;
+  static constexpr int misc = bars + 32 * 8;
+  static constexpr int bitmap = misc + 64;
+  static constexpr int fixed = bitmap;  // + bitmap words
+  // TMEM columns: S0 [0,64), S1 [64,128), O [128,128+D), row sums [128+D, 144+D)
+  static constexpr uint32_t kSumCol = 128 + D;
+  static constexpr uint32_t kTmemCols = (kSumCol + 16 <= 256) ? 256 : 512;
+};
+
+struct Bars {
+  uint64_t q, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], p_full[2],
+      p_empty[2], o_full, done;
+};
+
+struct ChunkIter {
+  const uint32_t *bm;
+  int wi;
+  uint32_t word;
+  int n_own, own_next;  // own chunks: c0 + n_own - 1 down to c0
+  __device__ void init(const uint32_t *b, int c0, int nown) {
+    bm = b;
+    wi = 0;
+    word = b[0];
+    n_own = nown;
+    own_next = c0 + nown - 1;
+  }
+  __device__ int next() {
+    if (n_own > 0) {
+      --n_own;
+      return own_next--;
+    }
+    while (word == 0) word = bm[++wi];
+    const int c = wi * 32 + __ffs(word) - 1;
+    word &= word - 1;
+    return c;
+  }
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, RowSpec rs,
+                      const int32_t *__restrict__ sel, const float *__restrict__ chunk_w,
+                      __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out,
+                      float *__restrict__ wfin, uint32_t *__restrict__ err) {
+  using Lay = Layout<D>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte alignment for the 128B-swizzled tiles
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars *bars = reinterpret_cast<Bars *>(smem + Lay::bars);
+  uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(smem + Lay::misc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::misc + 4);
+  int *n_steps_slot = reinterpret_cast<int *>(smem + Lay::misc + 8);
+  uint32_t *bitmap = reinterpret_cast<uint32_t *>(smem + Lay::bitmap);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int b = bh / rs.Hq, hq = bh % rs.Hq, hkv = hq / (rs.Hq / rs.Hkv);
+  const int t0 = blockIdx.x * kRows;
+  const int L = rs.L, K = rs.topk;
+  const int nchunks = (L + kChunk - 1) / kChunk;
+  const int nwords = (nchunks + 31) / 32 + 1;  // +1: a zero guard word
+  const int c0 = t0 / kChunk;
+  const int n_own = (t0 + kChunk < L) ? 2 : 1;
+
+  // ---------------------------------------------------------------- setup
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->s_empty[i], kRows);
+      mbar_init(&bars->p_full[i], kRows);
+      mbar_init(&bars->p_empty[i], 1);
+    }
+    mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_slot, Lay::kTmemCols);
+    tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i < nwords; i += kThreads) bitmap[i] = 0;
+  for (int i = threadIdx.x; i < 16 * 128 / 4; i += kThreads)
+    reinterpret_cast<uint32_t *>(smem + Lay::ones)[i] = 0x3F803F80u;  // bf16 1.0 pairs
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_slot;
+
+  // ------------------------------------------------ per-row prologue (warps 2-5)
+  const bool is_row = warp >= 2;
+  const int r = 32 * (warp & 3) + lane;  // TMEM lane == tile row
+  const int t = t0 + r;
+  const bool valid = is_row && t < L;
+  const int own = t / kChunk;
+  const size_t row = (size_t)bh * L + t;
+  const int32_t *mysel = sel + row * K;
+  const float *myw = chunk_w + row * K;
+  int nsel = 0, walk_n = 0;
+  float wmax2 = -INFINITY, sumsel = 0.0f, w_c0 = 0.0f;
+  bool has_c0 = false;
+  if (valid) {
+    for (int i = 0; i < K; ++i) {
+      const int c = __ldg(mysel + i);
+      if (c < 0) break;
+      if (c >= own) { report(err, DEV_BAD_INDEX); break; }
+      atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+      wmax2 = fmaxf(wmax2, __ldg(myw + i) * kLog2e);
+      ++nsel;
+    }
+    for (int i = 0; i < nsel; ++i) sumsel += exp2f(__ldg(myw + i) * kLog2e - wmax2);
+    walk_n = nsel;
+    if (own == c0 + 1 && nsel > 0 && __ldg(mysel + nsel - 1) == c0) {
+      has_c0 = true;
+      w_c0 = __ldg(myw + nsel - 1) * kLog2e;
+      walk_n = nsel - 1;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // own chunks are processed first; take them out of the ascending walk
+    if (lane == 0) {
+      bitmap[c0 >> 5] &= ~(1u << (c0 & 31));
+      if (c0 + 1 < nchunks) bitmap[(c0 + 1) >> 5] &= ~(1u << ((c0 + 1) & 31));
+    }
+    __syncwarp();
+    int cnt = 0;
+    for (int i = lane; i < nwords; i += 32) cnt += __popc(bitmap[i]);
+    for (int o = 16; o; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    if (lane == 0) *n_steps_slot = n_own + cnt;
+  }
+  __syncthreads();
+  const int n_steps = *n_steps_slot;
+
+  const uint32_t s_tmem[2] = {tmem, tmem + 64};
+  const uint32_t o_tmem = tmem + 128;
+  const uint32_t sum_tmem = tmem + Lay::kSumCol;
+  unsigned char *q_s = smem + Lay::q;
+  const int kv_row0 = (b * rs.Hkv + hkv) * L;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_expect_tx(&bars->q, Lay::kQBytes);
+      for (int kb = 0; kb < D / 64; ++kb)
+        tma_load_2d(q_s + kb * kRows * 128, &tm_q, &bars->q, kb * 64, bh * L + t0);
+      ChunkIter it;
+      it.init(bitmap, c0, n_own);
+      int issued = 0;
+      for (int i = 0; i < n_steps; ++i) {
+        const int c = it.next();
+        const int s = i % kStages;
+        if (i >= kStages && !mbar_wait(&bars->kv_empty[s], ((i / kStages) - 1) & 1, abort_flag))
+          break;
+        mbar_expect_tx(&bars->kv_full[s], 2 * Lay::kKVBytes);
+        unsigned char *ks = smem + Lay::k0 + s * Lay::kKVBytes;
+        unsigned char *vs = smem + Lay::v0 + s * Lay::kKVBytes;
+        for (int kb = 0; kb < D / 64; ++kb) {
+          tma_load_2d(ks + kb * kChunk * 128, &tm_k, &bars->kv_full[s], kb * 64, kv_row0 + c * kChunk);
+          tma_load_2d(vs + kb * kChunk * 128, &tm_v, &bars->kv_full[s], kb * 64, kv_row0 + c * kChunk);
+        }
+        ++issued;
+      }
+      // every load issued must land before the CTA may exit
+      for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+        mbar_wait_bounded(&bars->kv_full[i % kStages], (i / kStages) & 1);
+      mbar_wait_bounded(&bars->q, 0);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kRows, kChunk, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kRows, D, false, true);
+      constexpr uint32_t idesc_sum = idesc_bf16_f32(kRows, 16, false, false);
+      const uint32_t ones_addr = smem_u32(smem + Lay::ones);
+      const uint32_t q_addr = smem_u32(q_s);
+      auto pv = [&](int j) -> bool {
+        const int sb = j & 1, s = j % kStages;
+        if (!mbar_wait(&bars->p_full[sb], (j >> 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t p_addr = smem_u32(smem + Lay::p0 + sb * Lay::kPBytes);
+        const uint32_t v_addr = smem_u32(smem + Lay::v0 + s * Lay::kKVBytes);
+#pragma unroll
+        for (int kk = 0; kk < kChunk / 16; ++kk) {
+          // A = P [128 x 64] K-major: 16 keys = 32 bytes along the 128-byte row
+          const uint64_t a = smem_desc_sw128(p_addr + kk * 32, 16, 1024);
+          // B = V [64 keys x D] MN-major: 16 keys = 16 rows of 128 bytes;
+          // the D axis is split into 64-wide blocks 64*128 bytes apart
+          const uint64_t bdesc = smem_desc_sw128(v_addr + kk * 16 * 128, kChunk * 128, 1024);
+          mma_bf16_ss(o_tmem, a, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        // row sums of the rounded P: P [128 x 64] times ones [64 x 16]
+#pragma unroll
+        for (int kk = 0; kk < kChunk / 16; ++kk) {
+          const uint64_t a = smem_desc_sw128(p_addr + kk * 32, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(ones_addr + kk * 32, 16, 1024);
+          mma_bf16_ss(sum_tmem, a, bdesc, idesc_sum, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&bars->kv_empty[s]);
+        mma_commit(&bars->p_empty[sb]);
+        return true;
+      };
+      bool ok = mbar_wait(&bars->q, 0, abort_flag);
+      for (int i = 0; ok && i < n_steps; ++i) {
+        const int s = i % kStages, sb = i & 1;
+        if (!mbar_wait(&bars->kv_full[s], (i / kStages) & 1, abort_flag)) { ok = false; break; }
+        if (i >= 2 && !mbar_wait(&bars->s_empty[sb], ((i >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + Lay::k0 + s * Lay::kKVBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int kb = kk >> 2, kw = kk & 3;
+          const uint64_t a = smem_desc_sw128(q_addr + kb * kRows * 128 + kw * 32, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(k_addr + kb * kChunk * 128 + kw * 32, 16, 1024);
+          mma_bf16_ss(s_tmem[sb], a, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->s_full[sb]);
+        if (i >= 1 && !pv(i - 1)) { ok = false; break; }
+      }
+      if (ok) ok = pv(n_steps - 1);
+      if (ok) mma_commit(&bars->o_full);
+      // all issued tensor-core work must finish before TMEM is released
+      mma_commit(&bars->done);
+      mbar_wait_bounded(&bars->done, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax rows
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    unsigned char *p_row0 = smem + Lay::p0 + r * 128;
+    const float scale2 = rs.scale * kLog2e;
+    float M2 = 0.0f, lse2_own = 0.0f;
+    int ptr = 0;
+    int nc = (valid && walk_n > 0) ? __ldg(mysel) : -1;
+    float nw = (valid && walk_n > 0) ? __ldg(myw) * kLog2e : 0.0f;
+    ChunkIter it;
+    it.init(bitmap, c0, n_own);
+    bool ok = true;
+    for (int i = 0; i < n_steps; ++i) {
+      const int c = it.next();
+      const int sb = i & 1;
+      ok = mbar_wait(&bars->s_full[sb], (i >> 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      float x[64];
+      {
+        float (&x0)[32] = *reinterpret_cast<float (*)[32]>(&x[0]);
+        float (&x1)[32] = *reinterpret_cast<float (*)[32]>(&x[32]);
+        tmem_ld32(s_tmem[sb] + lane_off, x0);
+        tmem_ld32(s_tmem[sb] + lane_off + 32, x1);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->s_empty[sb]);
+
+      // does this row attend chunk c, and with which logit?
+      int kind = 0;  // 0 none, 1 own, 2 selected
+      float logit2 = 0.0f;
+      if (valid) {
+        if (c == own) {
+          kind = 1;
+        } else if (c == c0 && has_c0) {
+          kind = 2;
+          logit2 = w_c0;
+        } else if (ptr < walk_n && c == nc) {
+          kind = 2;
+          logit2 = nw;
+          ++ptr;
+          if (ptr < walk_n) {
+            nc = __ldg(mysel + ptr);
+            nw = __ldg(myw + ptr) * kLog2e;
+          }
+        }
+      }
+      uint32_t pk[32];
+      if (kind != 0) {
+        const int jmax = (kind == 1) ? (t - c * kChunk) : (kChunk - 1);
+        float m = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          x[j] = (j <= jmax) ? x[j] * scale2 : -INFINITY;
+          m = fmaxf(m, x[j]);
+        }
+        float l = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          x[j] = exp2f(x[j] - m);
+          l += x[j];
+        }
+        float sc;
+        if (kind == 1) {
+          lse2_own = m + __log2f(l);
+          M2 = fmaxf(lse2_own, wmax2);
+          sc = exp2f(m - M2);
+        } else {
+          sc = exp2f(logit2 - M2) / l;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) pk[j] = pack_bf16(x[2 * j] * sc, x[2 * j + 1] * sc);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) pk[j] = 0u;
+      }
+      if (i >= 2) {
+        ok = mbar_wait(&bars->p_empty[sb], ((i >> 1) - 1) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      }
+      unsigned char *prow = p_row0 + sb * Lay::kPBytes;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint4 v4 = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        *reinterpret_cast<uint4 *>(prow + ((j ^ (r & 7)) << 4)) = v4;
+      }
+      fence_async_smem();
+      mbar_arrive(&bars->p_full[sb]);
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok) ok = mbar_wait(&bars->o_full, 0, abort_flag);
+    if (__all_sync(0xffffffffu, ok)) {
+      tc_fence_after();
+      const float lsum = exp2f(lse2_own - M2) + sumsel * exp2f(wmax2 - M2);
+      const float lsum_rounded = tmem_ld1(sum_tmem + lane_off);
+      tmem_wait_ld();
+      const float inv = 1.0f / lsum_rounded;
+      __nv_bfloat16 *orow = out + row * D;
+#pragma unroll
+      for (int cb = 0; cb < D / 32; ++cb) {
+        float o[32];
+        tmem_ld32(o_tmem + lane_off + cb * 32, o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 v4 = make_uint4(pack_bf16(o[8 * j] * inv, o[8 * j + 1] * inv),
+                                  pack_bf16(o[8 * j + 2] * inv, o[8 * j + 3] * inv),
+                                  pack_bf16(o[8 * j + 4] * inv, o[8 * j + 5] * inv),
+                                  pack_bf16(o[8 * j + 6] * inv, o[8 * j + 7] * inv));
+            *reinterpret_cast<uint4 *>(orow + cb * 32 + 8 * j) = v4;
+          }
+        }
+      }
+      if (valid) {
+        const float lse2 = M2 + __log2f(lsum);
+        lse_out[row] = lse2 * kLn2;
+        if (wfin) {
+          float *wr = wfin + row * (K + 1);
+          for (int i = 0; i < K; ++i)
+            wr[i] = i < nsel ? exp2f(__ldg(myw + i) * kLog2e - lse2) : 0.0f;
+          wr[K] = exp2f(lse2_own - lse2);
+        }
+        if (ptr != walk_n) report(err, DEV_BAD_INDEX);
+      }
+    }
+  }
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) report(err, DEV_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Lay::kTmemCols);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+}  // namespace
+
+// 2-D bf16 tensor map over a row-major [rows, cols] array with a
+// [box_rows, 64]-element box and 128-byte swizzle.
+cudaError_t make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                           uint32_t box_rows) {
+  static EncodeTiledFn encode = nullptr;
+  if (!encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+    encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+size_t attn_sm100_smem(int d, int L) {
+  const int nwords = ((L + 63) / 64 + 31) / 32 + 1;
+  const size_t fixed = d == 64 ? Layout<64>::fixed : Layout<128>::fixed;
+  return fixed + (size_t)nwords * 4 + 1024;
+}
+
+cudaError_t attn_sm100(const RowSpec &rs, const void *q, const void *k, const void *v,
+                       const int32_t *sel, const float *w, void *out, float *lse, float *wfin,
+                       uint32_t *err, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  cudaError_t e;
+  const uint64_t qrows = (uint64_t)rs.B * rs.Hq * rs.L, kvrows = (uint64_t)rs.B * rs.Hkv * rs.L;
+  if ((e = make_tmap_bf16(&tq, q, qrows, rs.d, kRows)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tk, k, kvrows, rs.d, kChunk)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16(&tv, v, kvrows, rs.d, kChunk)) != cudaSuccess) return e;
+  const size_t smem = attn_sm100_smem(rs.d, rs.L);
+  dim3 grid((rs.L + kRows - 1) / kRows, rs.B * rs.Hq);
+  if (rs.d == 64) {
+    auto kern = attn_sm100_kernel<64>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
+    kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, rs, sel, w, (__nv_bfloat16 *)out, lse, wfin, err);
+  } else {
+    auto kern = attn_sm100_kernel<128>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
+    kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, rs, sel, w, (__nv_bfloat16 *)out, lse, wfin, err);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace hils

@@ -54,6 +54,8 @@ hils_status check_params(const hils_params *p) {
   if (p->L > kMaxL) return fail(HILS_ERR_UNSUPPORTED, "L=%d above %d", p->L, kMaxL);
   if ((int64_t)p->B * p->Hq > (1 << 16) - 1)
     return fail(HILS_ERR_UNSUPPORTED, "B*Hq above 65535");
+  if ((int64_t)p->B * p->Hq * p->L >= (int64_t)1 << 31)
+    return fail(HILS_ERR_UNSUPPORTED, "B*Hq*L must be below 2^31");
   return HILS_OK;
 }
 
@@ -107,8 +109,12 @@ hils_status do_select(const hils_params *p, const hils::RowSpec &rs, const void 
 hils_status do_attn(const hils_params *p, const hils::RowSpec &rs, const void *q, const void *k,
                     const void *v, const int32_t *sel, const float *w, void *out, float *lse,
                     float *wfin, uint32_t *err, cudaStream_t st) {
-  cudaError_t e =
-      hils::attn_simt(rs, p->dtype == HILS_BF16, q, k, v, sel, w, out, lse, wfin, err, st);
+  // bf16 prefill runs on the tensor cores; fp32 (no exact tensor-core path)
+  // and the single decode row run on the CUDA cores
+  const bool tc = p->dtype == HILS_BF16 && rs.t_first == 0 && rs.t_count == rs.L;
+  cudaError_t e = tc ? hils::attn_sm100(rs, q, k, v, sel, w, out, lse, wfin, err, st)
+                     : hils::attn_simt(rs, p->dtype == HILS_BF16, q, k, v, sel, w, out, lse,
+                                       wfin, err, st);
   g_launches += 1;
   return e == cudaSuccess ? HILS_OK : cuda_fail(e, "attention launch");
 }

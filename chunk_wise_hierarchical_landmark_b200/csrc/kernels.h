@@ -25,6 +25,12 @@ cudaError_t attn_simt(const RowSpec &rs, bool bf16, const void *q, const void *k
                       uint32_t *err, cudaStream_t st);
 size_t simt_attn_smem(int d, int L, int C);
 
+// tcgen05 attention for bf16 prefill (attn_sm100.cu)
+cudaError_t attn_sm100(const RowSpec &rs, const void *q, const void *k, const void *v,
+                       const int32_t *sel, const float *w, void *out, float *lse, float *wfin,
+                       uint32_t *err, cudaStream_t st);
+size_t attn_sm100_smem(int d, int L);
+
 // Chunk union in CSR form (hils_union.cu)
 cudaError_t union_csr(int B, int Hq, int L, int C, int topk, int M, const int32_t *sel,
                       int32_t *u_off, int32_t *u_idx, int64_t u_cap, uint32_t *err,

@@ -20,7 +20,7 @@ class Workload:
     d: int
     C: int
     topk: int
-    M: int            # query-group size for the chunk union (prefill)
+    M: int            # query-group size for the chunk union (prefill only)
     dtype: str        # "f32" or "bf16"
     decode: bool = False
     q_kind: str = "iid"      # "iid" N(0,1) or "ar1" (stationary AR(1) walk)
@@ -51,7 +51,7 @@ PREFILL_128K = Workload("prefill_7b_gqa_bf16_L131072", B=1, Hq=32, Hkv=8, L=1310
                         C=64, topk=32, M=64, dtype="bf16", q_kind="ar1", q_sigma=0.05,
                         lmk_noise=0.5, seed=1002)
 DECODE_512K = Workload("decode_gqa_bf16_B16_N524288", B=16, Hq=32, Hkv=8, L=524288, d=128,
-                       C=64, topk=64, M=1, dtype="bf16", decode=True, lmk_noise=0.5, seed=1003)
+                       C=64, topk=64, M=64, dtype="bf16", decode=True, lmk_noise=0.5, seed=1003)
 PREFILL_512K = Workload("prefill_7b_gqa_bf16_L524288", B=1, Hq=32, Hkv=8, L=524288, d=128,
                         C=64, topk=64, M=128, dtype="bf16", q_kind="ar1", q_sigma=0.02,
                         needles=64, lmk_noise=0.5, seed=1004)

@@ -89,7 +89,7 @@ def compare_rows(p: oracle.Problem, inputs, rows, gpu: dict, ref: dict, dtype: s
                     exp_wfin[i] = r["wfin"][0]
     valid = gpu["sel"] >= 0
     assert (np.isneginf(gpu["w"]) == ~valid).all(), "chunk_w padding must be -inf"
-    dw = np.abs(np.where(valid, gpu["w"] - exp_w, 0.0))
+    dw = np.abs(np.where(valid, gpu["w"], 0.0) - np.where(valid, exp_w, 0.0))
     w_tol = tol["w"] * np.maximum(1.0, np.abs(np.where(valid, exp_w, 0.0)))
     assert (dw <= w_tol).all(), f"chunk_w error {dw.max():.3g}"
     out = gpu["out"].astype(np.float64)
