@@ -41,7 +41,8 @@ hils_status check_params(const hils_params *p) {
       p->topk < 1 || p->M < 1)
     return fail(HILS_ERR_INVALID_ARG, "shape fields must be >= 1");
   if (p->Hq % p->Hkv) return fail(HILS_ERR_INVALID_ARG, "Hq %% Hkv != 0");
-  if (!std::isfinite(p->scale)) return fail(HILS_ERR_INVALID_ARG, "scale is not finite");
+  if (!std::isfinite(p->scale) || !(p->scale > 0.0f))
+    return fail(HILS_ERR_INVALID_ARG, "scale must be finite and positive");
   if (p->dtype != HILS_F32 && p->dtype != HILS_BF16)
     return fail(HILS_ERR_INVALID_ARG, "unknown dtype %d", p->dtype);
   if (p->debug_checks != 0 && p->debug_checks != 1)
@@ -100,8 +101,12 @@ hils_status debug_end(uint32_t *err, cudaStream_t st) {
 }
 
 hils_status do_select(const hils_params *p, const hils::RowSpec &rs, const void *q,
-                      const void *lmk, int32_t *sel, float *w, float *lse_lmk, cudaStream_t st) {
-  cudaError_t e = hils::select_simt(rs, p->dtype == HILS_BF16, q, lmk, sel, w, lse_lmk, st);
+                      const void *lmk, int32_t *sel, float *w, float *lse_lmk, uint32_t *err,
+                      cudaStream_t st) {
+  // bf16 prefill scores on the tensor cores; fp32 and the decode row on the CUDA cores
+  const bool tc = p->dtype == HILS_BF16 && rs.t_first == 0 && rs.t_count == rs.L;
+  cudaError_t e = tc ? hils::select_sm100(rs, q, lmk, sel, w, lse_lmk, err, st)
+                     : hils::select_simt(rs, p->dtype == HILS_BF16, q, lmk, sel, w, lse_lmk, st);
   g_launches += 1;
   return e == cudaSuccess ? HILS_OK : cuda_fail(e, "select launch");
 }
@@ -137,10 +142,12 @@ HILS_API hils_status hils_select(const hils_params *p, const void *q, const void
   NEED(chunk_w);
   MAYBE(lse_lmk);
   if (p->L >= p->chunk) NEED(lmk_k);
-  (void)ws;
-  (void)ws_bytes;
-  return do_select(p, prefill_rows(p), q, lmk_k, sel_idx, chunk_w, lse_lmk,
-                   static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t *err = nullptr;
+  if ((s = debug_begin(p, ws, ws_bytes, &err, st)) != HILS_OK) return s;
+  if ((s = do_select(p, prefill_rows(p), q, lmk_k, sel_idx, chunk_w, lse_lmk, err, st)) != HILS_OK)
+    return s;
+  return debug_end(err, st);
 }
 
 HILS_API int64_t hils_union_capacity(const hils_params *p) {
@@ -222,7 +229,7 @@ HILS_API hils_status hils_decode_fwd(const hils_params *p, const void *q, const 
   uint32_t *err = nullptr;
   if ((s = debug_begin(p, ws, ws_bytes, &err, st)) != HILS_OK) return s;
   const hils::RowSpec rs = decode_rows(p);
-  if ((s = do_select(p, rs, q, lmk_k, sel_idx, chunk_w, lse_lmk, st)) != HILS_OK) return s;
+  if ((s = do_select(p, rs, q, lmk_k, sel_idx, chunk_w, lse_lmk, err, st)) != HILS_OK) return s;
   if ((s = do_attn(p, rs, q, k_cache, v_cache, sel_idx, chunk_w, out, lse, nullptr, err, st)) !=
       HILS_OK)
     return s;

@@ -31,6 +31,19 @@ cudaError_t attn_sm100(const RowSpec &rs, const void *q, const void *k, const vo
                        uint32_t *err, cudaStream_t st);
 size_t attn_sm100_smem(int d, int L);
 
+// tcgen05 landmark scoring + top-k for bf16 prefill (select_sm100.cu)
+cudaError_t select_sm100(const RowSpec &rs, const void *q, const void *lmk, int32_t *sel,
+                         float *w, float *lse_lmk, uint32_t *err, cudaStream_t st);
+
+}  // namespace hils
+
+#include <cuda.h>
+namespace hils {
+// 2-D bf16 TMA descriptor over a row-major [rows, cols] array: box
+// [box_rows x 64 elements], 128-byte swizzle (attn_sm100.cu)
+cudaError_t make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                           uint32_t box_rows);
+
 // Chunk union in CSR form (hils_union.cu)
 cudaError_t union_csr(int B, int Hq, int L, int C, int topk, int M, const int32_t *sel,
                       int32_t *u_off, int32_t *u_idx, int64_t u_cap, uint32_t *err,
