@@ -184,11 +184,18 @@ def dist_env():
 
 
 def max_over_ranks(x: float, ws: int) -> float:
+    """Largest value over all ranks (the slowest rank's time)."""
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_value(tokens_per_rank: int, ms_per_rank: float, ws: int) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * ws / (max_over_ranks(ms_per_rank, ws) * 1e-3)
 
 
 def barrier(ws):
@@ -494,7 +501,16 @@ def main():
     ap.add_argument("--extra", dest="extra", action="store_true", default=True)
     ap.add_argument("--no-extra", dest="extra", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--hq", type=int, default=None,
+                    help="override the query-head count (smaller cases for profiler captures)")
+    ap.add_argument("--hkv", type=int, default=None, help="override the KV-head count")
     args = ap.parse_args()
+    if args.hq or args.hkv:
+        base = W.BY_NAME[args.workload]
+        w = base.with_(Hq=args.hq or base.Hq, Hkv=args.hkv or base.Hkv)
+        w = w.with_(name=f"{base.name}_hq{w.Hq}_hkv{w.Hkv}")
+        W.BY_NAME[w.name] = w
+        args.workload = w.name
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -9,11 +9,14 @@
 //              row block's KV head into a 3-stage ring;
 //   warp 1     TMEM owner, MMA issuer: S = Q Lmk^T (128 x 128 fp32) into one of
 //              two TMEM buffers;
-//   warps 2-5  one thread per row: block-wise online log-sum-exp and a binary
-//              min-heap of the row's best k keys in shared memory.  A 32-wide
-//              block of candidates is skipped whole when its best score cannot
-//              enter the heap (chunks arrive in ascending order, so a later
-//              chunk never wins a tie).
+//   warps 2-5  one thread per row: block-wise online log-sum-exp (in base 2)
+//              and the row's best k keys in shared memory (8 groups of 8
+//              slots, group minima in registers).  Per 32-candidate block a
+//              row first tests the block maximum against its k-th best score;
+//              qualifying candidates are staged in shared memory and inserted
+//              one per lane per step, so the 32 rows of a warp insert together
+//              instead of one after another.  Chunks arrive in ascending
+//              order, so a later chunk never wins a tie.
 // The candidate scores never leave the chip.
 #include <cuda_bf16.h>
 
@@ -40,8 +43,9 @@ struct SelLayout {
   static constexpr int kLBytes = kTile * D * 2;
   static constexpr int q = 0;
   static constexpr int l0 = q + kQBytes;
-  static constexpr int heap = l0 + kStages * kLBytes;      // [kMaxK][128] uint64
-  static constexpr int bars = heap + kMaxK * kRows * 8;
+  static constexpr int heap = l0 + kStages * kLBytes;      // [kMaxK][128] uint64 slots
+  static constexpr int stage = heap + kMaxK * kRows * 8;   // [32][128] fp32 candidate staging
+  static constexpr int bars = stage + 32 * kRows * 4;
   static constexpr int misc = bars + 16 * 8;
   static constexpr int total = misc + 64;
   static constexpr uint32_t kTmemCols = 256;  // S0 [0,128), S1 [128,256)
@@ -51,45 +55,62 @@ struct SelBars {
   uint64_t q, l_full[kStages], l_empty[kStages], s_full[2], s_empty[2], done;
 };
 
-// Per-row top-k state: a binary min-heap of selection keys in shared memory
-// (entry i of the row at h[i * 128]); `thr` is the root's score once full.
-struct HeapState {
-  int cnt;
-  float thr;
+// Per-row top-k: kMaxK key slots in shared memory (slot i of the row at
+// h[i * 128]) in 8 groups of 8, each group's minimum (key and position) kept
+// in registers.  Replacing the overall minimum rescans one group (8
+// independent loads) instead of walking a heap.  Slots >= K count as +inf.
+struct TopK {
+  uint64_t gmin[8];
+  uint32_t gpos;  // 3 bits per group: position of the group's minimum
+  uint64_t mn;    // overall minimum (the entry a better key replaces)
+  int mg;         // its group
+  int cnt;        // filled slots
+  float thr;      // score of mn once all K slots are filled, -inf before
+
+  __device__ void rescan(const uint64_t *h, int g, int K) {
+    uint64_t m = ~0ull;
+    uint32_t pos = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int slot = g * 8 + i;
+      const uint64_t x = slot < K ? h[slot * kRows] : ~0ull;
+      if (x < m) { m = x; pos = i; }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (i == g) gmin[i] = m;
+    gpos = (gpos & ~(7u << (3 * g))) | (pos << (3 * g));
+  }
+  __device__ void overall() {
+    mn = gmin[0];
+    mg = 0;
+#pragma unroll
+    for (int i = 1; i < 8; ++i)
+      if (gmin[i] < mn) { mn = gmin[i]; mg = i; }
+    thr = key_score(mn);
+  }
+  // offer a candidate key (the caller filtered on thr); returns nothing
+  __device__ void offer(uint64_t *h, uint64_t key, int K) {
+    if (cnt < K) {
+      h[cnt * kRows] = key;
+      if (++cnt == K) {
+#pragma unroll
+        for (int g = 0; g < 8; ++g) rescan(h, g, K);
+        overall();
+      }
+    } else if (key > mn) {
+      const int slot = mg * 8 + ((gpos >> (3 * mg)) & 7u);
+      h[slot * kRows] = key;
+      rescan(h, mg, K);
+      overall();
+    }
+  }
 };
 
-// Insert `key` (the caller checked that it qualifies).  Kept out of line: it
-// runs for a small fraction of the candidates.
-__device__ __noinline__ HeapState heap_insert(uint64_t *h, HeapState st, int K, uint64_t key) {
-  if (st.cnt < K) {  // sift up from the end
-    int i = st.cnt;
-    while (i > 0) {
-      const int p = (i - 1) >> 1;
-      const uint64_t kp = h[p * kRows];
-      if (kp <= key) break;
-      h[i * kRows] = kp;
-      i = p;
-    }
-    h[i * kRows] = key;
-    ++st.cnt;
-  } else {  // replace the root and sift down
-    int i = 0;
-    while (true) {
-      int c = 2 * i + 1;
-      if (c >= K) break;
-      uint64_t kc = h[c * kRows];
-      if (c + 1 < K) {
-        const uint64_t kr = h[(c + 1) * kRows];
-        if (kr < kc) { kc = kr; ++c; }
-      }
-      if (key <= kc) break;
-      h[i * kRows] = kc;
-      i = c;
-    }
-    h[i * kRows] = key;
-  }
-  if (st.cnt == K) st.thr = key_score(h[0]);
-  return st;
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 template <int D>
@@ -197,11 +218,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool valid = t < L;
     const int n_c = valid ? min(t / C, nlmk) : 0;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    uint64_t *heap = reinterpret_cast<uint64_t *>(smem + Lay::heap) + r;
+    uint64_t *slots = reinterpret_cast<uint64_t *>(smem + Lay::heap) + r;
+    float *stage = reinterpret_cast<float *>(smem + Lay::stage) + r;
     const float c2 = rs.scale * kLog2e;
+    const float sc = rs.scale;
     const bool want_lse = lse_lmk != nullptr;
     float m2 = -INFINITY, l = 0.0f;
-    HeapState hs{0, -INFINITY};
+    TopK tk;
+    tk.cnt = 0;
+    tk.thr = -INFINITY;
+    tk.gpos = 0;
+    tk.mn = 0;
+    tk.mg = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) tk.gmin[i] = ~0ull;
     bool ok = true;
     for (int i = 0; i < n_ltiles; ++i) {
       const int sb = i & 1;
@@ -211,35 +241,57 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int blk = 0; blk < kTile / 32; ++blk) {
         float a[32];
-        __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the divergent heap work
+        __syncwarp();  // tcgen05.ld is warp-collective
         tmem_ld32(tmem + sb * kTile + blk * 32 + lane_off, a);
         tmem_wait_ld();
         const int cb = i * kTile + blk * 32;
-        if (cb >= n_c) continue;  // every candidate of this block is masked for this row
-        const int nv = min(32, n_c - cb);
+        const int nv = max(0, min(32, n_c - cb));
         if (nv < 32) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) a[j] = j < nv ? a[j] : -INFINITY;
         }
-        float bm = a[0];
+        // block maximum (tree)
+        float mx[16];
 #pragma unroll
-        for (int j = 1; j < 32; ++j) bm = fmaxf(bm, a[j]);
-        if (want_lse) {
+        for (int j = 0; j < 16; ++j) mx[j] = fmaxf(a[j], a[j + 16]);
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+          for (int j = 0; j < w; ++j) mx[j] = fmaxf(mx[j], mx[j + w]);
+        const float bm = mx[0];
+        if (want_lse && nv > 0) {
           const float bm2 = bm * c2;
           if (bm2 > m2) {
-            l *= exp2f(m2 - bm2);
+            l *= ex2_approx(m2 - bm2);
             m2 = bm2;
           }
-          float part = 0.0f;
+          float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-          for (int j = 0; j < 32; ++j) part += exp2f(fmaf(a[j], c2, -m2));
-          l += part;
+          for (int j = 0; j < 32; ++j) ps[j & 3] += ex2_approx(fmaf(a[j], c2, -m2));
+          l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         }
-        if (hs.cnt == K && bm * rs.scale <= hs.thr) continue;
+        // candidates that may enter the top-k (chunks arrive in ascending
+        // order, so an equal score never displaces a kept chunk)
+        uint32_t mask = 0;
+        if (nv > 0 && (tk.cnt < K || bm * sc > tk.thr)) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float s = a[j] * rs.scale;  // masked candidates are -inf and never qualify
-          if (j < nv && (hs.cnt < K || s > hs.thr)) hs = heap_insert(heap, hs, K, sel_key(s, cb + j));
+          for (int j = 0; j < 32; ++j)
+            mask |= (j < nv && (tk.cnt < K || a[j] * sc > tk.thr)) ? (1u << j) : 0u;
+        }
+        if (__any_sync(0xffffffffu, mask != 0)) {
+          if (mask) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) stage[j * kRows] = a[j];
+          }
+          // one candidate per lane per iteration: the lanes insert together
+          while (__any_sync(0xffffffffu, mask != 0)) {
+            if (mask) {
+              const int j = __ffs(mask) - 1;
+              mask &= mask - 1;
+              const float s = stage[j * kRows] * sc;
+              if (tk.cnt < K || s > tk.thr) tk.offer(slots, sel_key(s, cb + j), K);
+            }
+          }
         }
       }
       __syncwarp();
@@ -247,26 +299,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bars->s_empty[sb]);
     }
     if (__all_sync(0xffffffffu, ok) && valid) {
-      // ascending chunk order: insertion sort of the chunk ids in place
-      const int cnt = hs.cnt;
+      // ascending chunk order: insertion sort of the kept keys by chunk id
+      const int cnt = tk.cnt;
       for (int i = 1; i < cnt; ++i) {
-        const uint64_t x = heap[i * kRows];
+        const uint64_t x = slots[i * kRows];
         const int cx = key_chunk(x);
         int j = i - 1;
-        while (j >= 0 && key_chunk(heap[j * kRows]) > cx) {
-          heap[(j + 1) * kRows] = heap[j * kRows];
+        while (j >= 0 && key_chunk(slots[j * kRows]) > cx) {
+          slots[(j + 1) * kRows] = slots[j * kRows];
           --j;
         }
-        heap[(j + 1) * kRows] = x;
+        slots[(j + 1) * kRows] = x;
       }
       const size_t row = (size_t)bh * L + t;
       int32_t *srow = sel + row * K;
       float *wrow = chunk_w + row * K;
-      for (int i = 0; i < K; ++i) {
-        const bool have = i < cnt;
-        const uint64_t x = have ? heap[i * kRows] : 0;
-        srow[i] = have ? key_chunk(x) : -1;
-        wrow[i] = have ? key_score(x) : -INFINITY;
+      if ((K & 3) == 0) {
+        for (int i = 0; i < K; i += 4) {
+          int4 si;
+          float4 wi;
+          int *sp = &si.x;
+          float *wp = &wi.x;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const bool have = i + u < cnt;
+            const uint64_t x = have ? slots[(i + u) * kRows] : 0;
+            sp[u] = have ? key_chunk(x) : -1;
+            wp[u] = have ? key_score(x) : -INFINITY;
+          }
+          *reinterpret_cast<int4 *>(srow + i) = si;
+          *reinterpret_cast<float4 *>(wrow + i) = wi;
+        }
+      } else {
+        for (int i = 0; i < K; ++i) {
+          const bool have = i < cnt;
+          const uint64_t x = have ? slots[i * kRows] : 0;
+          srow[i] = have ? key_chunk(x) : -1;
+          wrow[i] = have ? key_score(x) : -INFINITY;
+        }
       }
       if (want_lse) lse_lmk[row] = n_c > 0 ? (m2 + __log2f(l)) * kLn2 : -INFINITY;
     }

@@ -38,36 +38,22 @@ def _randn(shape, g, device):
     return torch.randn(shape, generator=g, device=device, dtype=torch.float32)
 
 
-def _ar1(n_heads, L, d, sigma, g, device, block=64):
+def _ar1(n_heads, L, d, sigma, g, device):
     """Stationary AR(1) walk of length L for n_heads independent heads, [n, L, d] fp32.
 
-    Blocked evaluation of the linear recurrence: inside a block of `block`
-    steps the walk is a lower-triangular Toeplitz combination of the
-    innovations; the blocks are then chained through their carries."""
+    q_t = rho * q_{t-1} + sigma * eps_t with q_{-1} ~ N(0, 1), evaluated as a
+    log-depth scan of the linear recurrence (each doubling step adds the
+    contribution of the element 2^s positions back, weighted by rho^(2^s))."""
     rho = math.sqrt(1.0 - sigma * sigma)
-    out = torch.empty((n_heads, L, d), dtype=torch.float32, device=device)
-    T = block
-    i = torch.arange(T, device=device, dtype=torch.float64)
-    W = torch.where(i[:, None] >= i[None, :], rho ** (i[:, None] - i[None, :]),
-                    torch.zeros((), dtype=torch.float64, device=device)).float()
-    powers = (rho ** (i + 1)).float()  # rho^(i+1) for the carry term
-    for h in range(n_heads):
-        q0 = _randn((d,), g, device)
-        eps = _randn((L, d), g, device) * sigma
-        nb = (L + T - 1) // T
-        pad = nb * T - L
-        if pad:
-            eps = torch.cat([eps, torch.zeros((pad, d), device=device)], 0)
-        inner = torch.matmul(W, eps.view(nb, T, d))  # [nb, T, d]
-        carry = q0
-        qh = torch.empty((nb, T, d), dtype=torch.float32, device=device)
-        # chain the blocks: q[b, i] = inner[b, i] + rho^(i+1) * carry_{b-1}
-        # (the first block's carry is q_{-1} := q0, so q_0 = rho*q0 + sigma*eps_0)
-        for b in range(nb):
-            qh[b] = inner[b] + powers[:, None] * carry[None, :]
-            carry = qh[b, T - 1]
-        out[h] = qh.view(nb * T, d)[:L]
-    return out
+    q0 = _randn((n_heads, 1, d), g, device)
+    x = _randn((n_heads, L, d), g, device) * sigma
+    span = 1
+    while span < L:
+        x[:, span:] += (rho ** span) * x[:, :-span].clone()
+        span *= 2
+    t = torch.arange(1, L + 1, device=device, dtype=torch.float64)
+    x += (rho ** t).float()[None, :, None] * q0
+    return x
 
 
 def _finish(x, dtype):
@@ -115,8 +101,9 @@ def make_q(w: Workload, device="cpu", seed=None):
     q = torch.empty((B, H, L, d), dtype=dt, device=device)
     for b in range(B):
         if w.q_kind == "ar1":
-            for h in range(H):
-                q[b, h] = _finish(_ar1(1, L, d, w.q_sigma, g, device)[0], w.dtype)
+            for h0 in range(0, H, 8):
+                hs = min(8, H - h0)
+                q[b, h0:h0 + hs] = _finish(_ar1(hs, L, d, w.q_sigma, g, device), w.dtype)
         else:
             for h in range(H):
                 q[b, h] = _finish(_randn((L, d), g, device), w.dtype)
