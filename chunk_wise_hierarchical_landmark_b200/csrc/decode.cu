@@ -1,0 +1,646 @@
+// Decode step of HiLS attention (one new query per head, position t = N-1 of
+// a KV cache of length N that already holds the new token): landmark scoring,
+// inter-chunk normaliser and top-k (model card "HiLS-Attention", section
+// "What HiLS-Attention is"; molayo1419.me, "Core idea" step 1), then
+// attention inside the selected chunks and the own chunk fused by the chunk
+// logits (molayo1419.me step 2; aiweekly.co mechanism paragraph).
+//
+// The step is bound by HBM bytes: every landmark key of every (b, kv-head)
+// and the K/V of the chunks the G = Hq/Hkv query heads of a KV head attend.
+// All G heads of a KV head are served from one staged copy of each landmark
+// slab and of each chunk's K/V (bulk asynchronous copies into shared memory),
+// so the union of the heads' chunks crosses HBM once.
+//
+//   decode_score   grid (P, B*Hkv): slab p of 256 landmarks -> scores of the
+//                  G heads, per-head top-k of the slab (bitonic sort) and
+//                  per-head (max, sum of exp) of the slab
+//   decode_merge   grid (B*Hkv), one warp per head: k-way merge of the P
+//                  sorted slab lists -> sel_idx / chunk_w (ascending chunk
+//                  ids), lse_lmk; then the KV head's chunk union with a
+//                  per-entry head mask and per-head logits
+//   decode_attn    grid (Q, B*Hkv): up to 4 union chunks per CTA, each chunk's
+//                  K and V staged once; per head an online (max, sum, acc)
+//                  partial over its chunks
+//   decode_combine grid (B*Hq): partials -> out, lse
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace hils {
+namespace {
+
+using namespace sm100;
+
+constexpr int kSlab = 256;       // landmarks per scoring CTA
+constexpr int kChunksPerCta = 4; // union chunks per attention CTA
+constexpr int kMaxG = 8;         // query heads per KV head handled per CTA
+constexpr int kC = 64;
+
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
+                                         uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <typename T>
+__device__ __forceinline__ void load8(const T *p, float (&f)[8]);
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *p, float (&f)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4 *>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float *p, float (&f)[8]) {
+  const float4 a = reinterpret_cast<const float4 *>(p)[0];
+  const float4 b = reinterpret_cast<const float4 *>(p)[1];
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+// Bounded wait on a single-use barrier (phase 0); sets *abort on timeout.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort) {
+  return mbar_wait(bar, parity, abort);
+}
+
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(256) decode_score_kernel(DecodeSpec ds, const T *__restrict__ q,
+                                                           const T *__restrict__ lmk,
+                                                           uint64_t *__restrict__ part_keys,
+                                                           float2 *__restrict__ part_ml,
+                                                           uint32_t *__restrict__ err) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  T *slab = reinterpret_cast<T *>(smem);                          // [kSlab][D]
+  float *qs = reinterpret_cast<float *>(smem + kSlab * D * sizeof(T));  // [G][D]
+  uint64_t *keys = reinterpret_cast<uint64_t *>(qs + kMaxG * D);  // [G][kSlab]
+  float *red = reinterpret_cast<float *>(keys + kMaxG * kSlab);   // [8 warps][G]
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+
+  const int G = ds.Hq / ds.Hkv, K = ds.topk;
+  const int p = blockIdx.x, bk = blockIdx.y;  // bk = b*Hkv + hkv
+  const int b = bk / ds.Hkv, hkv = bk % ds.Hkv;
+  const int n_c = ds.n_c;
+  const int c0 = p * kSlab;
+  const int n = min(kSlab, n_c - c0);
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    const uint32_t bytes = (uint32_t)n * D * sizeof(T);
+    mbar_expect_tx(&bar, bytes);
+    const T *src = lmk + ((size_t)bk * ds.nlmk + c0) * D;
+    // bulk copies of at most 64 KB each
+    for (uint32_t off = 0; off < bytes; off += 65536u)
+      bulk_g2s(reinterpret_cast<unsigned char *>(slab) + off,
+               reinterpret_cast<const unsigned char *>(src) + off, min(65536u, bytes - off), &bar);
+  }
+  for (int i = tid; i < G * D; i += blockDim.x) {
+    const int g = i / D, e = i % D;
+    qs[i] = to_f(q[((size_t)b * ds.Hq + hkv * G + g) * D + e]) * ds.scale;
+  }
+  __syncthreads();
+  const bool ok = __syncthreads_and(wait_bar(&bar, 0, &abort_flag));
+  if (!ok && tid == 0) mbar_wait_bounded(&bar, 0);
+  float s[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) s[g] = -INFINITY;
+  if (ok && tid < n) {
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) s[g] = 0.0f;
+    const T *row = slab + tid * D;
+    for (int cc = 0; cc < D / 8; ++cc) {
+      const int c = (cc + tid) % (D / 8);  // rotated 16-byte column: spreads the banks
+      float f[8];
+      load8<T>(row + c * 8, f);
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g) {
+        if (g < G) {
+          const float4 qa = *reinterpret_cast<const float4 *>(qs + g * D + c * 8);
+          const float4 qb = *reinterpret_cast<const float4 *>(qs + g * D + c * 8 + 4);
+          float a = s[g];
+          a = fmaf(f[0], qa.x, a); a = fmaf(f[1], qa.y, a); a = fmaf(f[2], qa.z, a);
+          a = fmaf(f[3], qa.w, a); a = fmaf(f[4], qb.x, a); a = fmaf(f[5], qb.y, a);
+          a = fmaf(f[6], qb.z, a); a = fmaf(f[7], qb.w, a);
+          s[g] = a;
+        }
+      }
+    }
+  }
+  // keys for the per-head sort; slots without a candidate get key 0 (never kept)
+  for (int g = 0; g < G; ++g) keys[g * kSlab + tid] = (tid < n && ok) ? sel_key(s[g], c0 + tid) : 0ull;
+  // per-head (max, sum exp) of the slab
+  const int lane = tid & 31, warp = tid >> 5;
+  for (int g = 0; g < G; ++g) {
+    float m = s[g];
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) red[warp * kMaxG + g] = m;
+  }
+  __syncthreads();
+  float mh[kMaxG];
+  for (int g = 0; g < G; ++g) {
+    float m = -INFINITY;
+    for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w * kMaxG + g]);
+    mh[g] = m;
+  }
+  __syncthreads();
+  for (int g = 0; g < G; ++g) {
+    float e = (tid < n && ok) ? __expf(s[g] - mh[g]) : 0.0f;
+    for (int o = 16; o; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+    if (lane == 0) red[warp * kMaxG + g] = e;
+  }
+  __syncthreads();
+  if (tid < G) {
+    float l = 0.0f;
+    for (int w = 0; w < 8; ++w) l += red[w * kMaxG + tid];
+    part_ml[((size_t)bk * ds.P + p) * G + tid] = make_float2(mh[tid], l);
+  }
+  // bitonic sort of each head's 256 keys, descending
+  for (int size = 2; size <= kSlab; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      __syncthreads();
+      for (int pr = tid; pr < G * (kSlab / 2); pr += blockDim.x) {
+        const int g = pr / (kSlab / 2), i0 = pr % (kSlab / 2);
+        const int lo = 2 * i0 - (i0 & (stride - 1));
+        const int hi = lo + stride;
+        const bool desc = (lo & size) == 0;
+        uint64_t *kk = keys + g * kSlab;
+        const uint64_t a = kk[lo], c = kk[hi];
+        if ((a < c) == desc) {
+          kk[lo] = c;
+          kk[hi] = a;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < G * K; i += blockDim.x) {
+    const int g = i / K, j = i % K;
+    part_keys[(((size_t)bk * ds.P + p) * G + g) * K + j] = j < kSlab ? keys[g * kSlab + j] : 0ull;
+  }
+  if (tid == 0 && abort_flag) report(err, DEV_TIMEOUT);
+}
+
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) decode_merge_kernel(DecodeSpec ds,
+                                                           const uint64_t *__restrict__ part_keys,
+                                                           const float2 *__restrict__ part_ml,
+                                                           int32_t *__restrict__ sel,
+                                                           float *__restrict__ chunk_w,
+                                                           float *__restrict__ lse_lmk,
+                                                           int32_t *__restrict__ u_c,
+                                                           uint32_t *__restrict__ u_mask,
+                                                           float *__restrict__ u_logit,
+                                                           int32_t *__restrict__ u_count) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int G = ds.Hq / ds.Hkv, K = ds.topk, P = ds.P;
+  uint64_t *chosen = reinterpret_cast<uint64_t *>(smem);          // [G][K]
+  uint32_t *bitmap = reinterpret_cast<uint32_t *>(chosen + G * K);  // [nwords]
+  int *prefix = reinterpret_cast<int *>(bitmap + ds.nwords);       // [nwords]
+  int *cursor = prefix + ds.nwords;                                // [G][P]
+  __shared__ int total;
+  const int bk = blockIdx.x;
+  const int b = bk / ds.Hkv, hkv = bk % ds.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int own = ds.own;
+
+  for (int i = tid; i < ds.nwords; i += blockDim.x) bitmap[i] = 0;
+  for (int i = tid; i < G * P; i += blockDim.x) cursor[i] = 0;
+  __syncthreads();
+  // one warp per head: k-way merge of the P descending slab lists
+  for (int g = warp; g < G; g += blockDim.x / 32) {
+    const uint64_t *lists = part_keys + (size_t)bk * P * G * K;
+    // each lane walks the lists p = lane, lane+32, ...; its candidate is the
+    // best current head among them
+    int *cur = cursor + g * P;
+    int got = 0;
+    for (; got < K; ++got) {
+      uint64_t best = 0;
+      int bestp = -1;
+      for (int pl = lane; pl < P; pl += 32) {
+        if (cur[pl] < K) {
+          const uint64_t x = lists[((size_t)pl * G + g) * K + cur[pl]];
+          if (x > best) { best = x; bestp = pl; }
+        }
+      }
+      uint64_t wbest = best;
+      for (int o = 16; o; o >>= 1) {
+        const uint64_t y = __shfl_xor_sync(0xffffffffu, wbest, o);
+        wbest = y > wbest ? y : wbest;
+      }
+      if (wbest == 0) break;  // no candidate left
+      if (best == wbest && bestp >= 0) ++cur[bestp];  // keys are unique: one lane advances
+      if (lane == 0) chosen[g * K + got] = wbest;
+    }
+    __syncwarp();
+    // ascending chunk order (insertion sort by lane 0; K <= 64)
+    if (lane == 0) {
+      uint64_t *ch = chosen + g * K;
+      for (int i = 1; i < got; ++i) {
+        const uint64_t x = ch[i];
+        int j = i - 1;
+        while (j >= 0 && key_chunk(ch[j]) > key_chunk(x)) { ch[j + 1] = ch[j]; --j; }
+        ch[j + 1] = x;
+      }
+    }
+    __syncwarp();
+    const size_t hrow = (size_t)b * ds.Hq + hkv * G + g;
+    for (int i = lane; i < K; i += 32) {
+      const bool have = i < got;
+      const uint64_t x = have ? chosen[g * K + i] : 0;
+      sel[hrow * K + i] = have ? key_chunk(x) : -1;
+      chunk_w[hrow * K + i] = have ? key_score(x) : -INFINITY;
+      if (have) atomicOr(&bitmap[key_chunk(x) >> 5], 1u << (key_chunk(x) & 31));
+      if (!have) chosen[g * K + i] = 0;
+    }
+    if (lse_lmk && lane == 0) {
+      float m = -INFINITY;
+      for (int pl = 0; pl < P; ++pl) m = fmaxf(m, part_ml[((size_t)bk * P + pl) * G + g].x);
+      float l = 0.0f;
+      if (m > -INFINITY)
+        for (int pl = 0; pl < P; ++pl) {
+          const float2 ml = part_ml[((size_t)bk * P + pl) * G + g];
+          if (ml.x > -INFINITY) l += ml.y * __expf(ml.x - m);
+        }
+      lse_lmk[hrow] = (m > -INFINITY) ? m + __logf(l) : -INFINITY;
+    }
+  }
+  if (tid == 0) atomicOr(&bitmap[own >> 5], 1u << (own & 31));
+  __syncthreads();
+  // union positions: exclusive prefix of the bitmap popcounts (one warp)
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < ds.nwords; base += 32) {
+      const int i = base + lane;
+      const int c = i < ds.nwords ? __popc(bitmap[i]) : 0;
+      int x = c;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (i < ds.nwords) prefix[i] = carry + x - c;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) total = carry;
+  }
+  __syncthreads();
+  const int cap = ds.ucap;
+  int32_t *uc = u_c + (size_t)bk * cap;
+  uint32_t *um = u_mask + (size_t)bk * cap;
+  float *ul = u_logit + (size_t)bk * cap * G;
+  for (int i = tid; i < total; i += blockDim.x) um[i] = 0;
+  __syncthreads();
+  auto pos_of = [&](int c) {
+    return prefix[c >> 5] + __popc(bitmap[c >> 5] & ((1u << (c & 31)) - 1u));
+  };
+  for (int i = tid; i < G * K; i += blockDim.x) {
+    const int g = i / K;
+    const uint64_t x = chosen[i];
+    if (!x) continue;
+    const int c = key_chunk(x);
+    const int pos = pos_of(c);
+    uc[pos] = c;
+    atomicOr(&um[pos], 1u << g);
+    ul[pos * G + g] = key_score(x);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    const int pos = pos_of(own);
+    uc[pos] = own;
+    um[pos] = (1u << G) - 1u;  // every head attends its own chunk
+    u_count[bk] = total;
+  }
+}
+
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(256) decode_attn_kernel(DecodeSpec ds, const T *__restrict__ q,
+                                                          const T *__restrict__ kc,
+                                                          const T *__restrict__ vc,
+                                                          const int32_t *__restrict__ u_c,
+                                                          const uint32_t *__restrict__ u_mask,
+                                                          const float *__restrict__ u_logit,
+                                                          const int32_t *__restrict__ u_count,
+                                                          float *__restrict__ part,
+                                                          uint32_t *__restrict__ err) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  T *ks = reinterpret_cast<T *>(smem);             // [2][64][D]
+  T *vs = ks + 2 * kC * D;                         // [2][64][D]
+  float *qs = reinterpret_cast<float *>(vs + 2 * kC * D);  // [G][D] (scaled)
+  float *xs = qs + kMaxG * D;                      // [G][64] logits / probabilities
+  float *st = xs + kMaxG * kC;                     // [G][4]: per-chunk m, l, weight logit
+  __shared__ uint64_t bars[2];
+  __shared__ int abort_flag;
+
+  const int G = ds.Hq / ds.Hkv;
+  const int qi = blockIdx.x, bk = blockIdx.y;
+  const int b = bk / ds.Hkv, hkv = bk % ds.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int count = u_count[bk];
+  const int i0 = qi * kChunksPerCta, i1 = min(count, i0 + kChunksPerCta);
+  const int cap = ds.ucap;
+  const size_t kvbase = (size_t)bk * ds.N;
+  const int t = ds.N - 1, own = ds.own;
+
+  if (tid == 0) {
+    abort_flag = 0;
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+  }
+  for (int i = tid; i < G * D; i += blockDim.x) {
+    const int g = i / D, e = i % D;
+    qs[i] = to_f(q[((size_t)b * ds.Hq + hkv * G + g) * D + e]) * ds.scale;
+  }
+  __syncthreads();
+  auto issue = [&](int i, int buf) {
+    const int c = u_c[(size_t)bk * cap + i];
+    const int rows = min(kC, ds.N - c * kC);
+    const uint32_t bytes = (uint32_t)rows * D * sizeof(T);
+    mbar_expect_tx(&bars[buf], 2 * bytes);
+    bulk_g2s(ks + buf * kC * D, kc + (kvbase + (size_t)c * kC) * D, bytes, &bars[buf]);
+    bulk_g2s(vs + buf * kC * D, vc + (kvbase + (size_t)c * kC) * D, bytes, &bars[buf]);
+  };
+  if (tid == 0 && i0 < i1) issue(i0, 0);
+
+  // running (max M, sum L, acc) per head: thread (g, e-pair) owns 2 columns of acc
+  const int e2n = D / 2;
+  float acc[2 * ((kMaxG * (D / 2) + 255) / 256)];
+  constexpr int kAccSlots = (kMaxG * (D / 2) + 255) / 256;
+#pragma unroll
+  for (int s = 0; s < 2 * kAccSlots; ++s) acc[s] = 0.0f;
+  float Mr[kMaxG], Lr[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) { Mr[g] = -INFINITY; Lr[g] = 0.0f; }
+
+  bool ok = true;
+  for (int i = i0; i < i1; ++i) {
+    const int buf = (i - i0) & 1;
+    if (tid == 0 && i + 1 < i1) issue(i + 1, buf ^ 1);
+    ok = __syncthreads_and(wait_bar(&bars[buf], ((i - i0) >> 1) & 1, &abort_flag));
+    if (!ok) {
+      // drain: a copy issued for the next chunk must land before the CTA exits
+      if (tid == 0 && i + 1 < i1) mbar_wait_bounded(&bars[buf ^ 1], ((i + 1 - i0) >> 1) & 1);
+      break;
+    }
+    const int c = u_c[(size_t)bk * cap + i];
+    const uint32_t mask = u_mask[(size_t)bk * cap + i];
+    const int jmax = (c == own) ? (t - c * kC) : (kC - 1);
+    const T *kt = ks + buf * kC * D;
+    const T *vt = vs + buf * kC * D;
+    // logits x[g][j] = scale * <q_g, k_j>
+    for (int pr = tid; pr < G * kC; pr += blockDim.x) {
+      const int g = pr / kC, j = pr % kC;
+      float a = -INFINITY;
+      if (((mask >> g) & 1u) && j <= jmax) {
+        a = 0.0f;
+        for (int cc = 0; cc < D / 8; ++cc) {
+          const int col = (cc + j) % (D / 8);
+          float f[8];
+          load8<T>(kt + j * D + col * 8, f);
+          const float *qq = qs + g * D + col * 8;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) a = fmaf(f[u], qq[u], a);
+        }
+      }
+      xs[g * kC + j] = a;
+    }
+    __syncthreads();
+    // per head: m, l over the chunk; probabilities e_j = exp(x_j - m)
+    for (int g = warp; g < G; g += blockDim.x / 32) {
+      const float a0 = xs[g * kC + lane], a1 = xs[g * kC + lane + 32];
+      float m = fmaxf(a0, a1);
+      for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const float e0 = (m > -INFINITY) ? __expf(a0 - m) : 0.0f;
+      const float e1 = (m > -INFINITY) ? __expf(a1 - m) : 0.0f;
+      float l = e0 + e1;
+      for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      xs[g * kC + lane] = e0;
+      xs[g * kC + lane + 32] = e1;
+      if (lane == 0) {
+        st[g * 4 + 0] = m;
+        st[g * 4 + 1] = l;
+        // the chunk's fusion logit: its landmark logit, or for the own chunk
+        // the log-sum-exp of its causal token logits
+        st[g * 4 + 2] = (c == own) ? m + __logf(l) : u_logit[((size_t)bk * cap + i) * G + g];
+      }
+    }
+    __syncthreads();
+    // acc_g = acc_g * exp(M_old - M_new) + exp(logit - M_new) / l * sum_j e_j v_j
+#pragma unroll
+    for (int s = 0; s < kAccSlots; ++s) {
+      const int pr = tid + s * 256;
+      const int g = pr / e2n, e2 = pr % e2n;
+      if (g < G && ((mask >> g) & 1u)) {
+        float o0 = 0.0f, o1 = 0.0f;
+        for (int j = 0; j <= jmax; ++j) {
+          const float pj = xs[g * kC + j];
+          float v0, v1;
+          if constexpr (sizeof(T) == 2) {
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(vt + j * D + 2 * e2);
+            v0 = __uint_as_float(w << 16);
+            v1 = __uint_as_float(w & 0xFFFF0000u);
+          } else {
+            const float2 w = *reinterpret_cast<const float2 *>(vt + j * D + 2 * e2);
+            v0 = w.x;
+            v1 = w.y;
+          }
+          o0 = fmaf(pj, v0, o0);
+          o1 = fmaf(pj, v1, o1);
+        }
+        const float lg = st[g * 4 + 2], l = st[g * 4 + 1];
+        float mo = 0.0f, ln = 0.0f;
+#pragma unroll
+        for (int gg = 0; gg < kMaxG; ++gg)
+          if (gg == g) { mo = Mr[gg]; ln = Lr[gg]; }
+        const float mn = fmaxf(mo, lg);
+        const float so = __expf(mo - mn), sn = __expf(lg - mn);
+        acc[2 * s] = acc[2 * s] * so + sn * o0 / l;
+        acc[2 * s + 1] = acc[2 * s + 1] * so + sn * o1 / l;
+      }
+    }
+    // running max / sum per head (every thread keeps all heads' copies)
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) {
+      if (g < G && ((mask >> g) & 1u)) {
+        const float lg = st[g * 4 + 2];
+        const float mn = fmaxf(Mr[g], lg);
+        Lr[g] = Lr[g] * __expf(Mr[g] - mn) + __expf(lg - mn);
+        Mr[g] = mn;
+      }
+    }
+    __syncthreads();  // the buffer and xs are reused
+  }
+  // partial record per (bk, qi, g): [M, L, acc[D]]
+  const size_t rec = 2 + D;
+#pragma unroll
+  for (int s = 0; s < kAccSlots; ++s) {
+    const int pr = tid + s * 256;
+    const int g = pr / e2n, e2 = pr % e2n;
+    if (g < G) {
+      float *r = part + (((size_t)bk * ds.Q + qi) * G + g) * rec;
+      r[2 + 2 * e2] = acc[2 * s];
+      r[3 + 2 * e2] = acc[2 * s + 1];
+      if (e2 == 0) {
+        float mo = 0.0f, lo = 0.0f;
+#pragma unroll
+        for (int gg = 0; gg < kMaxG; ++gg)
+          if (gg == g) { mo = Mr[gg]; lo = Lr[gg]; }
+        r[0] = mo;
+        r[1] = lo;
+      }
+    }
+  }
+  if (tid == 0 && abort_flag) report(err, DEV_TIMEOUT);
+}
+
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(D) decode_combine_kernel(DecodeSpec ds,
+                                                           const float *__restrict__ part,
+                                                           T *__restrict__ out,
+                                                           float *__restrict__ lse) {
+  const int G = ds.Hq / ds.Hkv;
+  const int h = blockIdx.x;  // b*Hq + hq
+  const int b = h / ds.Hq, hq = h % ds.Hq;
+  const int bk = b * ds.Hkv + hq / G, g = hq % G;
+  const size_t rec = 2 + D;
+  float M = -INFINITY;
+  for (int s = 0; s < ds.Q; ++s) M = fmaxf(M, part[(((size_t)bk * ds.Q + s) * G + g) * rec]);
+  float L = 0.0f, o = 0.0f;
+  for (int s = 0; s < ds.Q; ++s) {
+    const float *r = part + (((size_t)bk * ds.Q + s) * G + g) * rec;
+    if (r[0] == -INFINITY) continue;
+    const float w = __expf(r[0] - M);
+    L += w * r[1];
+    o += w * r[2 + threadIdx.x];
+  }
+  out[(size_t)h * D + threadIdx.x] = from_f<T>(o / L);
+  if (threadIdx.x == 0) lse[h] = M + __logf(L);
+}
+
+}  // namespace
+
+DecodeSpec decode_spec(int B, int Hq, int Hkv, int N, int d, int topk, float scale) {
+  DecodeSpec ds{};
+  ds.B = B;
+  ds.Hq = Hq;
+  ds.Hkv = Hkv;
+  ds.N = N;
+  ds.d = d;
+  ds.topk = topk;
+  ds.scale = scale;
+  ds.own = (N - 1) / kC;
+  ds.nlmk = N / kC;
+  ds.n_c = ds.own;  // completed chunks of the query at N-1 (all of them have a landmark)
+  ds.P = (ds.n_c + kSlab - 1) / kSlab;
+  ds.nwords = ((N + kC - 1) / kC + 31) / 32;
+  const int G = Hq / Hkv;
+  ds.ucap = G * topk + 1;
+  ds.Q = (ds.ucap + kChunksPerCta - 1) / kChunksPerCta;
+  return ds;
+}
+
+// workspace carve-up (256-byte aligned pieces)
+static size_t al(size_t x) { return (x + 255) & ~size_t(255); }
+size_t decode_workspace_bytes(const DecodeSpec &ds) {
+  const int G = ds.Hq / ds.Hkv;
+  const size_t BK = (size_t)ds.B * ds.Hkv;
+  size_t n = 256;                                          // error word
+  n += al(BK * ds.P * G * ds.topk * sizeof(uint64_t));     // part_keys
+  n += al(BK * ds.P * G * sizeof(float2));                 // part_ml
+  n += al(BK * ds.ucap * sizeof(int32_t));                 // u_c
+  n += al(BK * ds.ucap * sizeof(uint32_t));                // u_mask
+  n += al(BK * ds.ucap * G * sizeof(float));               // u_logit
+  n += al(BK * sizeof(int32_t));                           // u_count
+  n += al(BK * ds.Q * G * (2 + ds.d) * sizeof(float));     // attention partials
+  return n;
+}
+
+size_t decode_max_g() { return kMaxG; }
+
+cudaError_t decode_fwd(const DecodeSpec &ds, bool bf16, const void *q, const void *k,
+                       const void *v, const void *lmk, int32_t *sel, float *w, float *lse_lmk,
+                       void *out, float *lse, void *ws, uint32_t *err, cudaStream_t st,
+                       int *launches) {
+  const int G = ds.Hq / ds.Hkv;
+  const size_t BK = (size_t)ds.B * ds.Hkv;
+  unsigned char *p = static_cast<unsigned char *>(ws) + 256;
+  auto take = [&](size_t bytes) {
+    unsigned char *r = p;
+    p += al(bytes);
+    return r;
+  };
+  uint64_t *part_keys = reinterpret_cast<uint64_t *>(take(BK * ds.P * G * ds.topk * 8));
+  float2 *part_ml = reinterpret_cast<float2 *>(take(BK * ds.P * G * sizeof(float2)));
+  int32_t *u_c = reinterpret_cast<int32_t *>(take(BK * ds.ucap * 4));
+  uint32_t *u_mask = reinterpret_cast<uint32_t *>(take(BK * ds.ucap * 4));
+  float *u_logit = reinterpret_cast<float *>(take(BK * ds.ucap * G * 4));
+  int32_t *u_count = reinterpret_cast<int32_t *>(take(BK * 4));
+  float *part = reinterpret_cast<float *>(take(BK * ds.Q * G * (2 + ds.d) * 4));
+  const size_t esz = bf16 ? 2 : 4;
+  cudaError_t e;
+
+  if (ds.P > 0) {
+    const size_t smem = kSlab * ds.d * esz + kMaxG * ds.d * 4 + kMaxG * kSlab * 8 + 8 * kMaxG * 4;
+#define HILS_SCORE(T, DD)                                                                       \
+  do {                                                                                          \
+    auto kern = decode_score_kernel<T, DD>;                                                     \
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e; \
+    kern<<<dim3(ds.P, (unsigned)BK), 256, smem, st>>>(ds, (const T *)q, (const T *)lmk, part_keys, part_ml, err); \
+  } while (0)
+    if (bf16) { if (ds.d == 64) HILS_SCORE(__nv_bfloat16, 64); else HILS_SCORE(__nv_bfloat16, 128); }
+    else { if (ds.d == 64) HILS_SCORE(float, 64); else HILS_SCORE(float, 128); }
+#undef HILS_SCORE
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ++*launches;
+  }
+  {
+    const size_t smem = (size_t)G * ds.topk * 8 + (size_t)ds.nwords * 8 + (size_t)G * ds.P * 4;
+    if ((e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
+    decode_merge_kernel<<<(unsigned)BK, 256, smem, st>>>(ds, part_keys, part_ml, sel, w, lse_lmk,
+                                                         u_c, u_mask, u_logit, u_count);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ++*launches;
+  }
+  {
+    const size_t smem = 4 * (size_t)kC * ds.d * esz + kMaxG * ds.d * 4 + kMaxG * kC * 4 + kMaxG * 16;
+#define HILS_ATTN(T, DD)                                                                        \
+  do {                                                                                          \
+    auto kern = decode_attn_kernel<T, DD>;                                                      \
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e; \
+    kern<<<dim3(ds.Q, (unsigned)BK), 256, smem, st>>>(ds, (const T *)q, (const T *)k, (const T *)v, u_c, u_mask, u_logit, u_count, part, err); \
+  } while (0)
+    if (bf16) { if (ds.d == 64) HILS_ATTN(__nv_bfloat16, 64); else HILS_ATTN(__nv_bfloat16, 128); }
+    else { if (ds.d == 64) HILS_ATTN(float, 64); else HILS_ATTN(float, 128); }
+#undef HILS_ATTN
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ++*launches;
+  }
+  {
+    const int nh = ds.B * ds.Hq;
+#define HILS_COMB(T, DD) decode_combine_kernel<T, DD><<<nh, DD, 0, st>>>(ds, part, (T *)out, lse)
+    if (bf16) { if (ds.d == 64) HILS_COMB(__nv_bfloat16, 64); else HILS_COMB(__nv_bfloat16, 128); }
+    else { if (ds.d == 64) HILS_COMB(float, 64); else HILS_COMB(float, 128); }
+#undef HILS_COMB
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ++*launches;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace hils

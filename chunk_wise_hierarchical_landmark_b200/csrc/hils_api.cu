@@ -73,9 +73,6 @@ hils_status check_params(const hils_params *p) {
 hils::RowSpec prefill_rows(const hils_params *p) {
   return hils::RowSpec{p->B, p->Hq, p->Hkv, p->L, p->d, p->chunk, p->topk, p->scale, 0, p->L};
 }
-hils::RowSpec decode_rows(const hils_params *p) {
-  return hils::RowSpec{p->B, p->Hq, p->Hkv, p->L, p->d, p->chunk, p->topk, p->scale, p->L - 1, 1};
-}
 
 // Debug mode: clear the device error word before the launches ...
 hils_status debug_begin(const hils_params *p, void *ws, size_t ws_bytes, uint32_t **err,
@@ -124,12 +121,26 @@ hils_status do_attn(const hils_params *p, const hils::RowSpec &rs, const void *q
   return e == cudaSuccess ? HILS_OK : cuda_fail(e, "attention launch");
 }
 
+hils::DecodeSpec decode_spec_of(const hils_params *p) {
+  return hils::decode_spec(p->B, p->Hq, p->Hkv, p->L, p->d, p->topk, p->scale);
+}
+
+hils_status check_decode(const hils_params *p) {
+  if ((size_t)(p->Hq / p->Hkv) > hils::decode_max_g())
+    return fail(HILS_ERR_UNSUPPORTED, "decode supports Hq/Hkv <= %zu", hils::decode_max_g());
+  return HILS_OK;
+}
+
 }  // namespace
 
 HILS_API size_t hils_workspace_size(const hils_params *p, int op) {
   if (check_params(p) != HILS_OK) return 0;
-  if (op != HILS_OP_PREFILL && op != HILS_OP_DECODE) return 0;
-  return p->debug_checks ? kDebugWs : 0;
+  if (op == HILS_OP_PREFILL) return p->debug_checks ? kDebugWs : 0;
+  if (op == HILS_OP_DECODE) {
+    if (check_decode(p) != HILS_OK) return 0;
+    return hils::decode_workspace_bytes(decode_spec_of(p));
+  }
+  return 0;
 }
 
 HILS_API hils_status hils_select(const hils_params *p, const void *q, const void *lmk_k,
@@ -225,14 +236,20 @@ HILS_API hils_status hils_decode_fwd(const hils_params *p, const void *q, const 
   NEED(lse);
   MAYBE(lse_lmk);
   if (p->L > p->chunk) NEED(lmk_k);
+  if ((s = check_decode(p)) != HILS_OK) return s;
+  const hils::DecodeSpec ds = decode_spec_of(p);
+  const size_t need = hils::decode_workspace_bytes(ds);
+  if (!ws || ws_bytes < need)
+    return fail(HILS_ERR_WORKSPACE, "decode needs %zu bytes of workspace, got %zu", need, ws_bytes);
+  NEED(ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t *err = nullptr;
   if ((s = debug_begin(p, ws, ws_bytes, &err, st)) != HILS_OK) return s;
-  const hils::RowSpec rs = decode_rows(p);
-  if ((s = do_select(p, rs, q, lmk_k, sel_idx, chunk_w, lse_lmk, err, st)) != HILS_OK) return s;
-  if ((s = do_attn(p, rs, q, k_cache, v_cache, sel_idx, chunk_w, out, lse, nullptr, err, st)) !=
-      HILS_OK)
-    return s;
+  int n = 0;
+  cudaError_t e = hils::decode_fwd(ds, p->dtype == HILS_BF16, q, k_cache, v_cache, lmk_k, sel_idx,
+                                   chunk_w, lse_lmk, out, lse, ws, err, st, &n);
+  g_launches += n;
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return debug_end(err, st);
 }
 

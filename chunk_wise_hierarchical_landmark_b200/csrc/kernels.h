@@ -44,6 +44,24 @@ namespace hils {
 cudaError_t make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
                            uint32_t box_rows);
 
+// Decode step (decode.cu).  One query per head at position N-1.
+struct DecodeSpec {
+  int B, Hq, Hkv, N, d, topk;
+  float scale;
+  int own, nlmk, n_c;  // own chunk, landmark rows per KV head, completed chunks
+  int P;               // landmark slabs of 256 (scoring CTAs per KV head)
+  int nwords;          // chunk bitmap words
+  int ucap;            // union capacity per KV head: G * topk + 1
+  int Q;               // attention CTAs per KV head
+};
+DecodeSpec decode_spec(int B, int Hq, int Hkv, int N, int d, int topk, float scale);
+size_t decode_workspace_bytes(const DecodeSpec &ds);
+size_t decode_max_g();
+cudaError_t decode_fwd(const DecodeSpec &ds, bool bf16, const void *q, const void *k,
+                       const void *v, const void *lmk, int32_t *sel, float *w, float *lse_lmk,
+                       void *out, float *lse, void *ws, uint32_t *err, cudaStream_t st,
+                       int *launches);
+
 // Chunk union in CSR form (hils_union.cu)
 cudaError_t union_csr(int B, int Hq, int L, int C, int topk, int M, const int32_t *sel,
                       int32_t *u_off, int32_t *u_idx, int64_t u_cap, uint32_t *err,

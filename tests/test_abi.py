@@ -89,3 +89,14 @@ def test_status_strings(lib):
         assert lib.hils_status_string(s)
     assert lib.hils_status_string(0) == b"ok"
     assert lib.hils_launch_count() >= 0
+
+
+def test_decode_workspace_size(lib):
+    p = hb.make_params(B=16, Hq=32, Hkv=8, L=524288, d=128, topk=64)
+    n = lib.hils_workspace_size(ctypes.byref(p), hb.HILS_OP_DECODE)
+    assert 10_000_000 < n < 100_000_000   # slab top-k lists, union, attention partials
+    too_many_heads = hb.make_params(B=1, Hq=32, Hkv=2, L=4096, d=128, topk=8)
+    assert lib.hils_workspace_size(ctypes.byref(too_many_heads), hb.HILS_OP_DECODE) == 0
+    rc = lib.hils_decode_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                             FAKE, None, 0, None)
+    assert rc == 3   # workspace too small, rejected before any launch
