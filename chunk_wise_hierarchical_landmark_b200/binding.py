@@ -37,8 +37,8 @@ class Params(ctypes.Structure):
 
 _lib = None
 EXPORTS = ["hils_workspace_size", "hils_select", "hils_union_capacity", "hils_union",
-           "hils_attn_fwd", "hils_prefill", "hils_decode_fwd", "hils_status_string",
-           "hils_last_error", "hils_launch_count"]
+           "hils_attn_fwd", "hils_prefill", "hils_decode_fwd", "hils_decode_fwd_noalloc",
+           "hils_status_string", "hils_last_error", "hils_launch_count"]
 
 
 def lib():
@@ -59,7 +59,9 @@ def lib():
         L.hils_attn_fwd.argtypes = [PP, P, P, P, P, P, P, P, P, P, SZ, P]
         L.hils_prefill.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.hils_decode_fwd.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, SZ, P]
-        for f in ("hils_select", "hils_union", "hils_attn_fwd", "hils_prefill", "hils_decode_fwd"):
+        L.hils_decode_fwd_noalloc.argtypes = [PP, P, P, P, P, P, P, P, P, P, P]
+        for f in ("hils_select", "hils_union", "hils_attn_fwd", "hils_prefill", "hils_decode_fwd",
+                  "hils_decode_fwd_noalloc"):
             getattr(L, f).restype = I
         L.hils_status_string.argtypes = [I]
         L.hils_status_string.restype = ctypes.c_char_p
@@ -146,6 +148,13 @@ def hils_decode_fwd(p: Params, q, k_cache, v_cache, lmk_k, sel_idx, chunk_w, lse
     _check(lib().hils_decode_fwd(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                  _ptr(lmk_k), _ptr(sel_idx), _ptr(chunk_w), _ptr(lse_lmk),
                                  _ptr(out), _ptr(lse), *_ws_args(ws), _stream(stream)))
+
+
+def hils_decode_fwd_noalloc(p: Params, q, k_cache, v_cache, lmk_k, sel_idx, chunk_w, lse_lmk,
+                            out, lse, stream=None):
+    _check(lib().hils_decode_fwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                         _ptr(lmk_k), _ptr(sel_idx), _ptr(chunk_w), _ptr(lse_lmk),
+                                         _ptr(out), _ptr(lse), _stream(stream)))
 
 
 def launch_count() -> int:

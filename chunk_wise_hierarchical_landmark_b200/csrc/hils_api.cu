@@ -268,4 +268,6 @@ HILS_API const char *hils_status_string(hils_status s) {
 
 HILS_API const char *hils_last_error(void) { return g_msg; }
 
+extern "C" void hils_internal_set_error(const char *msg) { fail(HILS_ERR_INVALID_ARG, "%s", msg); }
+
 HILS_API int64_t hils_launch_count(void) { return g_launches.load(); }

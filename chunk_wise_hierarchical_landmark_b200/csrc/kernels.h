@@ -62,6 +62,9 @@ cudaError_t decode_fwd(const DecodeSpec &ds, bool bf16, const void *q, const voi
                        void *out, float *lse, void *ws, uint32_t *err, cudaStream_t st,
                        int *launches);
 
+// Internal (not exported): set the calling thread's hils_last_error() text.
+extern "C" void hils_internal_set_error(const char *msg);
+
 // Chunk union in CSR form (hils_union.cu)
 cudaError_t union_csr(int B, int Hq, int L, int C, int topk, int M, const int32_t *sel,
                       int32_t *u_off, int32_t *u_idx, int64_t u_cap, uint32_t *err,

@@ -158,6 +158,27 @@ hils_status hils_decode_fwd(const hils_params *p, const void *q, const void *k_c
                             float *chunk_w, float *lse_lmk, void *out, float *lse, void *ws,
                             size_t ws_bytes, void *stream);
 
+/*
+ * Allocation-free variant of hils_decode_fwd.  The paper has no counterpart:
+ * this is a deployment aid.  It is for callers that cannot pass a workspace
+ * because they cannot allocate device memory -- e.g. a serving framework that
+ * reserves all GPU memory for its own pool and forbids cudaMalloc elsewhere,
+ * or a per-token decode loop where cudaMalloc/cudaFree would synchronise the
+ * device.  Arguments and results are those of hils_decode_fwd, without ws.
+ * The decode scratch lives in a fixed 32 MiB device array inside the library
+ * (held on every GPU that loads the library until the process exits); shapes
+ * that need more scratch return HILS_ERR_WORKSPACE before any launch.  The
+ * first call on a device looks the array up (cudaGetSymbolAddress, which may
+ * load the library's module there): make it before any stream capture.  All
+ * calls share the array and it keeps the last call's contents (each call
+ * writes every scratch entry it reads); calls that overlap on the GPU race
+ * and must be serialised by the caller.  Nothing here allocates.
+ */
+hils_status hils_decode_fwd_noalloc(const hils_params *p, const void *q, const void *k_cache,
+                                    const void *v_cache, const void *lmk_k, int32_t *sel_idx,
+                                    float *chunk_w, float *lse_lmk, void *out, float *lse,
+                                    void *stream);
+
 /* Static description of a status code. */
 const char *hils_status_string(hils_status s);
 
