@@ -14,8 +14,9 @@
 //              into an NS-stage ring;
 //   warp 1     TMEM owner and MMA issuer (one thread): S = Q K_c^T into one of
 //              two TMEM buffers, then O += P_c V_c into the TMEM accumulator;
-//   warps 2-5  one thread per row (TMEM lane): chunk softmax, P -> shared
-//              memory (bf16, 128B-swizzled K-major), epilogue.
+//   warps 2-5  one thread per row (TMEM lane): chunk softmax, P -> tensor
+//              memory (bf16, two per column; the PV product reads its A
+//              operand from tensor memory), epilogue.
 // Processing order: the tile's own chunks first (later one first), then the
 // rest of the union ascending.  After its own chunk a row knows its largest
 // fusion logit M = max(lse_own, max selected logit), so every chunk's
@@ -50,19 +51,19 @@ template <int D>
 struct Layout {
   static constexpr int kQBytes = kRows * D * 2;
   static constexpr int kKVBytes = kChunk * D * 2;  // one of K or V for one chunk
-  static constexpr int kPBytes = kRows * kChunk * 2;
   static constexpr int q = 0;
   static constexpr int k0 = q + kQBytes;
   static constexpr int v0 = k0 + kStages * kKVBytes;
-  static constexpr int p0 = v0 + kStages * kKVBytes;
-  static constexpr int ones = p0 + 2 * kPBytes;   // 16 x 64 bf16 ones (B of the row-sum MMA)
+  static constexpr int ones = v0 + kStages * kKVBytes;  // 16 x 64 bf16 ones (B of the row-sum MMA)
   static constexpr int bars = ones + 16 * 128;
   static constexpr int misc = bars + 32 * 8;
   static constexpr int bitmap = misc + 64;
   static constexpr int fixed = bitmap;  // + bitmap words
-  // TMEM columns: S0 [0,64), S1 [64,128), O [128,128+D), row sums [128+D, 144+D)
+  // TMEM columns: S0 [0,64), S1 [64,128), O [128,128+D), row sums [128+D, 144+D),
+  // P0 / P1 (bf16 pairs, 32 columns each) after the sums on a 32-column boundary
   static constexpr uint32_t kSumCol = 128 + D;
-  static constexpr uint32_t kTmemCols = (kSumCol + 16 <= 256) ? 256 : 512;
+  static constexpr uint32_t kPCol = ((kSumCol + 16 + 31) / 32) * 32;
+  static constexpr uint32_t kTmemCols = (kPCol + 64 <= 256) ? 256 : 512;
 };
 
 struct Bars {
@@ -212,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t s_tmem[2] = {tmem, tmem + 64};
   const uint32_t o_tmem = tmem + 128;
   const uint32_t sum_tmem = tmem + Lay::kSumCol;
+  const uint32_t p_tmem[2] = {tmem + Lay::kPCol, tmem + Lay::kPCol + 32};
   unsigned char *q_s = smem + Lay::q;
   const int kv_row0 = (b * rs.Hkv + hkv) * L;
 
@@ -255,23 +257,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sb = j & 1, s = j % kStages;
         if (!mbar_wait(&bars->p_full[sb], (j >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t p_addr = smem_u32(smem + Lay::p0 + sb * Lay::kPBytes);
         const uint32_t v_addr = smem_u32(smem + Lay::v0 + s * Lay::kKVBytes);
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk) {
-          // A = P [128 x 64] K-major: 16 keys = 32 bytes along the 128-byte row
-          const uint64_t a = smem_desc_sw128(p_addr + kk * 32, 16, 1024);
+          // A = P [128 x 64] in tensor memory: 16 keys = 8 columns
           // B = V [64 keys x D] MN-major: 16 keys = 16 rows of 128 bytes;
           // the D axis is split into 64-wide blocks 64*128 bytes apart
           const uint64_t bdesc = smem_desc_sw128(v_addr + kk * 16 * 128, kChunk * 128, 1024);
-          mma_bf16_ss(o_tmem, a, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(o_tmem, p_tmem[sb] + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         // row sums of the rounded P: P [128 x 64] times ones [64 x 16]
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk) {
-          const uint64_t a = smem_desc_sw128(p_addr + kk * 32, 16, 1024);
           const uint64_t bdesc = smem_desc_sw128(ones_addr + kk * 32, 16, 1024);
-          mma_bf16_ss(sum_tmem, a, bdesc, idesc_sum, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(sum_tmem, p_tmem[sb] + kk * 8, bdesc, idesc_sum, (j > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&bars->kv_empty[s]);
         mma_commit(&bars->p_empty[sb]);
@@ -303,7 +302,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax rows
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    unsigned char *p_row0 = smem + Lay::p0 + r * 128;
     const float scale2 = rs.scale * kLog2e;
     float M2 = 0.0f, lse2_own = 0.0f;
     int ptr = 0;
@@ -381,13 +379,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait(&bars->p_empty[sb], ((i >> 1) - 1) & 1, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       }
-      unsigned char *prow = p_row0 + sb * Lay::kPBytes;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        uint4 v4 = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-        *reinterpret_cast<uint4 *>(prow + ((j ^ (r & 7)) << 4)) = v4;
-      }
-      fence_async_smem();
+      __syncwarp();  // tcgen05.st is warp-collective
+      tmem_st32(p_tmem[sb] + lane_off, pk);
+      tmem_wait_st();
+      tc_fence_before();
       mbar_arrive(&bars->p_full[sb]);
     }
     // ---------------------------------------------------------- epilogue
