@@ -9,14 +9,19 @@
 // of 128 adjacent queries of one head loads the union of their chunks once.
 //
 // One CTA = one tile of 128 query rows (positions [t0, t0+128) of one
-// (b, hq)); 6 warps:
+// (b, hq)); two CTAs share an SM (about 100 KB of shared memory and 256 TMEM
+// columns each).  6 warps:
 //   warp 0     TMA producer: Q tile once, then K_c / V_c of every union chunk
-//              into an NS-stage ring;
-//   warp 1     TMEM owner and MMA issuer (one thread): S = Q K_c^T into one of
-//              two TMEM buffers, then O += P_c V_c into the TMEM accumulator;
+//              into a 2-stage ring;
+//   warp 1     TMEM owner and MMA issuer (one thread): S = Q K_c^T into TMEM,
+//              then O += P_c V_c and the row sums of P_c (against an all-ones
+//              tile), both reading P from tensor memory;
 //   warps 2-5  one thread per row (TMEM lane): chunk softmax, P -> tensor
-//              memory (bf16, two per column; the PV product reads its A
-//              operand from tensor memory), epilogue.
+//              memory (bf16, two per column), epilogue.
+// S and P are single-buffered: the MMA computes S for the next chunk while
+// the rows turn the current S into P, and P·V for a chunk while the rows work
+// on the next S.
+//
 // Processing order: the tile's own chunks first (later one first), then the
 // rest of the union ascending.  After its own chunk a row knows its largest
 // fusion logit M = max(lse_own, max selected logit), so every chunk's
@@ -25,10 +30,9 @@
 //   P_j = exp(x_j - M)                               (own chunk)
 // and O = sum_c P_c V_c needs no rescaling.  P is rounded to bf16 for the
 // tensor core; the output is normalised by the sum of the ROUNDED
-// probabilities, which the tensor core accumulates alongside O (P times an
-// all-ones 64x16 tile into a 16-column TMEM sum), so the weights applied to V
-// sum to one exactly: out = O / sum_j bf16(P_j).  lse stays the fp32 value
-// M + log(sum_c exp(s_c - M)).
+// probabilities, which the tensor core accumulates alongside O, so the
+// weights applied to V sum to one exactly: out = O / sum_j bf16(P_j).  lse
+// stays the fp32 value M + log(sum_c exp(s_c - M)).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -42,7 +46,7 @@ using namespace sm100;
 
 constexpr int kRows = 128;   // query rows per tile (UMMA M)
 constexpr int kChunk = 64;   // keys per chunk (UMMA N of QK^T, K of PV)
-constexpr int kStages = 3;   // K/V ring depth
+constexpr int kStages = 2;   // K/V ring depth
 constexpr int kThreads = 192;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -56,19 +60,15 @@ struct Layout {
   static constexpr int v0 = k0 + kStages * kKVBytes;
   static constexpr int ones = v0 + kStages * kKVBytes;  // 16 x 64 bf16 ones (B of the row-sum MMA)
   static constexpr int bars = ones + 16 * 128;
-  static constexpr int misc = bars + 32 * 8;
+  static constexpr int misc = bars + 16 * 8;
   static constexpr int bitmap = misc + 64;
   static constexpr int fixed = bitmap;  // + bitmap words
-  // TMEM columns: S0 [0,64), S1 [64,128), O [128,128+D), row sums [128+D, 144+D),
-  // P0 / P1 (bf16 pairs, 32 columns each) after the sums on a 32-column boundary
-  static constexpr uint32_t kSumCol = 128 + D;
-  static constexpr uint32_t kPCol = ((kSumCol + 16 + 31) / 32) * 32;
-  static constexpr uint32_t kTmemCols = (kPCol + 64 <= 256) ? 256 : 512;
+  // TMEM columns: S [0,64), P [64,96) (bf16 pairs), row sums [96,112), O [128,128+D)
+  static constexpr uint32_t kSCol = 0, kPCol = 64, kSumCol = 96, kOCol = 128, kTmemCols = 256;
 };
 
 struct Bars {
-  uint64_t q, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], p_full[2],
-      p_empty[2], o_full, done;
+  uint64_t q, kv_full[kStages], kv_empty[kStages], s_full, s_free, p_full, p_free, o_full, done;
 };
 
 struct ChunkIter {
@@ -100,8 +100,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, RowSpec rs,
@@ -109,10 +115,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                       __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out,
                       float *__restrict__ wfin, uint32_t *__restrict__ err) {
   using Lay = Layout<D>;
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  // 1024-byte alignment for the 128B-swizzled tiles
-  unsigned char *smem = reinterpret_cast<unsigned char *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // The 128-byte-swizzled tiles need a 1024-byte aligned base; the dynamic
+  // shared window starts there (no static shared memory), checked here.
+  extern __shared__ __align__(1024) unsigned char smem[];
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) report(err, DEV_BAD_INDEX);
+    return;
+  }
   Bars *bars = reinterpret_cast<Bars *>(smem + Lay::bars);
   uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(smem + Lay::misc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::misc + 4);
@@ -136,12 +145,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->s_empty[i], kRows);
-      mbar_init(&bars->p_full[i], kRows);
-      mbar_init(&bars->p_empty[i], 1);
-    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_free, kRows);
+    mbar_init(&bars->p_full, kRows);
+    mbar_init(&bars->p_free, 1);
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->done, 1);
     *abort_flag = 0;
@@ -186,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       wmax2 = fmaxf(wmax2, __ldg(myw + i) * kLog2e);
       ++nsel;
     }
-    for (int i = 0; i < nsel; ++i) sumsel += exp2f(__ldg(myw + i) * kLog2e - wmax2);
+    for (int i = 0; i < nsel; ++i) sumsel += ex2_approx(__ldg(myw + i) * kLog2e - wmax2);
     walk_n = nsel;
     if (own == c0 + 1 && nsel > 0 && __ldg(mysel + nsel - 1) == c0) {
       has_c0 = true;
@@ -210,10 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   const int n_steps = *n_steps_slot;
 
-  const uint32_t s_tmem[2] = {tmem, tmem + 64};
-  const uint32_t o_tmem = tmem + 128;
+  const uint32_t s_tmem = tmem + Lay::kSCol;
+  const uint32_t p_tmem = tmem + Lay::kPCol;
   const uint32_t sum_tmem = tmem + Lay::kSumCol;
-  const uint32_t p_tmem[2] = {tmem + Lay::kPCol, tmem + Lay::kPCol + 32};
+  const uint32_t o_tmem = tmem + Lay::kOCol;
   unsigned char *q_s = smem + Lay::q;
   const int kv_row0 = (b * rs.Hkv + hkv) * L;
 
@@ -254,8 +261,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ones_addr = smem_u32(smem + Lay::ones);
       const uint32_t q_addr = smem_u32(q_s);
       auto pv = [&](int j) -> bool {
-        const int sb = j & 1, s = j % kStages;
-        if (!mbar_wait(&bars->p_full[sb], (j >> 1) & 1, abort_flag)) return false;
+        const int s = j % kStages;
+        if (!mbar_wait(&bars->p_full, j & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(smem + Lay::v0 + s * Lay::kKVBytes);
 #pragma unroll
@@ -264,23 +271,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           // B = V [64 keys x D] MN-major: 16 keys = 16 rows of 128 bytes;
           // the D axis is split into 64-wide blocks 64*128 bytes apart
           const uint64_t bdesc = smem_desc_sw128(v_addr + kk * 16 * 128, kChunk * 128, 1024);
-          mma_bf16_ts(o_tmem, p_tmem[sb] + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         // row sums of the rounded P: P [128 x 64] times ones [64 x 16]
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk) {
           const uint64_t bdesc = smem_desc_sw128(ones_addr + kk * 32, 16, 1024);
-          mma_bf16_ts(sum_tmem, p_tmem[sb] + kk * 8, bdesc, idesc_sum, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(sum_tmem, p_tmem + kk * 8, bdesc, idesc_sum, (j > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&bars->kv_empty[s]);
-        mma_commit(&bars->p_empty[sb]);
+        mma_commit(&bars->p_free);
         return true;
       };
       bool ok = mbar_wait(&bars->q, 0, abort_flag);
       for (int i = 0; ok && i < n_steps; ++i) {
-        const int s = i % kStages, sb = i & 1;
+        const int s = i % kStages;
         if (!mbar_wait(&bars->kv_full[s], (i / kStages) & 1, abort_flag)) { ok = false; break; }
-        if (i >= 2 && !mbar_wait(&bars->s_empty[sb], ((i >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+        // S is single-buffered: the rows must have read the previous S
+        if (i >= 1 && !mbar_wait(&bars->s_free, (i - 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t k_addr = smem_u32(smem + Lay::k0 + s * Lay::kKVBytes);
 #pragma unroll
@@ -288,9 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int kb = kk >> 2, kw = kk & 3;
           const uint64_t a = smem_desc_sw128(q_addr + kb * kRows * 128 + kw * 32, 16, 1024);
           const uint64_t bdesc = smem_desc_sw128(k_addr + kb * kChunk * 128 + kw * 32, 16, 1024);
-          mma_bf16_ss(s_tmem[sb], a, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+          mma_bf16_ss(s_tmem, a, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bars->s_full[sb]);
+        mma_commit(&bars->s_full);
         if (i >= 1 && !pv(i - 1)) { ok = false; break; }
       }
       if (ok) ok = pv(n_steps - 1);
@@ -305,27 +313,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float scale2 = rs.scale * kLog2e;
     float M2 = 0.0f, lse2_own = 0.0f;
     int ptr = 0;
-    int nc = (valid && walk_n > 0) ? __ldg(mysel) : -1;
-    float nw = (valid && walk_n > 0) ? __ldg(myw) * kLog2e : 0.0f;
+    // the row's next two selected chunks (ids and base-2 logits), prefetched
+    int nc = -1, nc2 = -1;
+    float nw = 0.0f, nw2 = 0.0f;
+    if (valid && walk_n > 0) { nc = __ldg(mysel); nw = __ldg(myw) * kLog2e; }
+    if (valid && walk_n > 1) { nc2 = __ldg(mysel + 1); nw2 = __ldg(myw + 1) * kLog2e; }
     ChunkIter it;
     it.init(bitmap, c0, n_own);
     bool ok = true;
     for (int i = 0; i < n_steps; ++i) {
       const int c = it.next();
-      const int sb = i & 1;
-      ok = mbar_wait(&bars->s_full[sb], (i >> 1) & 1, abort_flag);
+      ok = mbar_wait(&bars->s_full, i & 1, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       float x[64];
       {
         float (&x0)[32] = *reinterpret_cast<float (*)[32]>(&x[0]);
         float (&x1)[32] = *reinterpret_cast<float (*)[32]>(&x[32]);
-        tmem_ld32(s_tmem[sb] + lane_off, x0);
-        tmem_ld32(s_tmem[sb] + lane_off + 32, x1);
+        tmem_ld32(s_tmem + lane_off, x0);
+        tmem_ld32(s_tmem + lane_off + 32, x1);
         tmem_wait_ld();
       }
       tc_fence_before();
-      mbar_arrive(&bars->s_empty[sb]);
+      mbar_arrive(&bars->s_free);
 
       // does this row attend chunk c, and with which logit?
       int kind = 0;  // 0 none, 1 own, 2 selected
@@ -340,34 +350,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           kind = 2;
           logit2 = nw;
           ++ptr;
-          if (ptr < walk_n) {
-            nc = __ldg(mysel + ptr);
-            nw = __ldg(myw + ptr) * kLog2e;
+          nc = nc2;
+          nw = nw2;
+          if (ptr + 1 < walk_n) {
+            nc2 = __ldg(mysel + ptr + 1);
+            nw2 = __ldg(myw + ptr + 1) * kLog2e;
           }
         }
       }
       uint32_t pk[32];
       if (kind != 0) {
-        const int jmax = (kind == 1) ? (t - c * kChunk) : (kChunk - 1);
-        float m = -INFINITY;
+        if (kind == 1) {  // causal keys of the own chunk
+          const int jmax = t - c * kChunk;
+#pragma unroll
+          for (int j = 0; j < 64; ++j) x[j] = (j <= jmax) ? x[j] : -INFINITY;
+        }
+        float mx[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) mx[j] = fmaxf(fmaxf(x[j], x[j + 16]), fmaxf(x[j + 32], x[j + 48]));
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+          for (int j = 0; j < w; ++j) mx[j] = fmaxf(mx[j], mx[j + w]);
+        const float m2 = mx[0] * scale2;
+        float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
-          x[j] = (j <= jmax) ? x[j] * scale2 : -INFINITY;
-          m = fmaxf(m, x[j]);
+          x[j] = ex2_approx(fmaf(x[j], scale2, -m2));
+          ls[j & 3] += x[j];
         }
-        float l = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          x[j] = exp2f(x[j] - m);
-          l += x[j];
-        }
+        const float l = (ls[0] + ls[1]) + (ls[2] + ls[3]);
         float sc;
         if (kind == 1) {
-          lse2_own = m + __log2f(l);
+          lse2_own = m2 + __log2f(l);
           M2 = fmaxf(lse2_own, wmax2);
-          sc = exp2f(m - M2);
+          sc = ex2_approx(m2 - M2);
         } else {
-          sc = exp2f(logit2 - M2) / l;
+          sc = ex2_approx(logit2 - M2) / l;
         }
 #pragma unroll
         for (int j = 0; j < 32; ++j) pk[j] = pack_bf16(x[2 * j] * sc, x[2 * j + 1] * sc);
@@ -375,21 +394,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 32; ++j) pk[j] = 0u;
       }
-      if (i >= 2) {
-        ok = mbar_wait(&bars->p_empty[sb], ((i >> 1) - 1) & 1, abort_flag);
+      // P is single-buffered: the previous chunk's PV product must be done
+      if (i >= 1) {
+        ok = mbar_wait(&bars->p_free, (i - 1) & 1, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       }
       __syncwarp();  // tcgen05.st is warp-collective
-      tmem_st32(p_tmem[sb] + lane_off, pk);
+      tmem_st32(p_tmem + lane_off, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->p_full[sb]);
+      mbar_arrive(&bars->p_full);
     }
     // ---------------------------------------------------------- epilogue
     if (ok) ok = mbar_wait(&bars->o_full, 0, abort_flag);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
-      const float lsum = exp2f(lse2_own - M2) + sumsel * exp2f(wmax2 - M2);
+      const float lsum = ex2_approx(lse2_own - M2) + sumsel * ex2_approx(wmax2 - M2);
       const float lsum_rounded = tmem_ld1(sum_tmem + lane_off);
       tmem_wait_ld();
       const float inv = 1.0f / lsum_rounded;
@@ -466,7 +486,7 @@ cudaError_t make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t rows, ui
 size_t attn_sm100_smem(int d, int L) {
   const int nwords = ((L + 63) / 64 + 31) / 32 + 1;
   const size_t fixed = d == 64 ? Layout<64>::fixed : Layout<128>::fixed;
-  return fixed + (size_t)nwords * 4 + 1024;
+  return fixed + (size_t)nwords * 4;
 }
 
 cudaError_t attn_sm100(const RowSpec &rs, const void *q, const void *k, const void *v,
