@@ -102,9 +102,15 @@ hils_status do_select(const hils_params *p, const hils::RowSpec &rs, const void 
                       cudaStream_t st) {
   // bf16 prefill scores on the tensor cores; fp32 and the decode row on the CUDA cores
   const bool tc = p->dtype == HILS_BF16 && rs.t_first == 0 && rs.t_count == rs.L;
-  cudaError_t e = tc ? hils::select_sm100(rs, q, lmk, sel, w, lse_lmk, err, st)
-                     : hils::select_simt(rs, p->dtype == HILS_BF16, q, lmk, sel, w, lse_lmk, st);
-  g_launches += 1;
+  int n = 0;
+  cudaError_t e;
+  if (tc) {
+    e = hils::select_sm100(rs, q, lmk, sel, w, lse_lmk, err, st, &n);
+  } else {
+    e = hils::select_simt(rs, p->dtype == HILS_BF16, q, lmk, sel, w, lse_lmk, st);
+    n = 1;
+  }
+  g_launches += n;
   return e == cudaSuccess ? HILS_OK : cuda_fail(e, "select launch");
 }
 

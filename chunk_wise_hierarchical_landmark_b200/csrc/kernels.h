@@ -33,7 +33,8 @@ size_t attn_sm100_smem(int d, int L);
 
 // tcgen05 landmark scoring + top-k for bf16 prefill (select_sm100.cu)
 cudaError_t select_sm100(const RowSpec &rs, const void *q, const void *lmk, int32_t *sel,
-                         float *w, float *lse_lmk, uint32_t *err, cudaStream_t st);
+                         float *w, float *lse_lmk, uint32_t *err, cudaStream_t st,
+                         int *launches);
 
 }  // namespace hils
 

@@ -7,17 +7,30 @@
 // One CTA = 128 query rows of one (b, hq); two CTAs share an SM.  6 warps:
 //   warp 0     TMA producer: the Q tile into the landmark ring (staging), then
 //              64-landmark tiles of the row block's KV head into a 2-stage ring;
-//   warp 1     TMEM owner, MMA issuer: S = Q Lmk^T (128 x 64 fp32) into one of
-//              two TMEM buffers, with Q as the A operand in tensor memory;
+//   warp 1     TMEM owner, MMA issuer: the seed scores, then S = Q Lmk^T
+//              (128 x 64 fp32) per landmark tile into one of two TMEM buffers,
+//              with Q as the A operand in tensor memory;
 //   warps 2-5  one thread per row (TMEM lane): copy the row's q into tensor
-//              memory, then per 32-candidate block an online log-sum-exp (base
-//              2) and the row's best k keys in shared memory (8 groups of 8
-//              slots, group minima in registers).  A block whose best score
-//              cannot enter is skipped; the first k candidates are appended
-//              without search; qualifying candidates later are staged in shared
-//              memory and inserted one per lane per step, so the 32 rows of a
-//              warp insert together.  Chunks arrive in ascending order, so a
-//              later chunk never wins a tie.
+//              memory, stage the seed landmarks, start the row's top-k from
+//              the seeds, then per 32-candidate block an online log-sum-exp
+//              (base 2) and, when the block's best score can enter, the
+//              insertion of its qualifying candidates (staged in shared memory,
+//              one per lane per step, so the 32 rows of a warp insert
+//              together).  The row's best k keys live in shared memory (8
+//              groups of 8 slots, group minima in registers).
+// Seeds.  Every row's top-k starts from k chunks (the seeds) whose scores an
+// extra MMA computes first: the k-th best seed bounds the row's k-th best
+// score from below (the seeds are candidates too), so the result stays exact
+// and the scan only inserts what beats that bound; seeds are masked out of
+// the scan, and since kept chunks are then not all earlier than the scan
+// position, equal scores are resolved on the full key.  The row tiles run in
+// kLevels launches: tiles of level 0 start from the chunks 0..k-1 (where a
+// plain scan starts), tiles of later levels from the selection of the last
+// row of a tile an earlier level finished (1, 2, 4, ... tiles before them),
+// which adjacent queries largely share.
+// The hot loop is kept small (one 32-candidate block per iteration, the rare
+// paths not unrolled): the kernel is bound by instruction issue, and code
+// that does not fit the instruction caches stalls it.
 // The candidate scores never leave the chip.
 #include <cuda_bf16.h>
 
@@ -35,6 +48,21 @@ constexpr int kTile = 64;     // landmarks per MMA tile (UMMA N)
 constexpr int kStages = 2;
 constexpr int kThreads = 192;
 constexpr int kMaxK = 64;
+// Row tiles run in kLevels launches (levels): with P = 2^(kLevels-1), level 0
+// takes the tiles P*i unseeded and level j >= 1 the tiles at offset P/2^j in
+// periods of P/2^(j-1), each seeded by the tile offset positions earlier
+// (which an earlier level finished).
+#ifndef HILS_SELECT_LEVELS
+#define HILS_SELECT_LEVELS 6
+#endif
+constexpr int kLevels = HILS_SELECT_LEVELS;
+constexpr int kLevelP = 1 << (kLevels - 1);
+__host__ __device__ constexpr int level_period(int lv) { return lv == 0 ? kLevelP : (kLevelP >> (lv - 1)); }
+__host__ __device__ constexpr int level_offset(int lv) { return lv == 0 ? 0 : (kLevelP >> lv); }
+__host__ __device__ inline int level_count(int lv, int ntiles) {
+  const int p = level_period(lv), o = level_offset(lv);
+  return ntiles > o ? (ntiles - o + p - 1) / p : 0;
+}
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -48,13 +76,15 @@ struct SelLayout {
   static constexpr int stage = heap + kMaxK * kRows * 8;     // [32][128] fp32 candidate staging
   static constexpr int bars = stage + 32 * kRows * 4;
   static constexpr int misc = bars + 16 * 8;
-  static constexpr int total = misc + 32;
+  static constexpr int seeds = misc + 32;                     // [kMaxK] int seed chunk ids
+  static constexpr int total = seeds + kMaxK * 4;
   // TMEM columns: Q [0, D/2) as bf16 pairs, S0 [64, 128), S1 [128, 192)
   static constexpr uint32_t kQCol = 0, kSCol = 64, kTmemCols = 256;
 };
 
 struct SelBars {
-  uint64_t q_smem, q_tmem, l_full[kStages], l_empty[kStages], s_full[2], s_empty[2], done;
+  uint64_t q_smem, q_tmem, l_full[kStages], l_empty[kStages], s_full[2], s_empty[2], done,
+      seed_ready, seed_full, seed_read;
 };
 
 // Per-row top-k: kMaxK key slots in shared memory (slot i of the row at
@@ -67,8 +97,7 @@ struct TopK {
   uint32_t gpos;  // 3 bits per group: position of the group's minimum
   uint64_t mn;    // overall minimum (the entry a better key replaces)
   int mg;         // its group
-  int cnt;        // filled slots
-  float thr;      // score of mn once all K slots are filled, -inf before
+  float thr;      // score of mn
 
   __device__ __forceinline__ void rescan(const uint64_t *h, int g, int K) {
     uint64_t x[8];
@@ -77,7 +106,6 @@ struct TopK {
       const int slot = g * 8 + i;
       x[i] = slot < K ? h[slot * kRows] : ~0ull;
     }
-    // tree minimum with positions
     const uint64_t m01 = x[0] <= x[1] ? x[0] : x[1];
     const uint32_t p01 = x[0] <= x[1] ? 0u : 1u;
     const uint64_t m23 = x[2] <= x[3] ? x[2] : x[3];
@@ -115,7 +143,8 @@ struct TopK {
     thr = key_score(mn);
   }
   __device__ __forceinline__ void build(const uint64_t *h, int K) {
-#pragma unroll
+    gpos = 0;
+#pragma unroll 1
     for (int g = 0; g < 8; ++g) rescan(h, g, K);
     overall();
   }
@@ -128,6 +157,16 @@ struct TopK {
   }
 };
 
+// Prefilter bound in the unscaled domain: every a with fl(a * scale) >= thr
+// satisfies a >= prefilter(thr) (the product rounds by at most 2^-24
+// relative; the bound leaves 2^-20 plus an absolute 2^-100).  Candidates that
+// pass are decided exactly on their full key.
+__device__ __forceinline__ float prefilter(float thr, float scale) {
+  if (isinf(thr)) return thr;
+  const float u = __fdiv_rd(thr, scale);
+  return u - fabsf(u) * 0x1p-20f - 0x1p-100f;
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -139,7 +178,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     select_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_l, RowSpec rs,
                         int32_t *__restrict__ sel, float *__restrict__ chunk_w,
-                        float *__restrict__ lse_lmk, uint32_t *__restrict__ err) {
+                        float *__restrict__ lse_lmk, uint32_t *__restrict__ err, int level,
+                        const __nv_bfloat16 *__restrict__ lmk_raw) {
   using Lay = SelLayout<D>;
   // The 128-byte-swizzled tiles need a 1024-byte aligned base; the dynamic
   // shared window starts there (there is no static shared memory), which the
@@ -152,16 +192,22 @@ __global__ void __launch_bounds__(kThreads, 2)
   SelBars *bars = reinterpret_cast<SelBars *>(smem + Lay::bars);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::misc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::misc + 4);
+  volatile int *nseed_slot = reinterpret_cast<volatile int *>(smem + Lay::misc + 8);
+  int *seed_list = reinterpret_cast<int *>(smem + Lay::seeds);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
   const int b = bh / rs.Hq, hq = bh % rs.Hq, hkv = hq / (rs.Hq / rs.Hkv);
+  // this launch's level: tiles offset + i * period, heaviest first
   const int ntiles_rows = (rs.L + kRows - 1) / kRows;
-  const int t0 = (ntiles_rows - 1 - blockIdx.x) * kRows;  // heaviest tiles first
+  const int tile = level_offset(level) +
+                   (level_count(level, ntiles_rows) - 1 - (int)blockIdx.x) * level_period(level);
+  const int t0 = tile * kRows;
   const int L = rs.L, K = rs.topk, C = rs.C;
   const int nlmk = L / C;
   const int t_last = min(t0 + kRows, L) - 1;
   const int n_cand = min(t_last / C, nlmk);  // candidates of the tile's last row
+  const int n_lo = min(t0 / C, nlmk);        // candidates of its first row
   const int n_ltiles = (n_cand + kTile - 1) / kTile;
 
   if (threadIdx.x == 0) {
@@ -176,6 +222,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&bars->s_empty[i], kRows);
     }
     mbar_init(&bars->done, 1);
+    mbar_init(&bars->seed_ready, kRows);
+    mbar_init(&bars->seed_full, 1);
+    mbar_init(&bars->seed_read, kRows);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -187,9 +236,41 @@ __global__ void __launch_bounds__(kThreads, 2)
     tmem_alloc(tmem_slot, Lay::kTmemCols);
     tmem_relinquish();
   }
+  // Seeds: the chunks every row's top-k starts from.  On levels above 0 they
+  // are the selection of the last row of the tile `offset` positions earlier,
+  // used when it is a full, strictly ascending set of that row's candidates
+  // (all of them are candidates of this tile's rows too).  Otherwise they are
+  // the chunks 0 .. min(k, n) - 1, which is where a plain scan would start.
+  if (warp == 0) {
+    int ns = 0;
+    if (n_ltiles > 0) {
+      bool anchored = false;
+      if (level > 0) {
+        const int anchor_t = min((tile - level_offset(level)) * kRows + kRows - 1, L - 1);
+        const int anchor_n = min(anchor_t / C, nlmk);
+        const int32_t *arow = sel + ((size_t)bh * L + anchor_t) * K;
+        bool good = true;
+        for (int i = lane; i < K; i += 32) {
+          const int c = arow[i];
+          const int prev = i > 0 ? arow[i - 1] : -1;
+          good = good && c > prev && c < anchor_n;
+          seed_list[i] = c;
+        }
+        anchored = __all_sync(0xffffffffu, good);
+      }
+      if (anchored) {
+        ns = K;
+      } else {
+        ns = min(K, n_cand);
+        for (int i = lane; i < ns; i += 32) seed_list[i] = i;
+      }
+    }
+    if (lane == 0) *nseed_slot = ns;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  const int ns = *nseed_slot;
   const uint32_t tmem = *tmem_slot;
   const uint32_t q_tmem = tmem + Lay::kQCol;
   const uint32_t s_tmem[2] = {tmem + Lay::kSCol, tmem + Lay::kSCol + kTile};
@@ -222,12 +303,25 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_ltiles > 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kRows, kTile, false, false);
-      const bool ok = mbar_wait(&bars->q_tmem, 0, abort_flag);
+      bool ok = mbar_wait(&bars->q_tmem, 0, abort_flag);
+      // seed scores: S1 = Q * seeds^T (the seed landmark rows, staged by the rows)
+      ok = ok && mbar_wait(&bars->seed_ready, 0, abort_flag);
       tc_fence_after();
+      if (ok) {
+        const uint32_t sd_addr = smem_u32(smem + Lay::stage);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int kb = kk >> 2, kw = kk & 3;
+          const uint64_t bd = smem_desc_sw128(sd_addr + kb * kTile * 128 + kw * 32, 16, 1024);
+          mma_bf16_ts(s_tmem[1], q_tmem + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->seed_full);
+      }
       for (int i = 0; ok && i < n_ltiles; ++i) {
         const int s = i % kStages, sb = i & 1;
         if (!mbar_wait(&bars->l_full[s], (i / kStages) & 1, abort_flag)) break;
         if (i >= 2 && !mbar_wait(&bars->s_empty[sb], ((i >> 1) - 1) & 1, abort_flag)) break;
+        if (i == 1 && !mbar_wait(&bars->seed_read, 0, abort_flag)) break;
         tc_fence_after();
         const uint32_t l_addr = smem_u32(smem + Lay::l0 + s * Lay::kLBytes);
 #pragma unroll
@@ -255,12 +349,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float sc = rs.scale;
     const bool want_lse = lse_lmk != nullptr;
     float m2 = -INFINITY, l = 0.0f;
+    // rows with at most k candidates keep all of them (no search)
+    const int cnt = n_c <= K ? n_c : K;
     TopK tk;
-    tk.cnt = 0;
-    tk.thr = -INFINITY;
-    tk.gpos = 0;
-    tk.mn = 0;
+    tk.thr = INFINITY;
+    tk.mn = ~0ull;
     tk.mg = 0;
+    tk.gpos = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) tk.gmin[i] = ~0ull;
     bool ok = true;
@@ -288,24 +383,61 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       tc_fence_before();
       mbar_arrive(&bars->q_tmem);
+      // stage the seed landmark rows (128-byte swizzled, as a TMA tile would
+      // be); rows past the seed count are zero
+      if (ok) {
+        constexpr int kPieces = D / 8;  // 16-byte pieces per row
+#pragma unroll 1
+        for (int pc = r; pc < kTile * kPieces; pc += kRows) {
+          const int sr = pc / kPieces, col = pc % kPieces, kb = col >> 3, j = col & 7;
+          uint4 v4 = make_uint4(0u, 0u, 0u, 0u);
+          if (sr < ns)
+            v4 = *reinterpret_cast<const uint4 *>(
+                reinterpret_cast<const unsigned char *>(lmk_raw) +
+                ((size_t)(lrow0 + seed_list[sr]) * D + kb * 64 + j * 8) * 2);
+          *reinterpret_cast<uint4 *>(smem + Lay::stage + kb * kTile * 128 + sr * 128 +
+                                     ((j ^ (sr & 7)) << 4)) = v4;
+        }
+      }
+      fence_async_smem();
+      mbar_arrive(&bars->seed_ready);
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->seed_full, 0, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        float sa[2][32];
+        tmem_ld32(s_tmem[1] + lane_off, sa[0]);
+        tmem_ld32(s_tmem[1] + lane_off + 32, sa[1]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars->seed_read);
+        // the row's starting set: the first `cnt` seeds (all seeds when the
+        // row has more than k candidates)
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+          if (j < cnt) slots[j * kRows] = sel_key(sa[j >> 5][j & 31] * sc, seed_list[j]);
+        if (n_c > K) tk.build(slots, K);
+      }
     }
+    float thr_u = prefilter(tk.thr, sc);
+    int sp = 0;  // cursor into the ascending seed list
     for (int i = 0; ok && i < n_ltiles; ++i) {
       const int sb = i & 1;
       ok = mbar_wait(&bars->s_full[sb], (i >> 1) & 1, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      float a2[2][32];
-      tmem_ld32(s_tmem[sb] + lane_off, a2[0]);
-      tmem_ld32(s_tmem[sb] + lane_off + 32, a2[1]);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bars->s_empty[sb]);
-#pragma unroll
+#pragma unroll 1
       for (int blk = 0; blk < 2; ++blk) {
-        float(&a)[32] = a2[blk];
         const int cb = i * kTile + blk * 32;
+        float a[32];
+        tmem_ld32(s_tmem[sb] + lane_off + blk * 32, a);
+        tmem_wait_ld();
+        if (blk == 1) {
+          tc_fence_before();
+          mbar_arrive(&bars->s_empty[sb]);
+        }
+        if (cb >= n_cand) break;
         const int nv = max(0, min(32, n_c - cb));
-        if (nv < 32) {
+        if (cb + 32 > n_lo) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) a[j] = j < nv ? a[j] : -INFINITY;
         }
@@ -329,79 +461,84 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int j = 0; j < 32; ++j) ps[j & 3] += ex2_approx(fmaf(a[j], c2, -m2));
           l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         }
-        const bool fill = nv > 0 && tk.cnt + nv <= K;
-        if (fill) {
-          // fill phase: every candidate is kept; append without search
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j < nv) slots[(tk.cnt + j) * kRows] = sel_key(a[j] * sc, cb + j);
-          tk.cnt += nv;
-          if (tk.cnt == K) tk.build(slots, K);
-        }
-        // candidates that may enter the top-k (the vote below is warp-wide:
-        // every lane reaches it, filling lanes with an empty mask)
+        // candidates that may enter the top-k; seeds are already kept
+        const bool pass = bm >= thr_u;
+        if (!__any_sync(0xffffffffu, pass)) continue;
         uint32_t mask = 0;
-        if (!fill && nv > 0 && (tk.cnt < K || bm * sc > tk.thr)) {
+        if (pass) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            mask |= (j < nv && (tk.cnt < K || a[j] * sc > tk.thr)) ? (1u << j) : 0u;
+          for (int j = 0; j < 32; ++j) mask |= a[j] >= thr_u ? (1u << j) : 0u;
+          while (sp < ns && seed_list[sp] < cb) ++sp;
+          for (int u = sp; u < ns && seed_list[u] < cb + 32; ++u) mask &= ~(1u << (seed_list[u] - cb));
         }
-        if (__any_sync(0xffffffffu, mask != 0)) {
-          if (mask) {
+        if (!__any_sync(0xffffffffu, mask != 0)) continue;
+        if (mask) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) stage[j * kRows] = a[j];
-          }
-          // one candidate per lane per iteration: the lanes insert together
-          while (__any_sync(0xffffffffu, mask != 0)) {
-            if (mask) {
-              const int j = __ffs(mask) - 1;
-              mask &= mask - 1;
-              const float s = stage[j * kRows] * sc;
-              const uint64_t key = sel_key(s, cb + j);
-              if (tk.cnt < K) {
-                slots[tk.cnt * kRows] = key;
-                if (++tk.cnt == K) tk.build(slots, K);
-              } else if (s > tk.thr) {
-                tk.replace(slots, key, K);
-              }
+          for (int j = 0; j < 32; ++j) stage[j * kRows] = a[j];
+        }
+        // one candidate per lane per iteration: the lanes insert together
+        while (__any_sync(0xffffffffu, mask != 0)) {
+          if (mask) {
+            const int j = __ffs(mask) - 1;
+            mask &= mask - 1;
+            const uint64_t key = sel_key(stage[j * kRows] * sc, cb + j);
+            if (key > tk.mn) {
+              tk.replace(slots, key, K);
+              thr_u = prefilter(tk.thr, sc);
             }
           }
         }
       }
     }
+    // ---------------------------------------------------------- epilogue
     if (__all_sync(0xffffffffu, ok) && valid) {
-      // ascending chunk order: insertion sort of the kept keys by chunk id
-      const int cnt = tk.cnt;
-      for (int i = 1; i < cnt; ++i) {
-        const uint64_t x = slots[i * kRows];
-        const int cx = key_chunk(x);
-        int j = i - 1;
-        while (j >= 0 && key_chunk(slots[j * kRows]) > cx) {
-          slots[(j + 1) * kRows] = slots[j * kRows];
-          --j;
+      // ascending chunk order: bitonic sort of the kept keys on their chunk
+      // ids, in place (rows that kept every candidate are in order already;
+      // slots from K up to the power of two hold a chunk id past any real one)
+      if (n_c > K) {
+        int N = 1;
+        while (N < K) N <<= 1;
+        for (int i = K; i < N; ++i) slots[i * kRows] = 0x80000000ull;
+#pragma unroll 1
+        for (int size = 2; size <= N; size <<= 1) {
+#pragma unroll 1
+          for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll 4
+            for (int p = 0; p < N / 2; ++p) {
+              const int i = ((p & ~(stride - 1)) << 1) | (p & (stride - 1));
+              const int j = i | stride;
+              const uint64_t x = slots[i * kRows], y = slots[j * kRows];
+              const bool up = (i & size) == 0;
+              if ((key_chunk(x) > key_chunk(y)) == up) {
+                slots[i * kRows] = y;
+                slots[j * kRows] = x;
+              }
+            }
+          }
         }
-        slots[(j + 1) * kRows] = x;
       }
       const size_t row = (size_t)bh * L + t;
       int32_t *srow = sel + row * K;
       float *wrow = chunk_w + row * K;
       if ((K & 3) == 0) {
+#pragma unroll 1
         for (int i = 0; i < K; i += 4) {
           int4 si;
           float4 wi;
-          int *sp = &si.x;
-          float *wp = &wi.x;
+          int *sp4 = &si.x;
+          float *wp4 = &wi.x;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const bool have = i + u < cnt;
             const uint64_t x = have ? slots[(i + u) * kRows] : 0;
-            sp[u] = have ? key_chunk(x) : -1;
-            wp[u] = have ? key_score(x) : -INFINITY;
+            sp4[u] = have ? key_chunk(x) : -1;
+            wp4[u] = have ? key_score(x) : -INFINITY;
           }
           *reinterpret_cast<int4 *>(srow + i) = si;
           *reinterpret_cast<float4 *>(wrow + i) = wi;
         }
       } else {
+#pragma unroll 1
         for (int i = 0; i < K; ++i) {
           const bool have = i < cnt;
           const uint64_t x = have ? slots[i * kRows] : 0;
@@ -424,7 +561,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 }  // namespace
 
 cudaError_t select_sm100(const RowSpec &rs, const void *q, const void *lmk, int32_t *sel,
-                         float *w, float *lse_lmk, uint32_t *err, cudaStream_t st) {
+                         float *w, float *lse_lmk, uint32_t *err, cudaStream_t st,
+                         int *launches) {
   CUtensorMap tq, tl;
   cudaError_t e;
   const int nlmk = rs.L / rs.C;
@@ -433,19 +571,22 @@ cudaError_t select_sm100(const RowSpec &rs, const void *q, const void *lmk, int3
   if ((e = make_tmap_bf16(&tq, q, qrows, rs.d, kRows)) != cudaSuccess) return e;
   // with no complete chunk the landmark map is never read; point it at q
   if ((e = make_tmap_bf16(&tl, nlmk > 0 ? lmk : q, lrows, rs.d, kTile)) != cudaSuccess) return e;
-  dim3 grid((rs.L + kRows - 1) / kRows, rs.B * rs.Hq);
-  if (rs.d == 64) {
-    const size_t smem = SelLayout<64>::total;
-    auto kern = select_sm100_kernel<64>;
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, st>>>(tq, tl, rs, sel, w, lse_lmk, err);
-  } else {
-    const size_t smem = SelLayout<128>::total;
-    auto kern = select_sm100_kernel<128>;
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, st>>>(tq, tl, rs, sel, w, lse_lmk, err);
-  }
-  return cudaGetLastError();
+  const int ntiles = (rs.L + kRows - 1) / kRows;
+  const __nv_bfloat16 *lraw = static_cast<const __nv_bfloat16 *>(lmk);
+  auto launch = [&](auto kern, size_t smem) -> cudaError_t {
+    cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e2 != cudaSuccess) return e2;
+    for (int lv = 0; lv < kLevels; ++lv) {
+      const int n = level_count(lv, ntiles);
+      if (n == 0) continue;
+      kern<<<dim3(n, rs.B * rs.Hq), kThreads, smem, st>>>(tq, tl, rs, sel, w, lse_lmk, err, lv, lraw);
+      ++*launches;
+      if ((e2 = cudaGetLastError()) != cudaSuccess) return e2;
+    }
+    return cudaSuccess;
+  };
+  if (rs.d == 64) return launch(select_sm100_kernel<64>, SelLayout<64>::total);
+  return launch(select_sm100_kernel<128>, SelLayout<128>::total);
 }
 
 }  // namespace hils
