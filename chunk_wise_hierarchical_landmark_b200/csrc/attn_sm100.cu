@@ -313,11 +313,16 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float scale2 = rs.scale * kLog2e;
     float M2 = 0.0f, lse2_own = 0.0f;
     int ptr = 0;
-    // the row's next two selected chunks (ids and base-2 logits), prefetched
-    int nc = -1, nc2 = -1;
-    float nw = 0.0f, nw2 = 0.0f;
-    if (valid && walk_n > 0) { nc = __ldg(mysel); nw = __ldg(myw) * kLog2e; }
-    if (valid && walk_n > 1) { nc2 = __ldg(mysel + 1); nw2 = __ldg(myw + 1) * kLog2e; }
+    // the row's next four selected chunks (ids and logits), loaded ahead so
+    // that a global load has several steps to land before it is used
+    int qc[4];
+    float qw[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const bool have = valid && u < walk_n;
+      qc[u] = have ? __ldg(mysel + u) : -1;
+      qw[u] = have ? __ldg(myw + u) : 0.0f;
+    }
     ChunkIter it;
     it.init(bitmap, c0, n_own);
     bool ok = true;
@@ -346,16 +351,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         } else if (c == c0 && has_c0) {
           kind = 2;
           logit2 = w_c0;
-        } else if (ptr < walk_n && c == nc) {
+        } else if (ptr < walk_n && c == qc[0]) {
           kind = 2;
-          logit2 = nw;
+          logit2 = qw[0] * kLog2e;
           ++ptr;
-          nc = nc2;
-          nw = nw2;
-          if (ptr + 1 < walk_n) {
-            nc2 = __ldg(mysel + ptr + 1);
-            nw2 = __ldg(myw + ptr + 1) * kLog2e;
-          }
+          qc[0] = qc[1];
+          qc[1] = qc[2];
+          qc[2] = qc[3];
+          qw[0] = qw[1];
+          qw[1] = qw[2];
+          qw[2] = qw[3];
+          const bool have = ptr + 3 < walk_n;
+          qc[3] = have ? __ldg(mysel + ptr + 3) : -1;
+          qw[3] = have ? __ldg(myw + ptr + 3) : 0.0f;
         }
       }
       uint32_t pk[32];

@@ -46,6 +46,7 @@ using namespace sm100;
 constexpr int kRows = 128;
 constexpr int kTile = 64;     // landmarks per MMA tile (UMMA N)
 constexpr int kStages = 2;
+constexpr int kSBufs = 3;     // score tiles in tensor memory
 constexpr int kThreads = 192;
 constexpr int kMaxK = 64;
 // Row tiles run in kLevels launches (levels): with P = 2^(kLevels-1), level 0
@@ -78,12 +79,13 @@ struct SelLayout {
   static constexpr int misc = bars + 16 * 8;
   static constexpr int seeds = misc + 32;                     // [kMaxK] int seed chunk ids
   static constexpr int total = seeds + kMaxK * 4;
-  // TMEM columns: Q [0, D/2) as bf16 pairs, S0 [64, 128), S1 [128, 192)
+  // TMEM columns: Q [0, D/2) as bf16 pairs, S0..S2 [64, 256)
   static constexpr uint32_t kQCol = 0, kSCol = 64, kTmemCols = 256;
+  static_assert(kSCol + kSBufs * kTile <= kTmemCols, "score tiles fit the allocation");
 };
 
 struct SelBars {
-  uint64_t q_smem, q_tmem, l_full[kStages], l_empty[kStages], s_full[2], s_empty[2], done,
+  uint64_t q_smem, q_tmem, l_full[kStages], l_empty[kStages], s_full[kSBufs], s_empty[kSBufs], done,
       seed_ready, seed_full, seed_read;
 };
 
@@ -158,13 +160,103 @@ struct TopK {
 };
 
 // Prefilter bound in the unscaled domain: every a with fl(a * scale) >= thr
-// satisfies a >= prefilter(thr) (the product rounds by at most 2^-24
-// relative; the bound leaves 2^-20 plus an absolute 2^-100).  Candidates that
-// pass are decided exactly on their full key.
-__device__ __forceinline__ float prefilter(float thr, float scale) {
+// satisfies a >= prefilter(thr, 1 / scale).  The product and thr * (1/scale)
+// each round by at most 2^-24 relative; the bound leaves 2^-20 plus an
+// absolute 2^-100.  Candidates that pass are decided exactly on their key.
+__device__ __forceinline__ float prefilter(float thr, float inv_scale) {
   if (isinf(thr)) return thr;
-  const float u = __fdiv_rd(thr, scale);
+  const float u = thr * inv_scale;
   return u - fabsf(u) * 0x1p-20f - 0x1p-100f;
+}
+
+// Writes a row's first cnt kept keys in slot order (ids, logits; -1 / -inf
+// padding up to K).
+__device__ __forceinline__ void write_in_order(const uint64_t *slots, int cnt, int K,
+                                               int32_t *__restrict__ srow,
+                                               float *__restrict__ wrow) {
+  if ((K & 3) == 0) {
+#pragma unroll 1
+    for (int i = 0; i < K; i += 4) {
+      int4 si;
+      float4 wi;
+      int *sp4 = &si.x;
+      float *wp4 = &wi.x;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const bool have = i + u < cnt;
+        const uint64_t x = have ? slots[(i + u) * kRows] : 0;
+        sp4[u] = have ? key_chunk(x) : -1;
+        wp4[u] = have ? key_score(x) : -INFINITY;
+      }
+      *reinterpret_cast<int4 *>(srow + i) = si;
+      *reinterpret_cast<float4 *>(wrow + i) = wi;
+    }
+  } else {
+#pragma unroll 1
+    for (int i = 0; i < K; ++i) {
+      const bool have = i < cnt;
+      const uint64_t x = have ? slots[i * kRows] : 0;
+      srow[i] = have ? key_chunk(x) : -1;
+      wrow[i] = have ? key_score(x) : -INFINITY;
+    }
+  }
+}
+
+// Sorts a full row's K kept keys by chunk id and writes them.  Chunk ids are
+// below 2^25 (L < 2^31, C = 64), so (id << 6 | slot) fits a 32-bit word; a
+// bitonic network of N/2 log N (log N + 1) / 2 min/max pairs sorts N words in
+// registers without branches (words past K sort last).
+template <int N>
+__device__ __forceinline__ void write_sorted(const uint64_t *slots, int K,
+                                             int32_t *__restrict__ srow,
+                                             float *__restrict__ wrow) {
+  uint32_t v[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    const uint32_t lo = i < K ? reinterpret_cast<const uint32_t *>(slots + i * kRows)[0] : 0u;
+    v[i] = i < K ? (((0xFFFFFFFFu - lo) << 6) | (uint32_t)i) : 0xFFFFFFFFu;
+  }
+#pragma unroll
+  for (int size = 2; size <= N; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1)
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const uint32_t x = v[i], y = v[j];
+          const bool up = (i & size) == 0;
+          v[i] = up ? min(x, y) : max(x, y);
+          v[j] = up ? max(x, y) : min(x, y);
+        }
+      }
+  if ((K & 3) == 0) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+      if (i < K) {
+        int4 si;
+        float4 wi;
+        si.x = (int)(v[i] >> 6);
+        si.y = (int)(v[i + 1] >> 6);
+        si.z = (int)(v[i + 2] >> 6);
+        si.w = (int)(v[i + 3] >> 6);
+        wi.x = key_score(slots[(v[i] & 63u) * kRows]);
+        wi.y = key_score(slots[(v[i + 1] & 63u) * kRows]);
+        wi.z = key_score(slots[(v[i + 2] & 63u) * kRows]);
+        wi.w = key_score(slots[(v[i + 3] & 63u) * kRows]);
+        *reinterpret_cast<int4 *>(srow + i) = si;
+        *reinterpret_cast<float4 *>(wrow + i) = wi;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      if (i < K) {
+        srow[i] = (int)(v[i] >> 6);
+        wrow[i] = key_score(slots[(v[i] & 63u) * kRows]);
+      }
+    }
+  }
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -217,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&bars->l_full[s], 1);
       mbar_init(&bars->l_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&bars->s_full[i], 1);
       mbar_init(&bars->s_empty[i], kRows);
     }
@@ -273,7 +365,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int ns = *nseed_slot;
   const uint32_t tmem = *tmem_slot;
   const uint32_t q_tmem = tmem + Lay::kQCol;
-  const uint32_t s_tmem[2] = {tmem + Lay::kSCol, tmem + Lay::kSCol + kTile};
+  const uint32_t s_tmem0 = tmem + Lay::kSCol;  // score tile sb at s_tmem0 + sb * kTile
+  const uint32_t seed_tmem = s_tmem0 + (kSBufs - 1) * kTile;  // free until tile kSBufs - 1
   const int lrow0 = (b * rs.Hkv + hkv) * nlmk;
 
   if (warp == 0) {
@@ -313,22 +406,22 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int kk = 0; kk < D / 16; ++kk) {
           const int kb = kk >> 2, kw = kk & 3;
           const uint64_t bd = smem_desc_sw128(sd_addr + kb * kTile * 128 + kw * 32, 16, 1024);
-          mma_bf16_ts(s_tmem[1], q_tmem + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
+          mma_bf16_ts(seed_tmem, q_tmem + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars->seed_full);
       }
       for (int i = 0; ok && i < n_ltiles; ++i) {
-        const int s = i % kStages, sb = i & 1;
+        const int s = i % kStages, sb = i % kSBufs;
         if (!mbar_wait(&bars->l_full[s], (i / kStages) & 1, abort_flag)) break;
-        if (i >= 2 && !mbar_wait(&bars->s_empty[sb], ((i >> 1) - 1) & 1, abort_flag)) break;
-        if (i == 1 && !mbar_wait(&bars->seed_read, 0, abort_flag)) break;
+        if (i >= kSBufs && !mbar_wait(&bars->s_empty[sb], ((i / kSBufs) - 1) & 1, abort_flag)) break;
+        if (i == kSBufs - 1 && !mbar_wait(&bars->seed_read, 0, abort_flag)) break;
         tc_fence_after();
         const uint32_t l_addr = smem_u32(smem + Lay::l0 + s * Lay::kLBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int kb = kk >> 2, kw = kk & 3;
           const uint64_t bd = smem_desc_sw128(l_addr + kb * kTile * 128 + kw * 32, 16, 1024);
-          mma_bf16_ts(s_tmem[sb], q_tmem + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
+          mma_bf16_ts((s_tmem0 + sb * kTile), q_tmem + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars->s_full[sb]);
         mma_commit(&bars->l_empty[s]);
@@ -405,8 +498,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (ok) {
         tc_fence_after();
         float sa[2][32];
-        tmem_ld32(s_tmem[1] + lane_off, sa[0]);
-        tmem_ld32(s_tmem[1] + lane_off + 32, sa[1]);
+        tmem_ld32(seed_tmem + lane_off, sa[0]);
+        tmem_ld32(seed_tmem + lane_off + 32, sa[1]);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&bars->seed_read);
@@ -418,18 +511,20 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (n_c > K) tk.build(slots, K);
       }
     }
-    float thr_u = prefilter(tk.thr, sc);
+    const float inv_sc = 1.0f / sc;
+    float thr_u = prefilter(tk.thr, inv_sc);
     int sp = 0;  // cursor into the ascending seed list
+    int next_seed = ns > 0 ? seed_list[0] : INT_MAX;
     for (int i = 0; ok && i < n_ltiles; ++i) {
-      const int sb = i & 1;
-      ok = mbar_wait(&bars->s_full[sb], (i >> 1) & 1, abort_flag);
+      const int sb = i % kSBufs;
+      ok = mbar_wait(&bars->s_full[sb], (i / kSBufs) & 1, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll 1
       for (int blk = 0; blk < 2; ++blk) {
         const int cb = i * kTile + blk * 32;
         float a[32];
-        tmem_ld32(s_tmem[sb] + lane_off + blk * 32, a);
+        tmem_ld32((s_tmem0 + sb * kTile) + lane_off + blk * 32, a);
         tmem_wait_ld();
         if (blk == 1) {
           tc_fence_before();
@@ -466,10 +561,17 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!__any_sync(0xffffffffu, pass)) continue;
         uint32_t mask = 0;
         if (pass) {
+          uint32_t mq[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-          for (int j = 0; j < 32; ++j) mask |= a[j] >= thr_u ? (1u << j) : 0u;
-          while (sp < ns && seed_list[sp] < cb) ++sp;
-          for (int u = sp; u < ns && seed_list[u] < cb + 32; ++u) mask &= ~(1u << (seed_list[u] - cb));
+          for (int j = 0; j < 32; ++j) mq[j >> 3] |= a[j] >= thr_u ? (1u << j) : 0u;
+          mask = (mq[0] | mq[1]) | (mq[2] | mq[3]);
+        }
+        // the seeds in this block, the same for every row: all lanes walk the
+        // ascending seed list together (seeds of skipped blocks are passed over)
+        while (next_seed < cb + 32) {
+          if (next_seed >= cb) mask &= ~(1u << (next_seed - cb));
+          ++sp;
+          next_seed = sp < ns ? seed_list[sp] : INT_MAX;
         }
         if (!__any_sync(0xffffffffu, mask != 0)) continue;
         if (mask) {
@@ -484,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const uint64_t key = sel_key(stage[j * kRows] * sc, cb + j);
             if (key > tk.mn) {
               tk.replace(slots, key, K);
-              thr_u = prefilter(tk.thr, sc);
+              thr_u = prefilter(tk.thr, inv_sc);
             }
           }
         }
@@ -492,60 +594,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     // ---------------------------------------------------------- epilogue
     if (__all_sync(0xffffffffu, ok) && valid) {
-      // ascending chunk order: bitonic sort of the kept keys on their chunk
-      // ids, in place (rows that kept every candidate are in order already;
-      // slots from K up to the power of two hold a chunk id past any real one)
-      if (n_c > K) {
-        int N = 1;
-        while (N < K) N <<= 1;
-        for (int i = K; i < N; ++i) slots[i * kRows] = 0x80000000ull;
-#pragma unroll 1
-        for (int size = 2; size <= N; size <<= 1) {
-#pragma unroll 1
-          for (int stride = size >> 1; stride > 0; stride >>= 1) {
-#pragma unroll 4
-            for (int p = 0; p < N / 2; ++p) {
-              const int i = ((p & ~(stride - 1)) << 1) | (p & (stride - 1));
-              const int j = i | stride;
-              const uint64_t x = slots[i * kRows], y = slots[j * kRows];
-              const bool up = (i & size) == 0;
-              if ((key_chunk(x) > key_chunk(y)) == up) {
-                slots[i * kRows] = y;
-                slots[j * kRows] = x;
-              }
-            }
-          }
-        }
-      }
       const size_t row = (size_t)bh * L + t;
       int32_t *srow = sel + row * K;
       float *wrow = chunk_w + row * K;
-      if ((K & 3) == 0) {
-#pragma unroll 1
-        for (int i = 0; i < K; i += 4) {
-          int4 si;
-          float4 wi;
-          int *sp4 = &si.x;
-          float *wp4 = &wi.x;
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const bool have = i + u < cnt;
-            const uint64_t x = have ? slots[(i + u) * kRows] : 0;
-            sp4[u] = have ? key_chunk(x) : -1;
-            wp4[u] = have ? key_score(x) : -INFINITY;
-          }
-          *reinterpret_cast<int4 *>(srow + i) = si;
-          *reinterpret_cast<float4 *>(wrow + i) = wi;
-        }
-      } else {
-#pragma unroll 1
-        for (int i = 0; i < K; ++i) {
-          const bool have = i < cnt;
-          const uint64_t x = have ? slots[i * kRows] : 0;
-          srow[i] = have ? key_chunk(x) : -1;
-          wrow[i] = have ? key_score(x) : -INFINITY;
-        }
-      }
+      // ascending chunk order (rows that kept every candidate are in order)
+      if (n_c <= K)
+        write_in_order(slots, cnt, K, srow, wrow);
+      else if (K <= 16)
+        write_sorted<16>(slots, K, srow, wrow);
+      else if (K <= 32)
+        write_sorted<32>(slots, K, srow, wrow);
+      else
+        write_sorted<64>(slots, K, srow, wrow);
       if (want_lse) lse_lmk[row] = n_c > 0 ? (m2 + __log2f(l)) * kLn2 : -INFINITY;
     }
   }
