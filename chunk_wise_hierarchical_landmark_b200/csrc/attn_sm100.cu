@@ -67,8 +67,11 @@ struct Layout {
   static constexpr uint32_t kSCol = 0, kPCol = 64, kSumCol = 96, kOCol = 128, kTmemCols = 256;
 };
 
+// K and V have their own barriers: a K slot frees when its QK^T is done, a V
+// slot only when its PV is, so K can be fetched further ahead.
 struct Bars {
-  uint64_t q, kv_full[kStages], kv_empty[kStages], s_full, s_free, p_full, p_free, o_full, done;
+  uint64_t q, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages], s_full,
+      s_free, p_full, p_free, o_full, done;
 };
 
 struct ChunkIter {
@@ -142,8 +145,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (threadIdx.x == 0) {
     mbar_init(&bars->q, 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->kv_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_free, kRows);
@@ -185,19 +190,66 @@ __global__ void __launch_bounds__(kThreads, 2)
   float wmax2 = -INFINITY, sumsel = 0.0f, w_c0 = 0.0f;
   bool has_c0 = false;
   if (valid) {
-    for (int i = 0; i < K; ++i) {
-      const int c = __ldg(mysel + i);
-      if (c < 0) break;
-      if (c >= own) { report(err, DEV_BAD_INDEX); break; }
-      atomicOr(&bitmap[c >> 5], 1u << (c & 31));
-      wmax2 = fmaxf(wmax2, __ldg(myw + i) * kLog2e);
-      ++nsel;
+    // the row's selection, 16 entries per round with all loads in flight
+    // together: ids ascending with -1 padding at the end, and their logits;
+    // a running maximum / rescaled sum gives sum_c exp(s_c - max) (base 2)
+    int last_c = -1;
+    float last_w2 = 0.0f;
+    bool done = false;
+    for (int i0 = 0; i0 < K && !done; i0 += 16) {
+      int cc[16];
+      float ww[16];
+      if ((K & 3) == 0) {
+#pragma unroll
+        for (int u = 0; u < 16; u += 4) {
+          const bool in = i0 + u < K;
+          const int4 c4 = in ? __ldg(reinterpret_cast<const int4 *>(mysel + i0 + u)) : make_int4(-1, -1, -1, -1);
+          const float4 w4 = in ? __ldg(reinterpret_cast<const float4 *>(myw + i0 + u)) : make_float4(0.f, 0.f, 0.f, 0.f);
+          cc[u] = c4.x; cc[u + 1] = c4.y; cc[u + 2] = c4.z; cc[u + 3] = c4.w;
+          ww[u] = w4.x; ww[u + 1] = w4.y; ww[u + 2] = w4.z; ww[u + 3] = w4.w;
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const bool in = i0 + u < K;
+          cc[u] = in ? __ldg(mysel + i0 + u) : -1;
+          ww[u] = in ? __ldg(myw + i0 + u) : 0.0f;
+        }
+      }
+      float gm = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int c = cc[u];
+        if (done || c < 0) {
+          done = true;
+          cc[u] = -1;
+          continue;
+        }
+        if (c >= own) {
+          report(err, DEV_BAD_INDEX);
+          done = true;
+          cc[u] = -1;
+          continue;
+        }
+        atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+        ww[u] *= kLog2e;
+        gm = fmaxf(gm, ww[u]);
+        last_c = c;
+        last_w2 = ww[u];
+        ++nsel;
+      }
+      if (gm > wmax2) {
+        sumsel *= ex2_approx(wmax2 - gm);
+        wmax2 = gm;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        if (cc[u] >= 0) sumsel += ex2_approx(ww[u] - wmax2);
     }
-    for (int i = 0; i < nsel; ++i) sumsel += ex2_approx(__ldg(myw + i) * kLog2e - wmax2);
     walk_n = nsel;
-    if (own == c0 + 1 && nsel > 0 && __ldg(mysel + nsel - 1) == c0) {
+    if (own == c0 + 1 && nsel > 0 && last_c == c0) {
       has_c0 = true;
-      w_c0 = __ldg(myw + nsel - 1) * kLog2e;
+      w_c0 = last_w2;
       walk_n = nsel - 1;
     }
   }
@@ -230,26 +282,46 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_expect_tx(&bars->q, Lay::kQBytes);
       for (int kb = 0; kb < D / 64; ++kb)
         tma_load_2d(q_s + kb * kRows * 128, &tm_q, &bars->q, kb * 64, bh * L + t0);
-      ChunkIter it;
-      it.init(bitmap, c0, n_own);
-      int issued = 0;
-      for (int i = 0; i < n_steps; ++i) {
-        const int c = it.next();
-        const int s = i % kStages;
-        if (i >= kStages && !mbar_wait(&bars->kv_empty[s], ((i / kStages) - 1) & 1, abort_flag))
-          break;
-        mbar_expect_tx(&bars->kv_full[s], 2 * Lay::kKVBytes);
+      // K runs one step ahead of V in the issue order: K(j + 1) waits only
+      // for QK^T(j - 1), V(j) for PV(j - 2)
+      ChunkIter itk, itv;
+      itk.init(bitmap, c0, n_own);
+      itv.init(bitmap, c0, n_own);
+      int k_issued = 0, v_issued = 0;
+      auto load_k = [&](int j) -> bool {
+        const int c = itk.next();
+        const int s = j % kStages;
+        if (j >= kStages && !mbar_wait(&bars->k_empty[s], ((j / kStages) - 1) & 1, abort_flag))
+          return false;
+        mbar_expect_tx(&bars->k_full[s], Lay::kKVBytes);
         unsigned char *ks = smem + Lay::k0 + s * Lay::kKVBytes;
+        for (int kb = 0; kb < D / 64; ++kb)
+          tma_load_2d(ks + kb * kChunk * 128, &tm_k, &bars->k_full[s], kb * 64, kv_row0 + c * kChunk);
+        ++k_issued;
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        const int c = itv.next();
+        const int s = j % kStages;
+        if (j >= kStages && !mbar_wait(&bars->v_empty[s], ((j / kStages) - 1) & 1, abort_flag))
+          return false;
+        mbar_expect_tx(&bars->v_full[s], Lay::kKVBytes);
         unsigned char *vs = smem + Lay::v0 + s * Lay::kKVBytes;
-        for (int kb = 0; kb < D / 64; ++kb) {
-          tma_load_2d(ks + kb * kChunk * 128, &tm_k, &bars->kv_full[s], kb * 64, kv_row0 + c * kChunk);
-          tma_load_2d(vs + kb * kChunk * 128, &tm_v, &bars->kv_full[s], kb * 64, kv_row0 + c * kChunk);
-        }
-        ++issued;
+        for (int kb = 0; kb < D / 64; ++kb)
+          tma_load_2d(vs + kb * kChunk * 128, &tm_v, &bars->v_full[s], kb * 64, kv_row0 + c * kChunk);
+        ++v_issued;
+        return true;
+      };
+      bool ok = n_steps > 0 ? load_k(0) : true;
+      for (int j = 0; ok && j < n_steps; ++j) {
+        if (j + 1 < n_steps) ok = load_k(j + 1);
+        if (ok) ok = load_v(j);
       }
       // every load issued must land before the CTA may exit
-      for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-        mbar_wait_bounded(&bars->kv_full[i % kStages], (i / kStages) & 1);
+      for (int i = (k_issued > kStages ? k_issued - kStages : 0); i < k_issued; ++i)
+        mbar_wait_bounded(&bars->k_full[i % kStages], (i / kStages) & 1);
+      for (int i = (v_issued > kStages ? v_issued - kStages : 0); i < v_issued; ++i)
+        mbar_wait_bounded(&bars->v_full[i % kStages], (i / kStages) & 1);
       mbar_wait_bounded(&bars->q, 0);
     }
   } else if (warp == 1) {
@@ -262,6 +334,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t q_addr = smem_u32(q_s);
       auto pv = [&](int j) -> bool {
         const int s = j % kStages;
+        if (!mbar_wait(&bars->v_full[s], (j / kStages) & 1, abort_flag)) return false;
         if (!mbar_wait(&bars->p_full, j & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(smem + Lay::v0 + s * Lay::kKVBytes);
@@ -279,14 +352,14 @@ __global__ void __launch_bounds__(kThreads, 2)
           const uint64_t bdesc = smem_desc_sw128(ones_addr + kk * 32, 16, 1024);
           mma_bf16_ts(sum_tmem, p_tmem + kk * 8, bdesc, idesc_sum, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&bars->kv_empty[s]);
+        mma_commit(&bars->v_empty[s]);
         mma_commit(&bars->p_free);
         return true;
       };
       bool ok = mbar_wait(&bars->q, 0, abort_flag);
       for (int i = 0; ok && i < n_steps; ++i) {
         const int s = i % kStages;
-        if (!mbar_wait(&bars->kv_full[s], (i / kStages) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&bars->k_full[s], (i / kStages) & 1, abort_flag)) { ok = false; break; }
         // S is single-buffered: the rows must have read the previous S
         if (i >= 1 && !mbar_wait(&bars->s_free, (i - 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -299,6 +372,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           mma_bf16_ss(s_tmem, a, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars->s_full);
+        mma_commit(&bars->k_empty[s]);
         if (i >= 1 && !pv(i - 1)) { ok = false; break; }
       }
       if (ok) ok = pv(n_steps - 1);
