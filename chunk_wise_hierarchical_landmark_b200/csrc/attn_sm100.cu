@@ -440,8 +440,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           qw[3] = have ? __ldg(myw + ptr + 3) : 0.0f;
         }
       }
+      // Rows of the warp that do not attend chunk c run the same softmax on
+      // their (finite) scores and scale it by 0, so the warp takes one path.
       uint32_t pk[32];
-      if (kind != 0) {
+      if (__any_sync(0xffffffffu, kind != 0)) {
         if (kind == 1) {  // causal keys of the own chunk
           const int jmax = t - c * kChunk;
 #pragma unroll
@@ -467,8 +469,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           lse2_own = m2 + __log2f(l);
           M2 = fmaxf(lse2_own, wmax2);
           sc = ex2_approx(m2 - M2);
-        } else {
+        } else if (kind == 2) {
           sc = ex2_approx(logit2 - M2) / l;
+        } else {
+          sc = 0.0f;
         }
 #pragma unroll
         for (int j = 0; j < 32; ++j) pk[j] = pack_bf16(x[2 * j] * sc, x[2 * j + 1] * sc);
