@@ -457,13 +457,17 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
           for (int j = 0; j < w; ++j) mx[j] = fmaxf(mx[j], mx[j + w]);
         const float m2 = mx[0] * scale2;
-        float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        // elementwise fp32 work on pairs (packed f32x2 FMA / add / multiply)
+        const float2 c2v = make_float2(scale2, scale2), nm2 = make_float2(-m2, -m2);
+        float2 ls[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          x[j] = ex2_approx(fmaf(x[j], scale2, -m2));
-          ls[j & 3] += x[j];
+        for (int j = 0; j < 32; ++j) {
+          const float2 y = __ffma2_rn(make_float2(x[2 * j], x[2 * j + 1]), c2v, nm2);
+          x[2 * j] = ex2_approx(y.x);
+          x[2 * j + 1] = ex2_approx(y.y);
+          ls[j & 1] = __fadd2_rn(ls[j & 1], make_float2(x[2 * j], x[2 * j + 1]));
         }
-        const float l = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        const float l = (ls[0].x + ls[1].x) + (ls[0].y + ls[1].y);
         float sc;
         if (kind == 1) {
           lse2_own = m2 + __log2f(l);
@@ -474,8 +478,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         } else {
           sc = 0.0f;
         }
+        const float2 scv = make_float2(sc, sc);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) pk[j] = pack_bf16(x[2 * j] * sc, x[2 * j + 1] * sc);
+        for (int j = 0; j < 32; ++j) {
+          const float2 pj = __fmul2_rn(make_float2(x[2 * j], x[2 * j + 1]), scv);
+          pk[j] = pack_bf16(pj.x, pj.y);
+        }
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) pk[j] = 0u;

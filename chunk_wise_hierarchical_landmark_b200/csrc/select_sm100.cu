@@ -551,10 +551,15 @@ __global__ void __launch_bounds__(kThreads, 2)
             l *= ex2_approx(m2 - bm2);
             m2 = bm2;
           }
-          float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          // pairs of candidates through packed f32x2 FMA and add
+          const float2 c2v = make_float2(c2, c2), nm2 = make_float2(-m2, -m2);
+          float2 ps[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
-          for (int j = 0; j < 32; ++j) ps[j & 3] += ex2_approx(fmaf(a[j], c2, -m2));
-          l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+          for (int j = 0; j < 16; ++j) {
+            const float2 y = __ffma2_rn(make_float2(a[2 * j], a[2 * j + 1]), c2v, nm2);
+            ps[j & 1] = __fadd2_rn(ps[j & 1], make_float2(ex2_approx(y.x), ex2_approx(y.y)));
+          }
+          l += (ps[0].x + ps[1].x) + (ps[0].y + ps[1].y);
         }
         // candidates that may enter the top-k; seeds are already kept
         const bool pass = bm >= thr_u;
