@@ -136,8 +136,8 @@ def pin_topk_planted_ties(orc):
     """Hand values (tests/golden/hand_cases.json "planted_ties"): with q = e_0
     and landmark first coordinates (0.1, 0.5, 0.5, 0.9, 0.5, 0.2) the top-2 are
     {3, 1} and the top-3 {3, 1, 2}: equal scores go to the lower chunk index;
-    the selection is reported in ascending chunk order [MC "selects top-k
-    chunks"]."""
+    the selection is reported in ascending chunk order ([MC]: the top-k
+    chunks are kept)."""
     g = _golden("planted_ties")
     d, C, L, t = g["d"], g["C"], g["L"], g["row"]
     vals = g["landmark_first_coord"]
