@@ -33,6 +33,13 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
 // (an order-preserving map of the fp32 bits), the lower word orders chunk
 // ids descending, so that among equal scores the lower chunk id ranks first.
 // Adding +0.0f turns -0.0 into +0.0 so that the two zeros tie.
+// Three-input maximum (one sm_100 instruction).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint64_t sel_key(float s, int c) {
   uint32_t b = __float_as_uint(s + 0.0f);
   b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);

@@ -536,15 +536,13 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
           for (int j = 0; j < 32; ++j) a[j] = j < nv ? a[j] : -INFINITY;
         }
-        // block maximum (tree)
-        float mx[16];
+        // block maximum: a tree of three-input maxima (32 -> 11 -> 4 -> 1)
+        float y[11];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) mx[j] = fmaxf(a[j], a[j + 16]);
-#pragma unroll
-        for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-          for (int j = 0; j < w; ++j) mx[j] = fmaxf(mx[j], mx[j + w]);
-        const float bm = mx[0];
+        for (int j = 0; j < 10; ++j) y[j] = max3f(a[3 * j], a[3 * j + 1], a[3 * j + 2]);
+        y[10] = fmaxf(a[30], a[31]);
+        const float bm = max3f(max3f(y[0], y[1], y[2]), max3f(y[3], y[4], y[5]),
+                               max3f(y[6], y[7], max3f(y[8], y[9], y[10])));
         if (want_lse && nv > 0) {
           const float bm2 = bm * c2;
           if (bm2 > m2) {
