@@ -24,6 +24,8 @@
 //   decode_combine grid (B*Hq): partials -> out, lse
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -33,7 +35,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kSlab = 256;       // landmarks per scoring CTA
+constexpr int kGemvThreads = 128; // landmarks per scoring CTA
 constexpr int kChunksPerCta = 4; // union chunks per attention CTA
 constexpr int kMaxG = 8;         // query heads per KV head handled per CTA
 constexpr int kC = 64;
@@ -67,151 +69,257 @@ __device__ __forceinline__ void load8<float>(const float *p, float (&f)[8]) {
   f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
+// 8 consecutive elements through the read-only path, widened to fp32
+template <typename T>
+__device__ __forceinline__ void ldg8(const T *p, float (&f)[8]);
+template <>
+__device__ __forceinline__ void ldg8<__nv_bfloat16>(const __nv_bfloat16 *p, float (&f)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+template <>
+__device__ __forceinline__ void ldg8<float>(const float *p, float (&f)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
 // Bounded wait on a single-use barrier (phase 0); sets *abort on timeout.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort) {
   return mbar_wait(bar, parity, abort);
 }
 
 // ---------------------------------------------------------------------------
+// Landmark logits of the G query heads of one KV head: one thread per
+// landmark, its row streamed from HBM with 16-byte loads all in flight, the
+// scaled queries broadcast from shared memory.
 template <typename T, int D>
-__global__ void __launch_bounds__(256) decode_score_kernel(DecodeSpec ds, const T *__restrict__ q,
-                                                           const T *__restrict__ lmk,
-                                                           uint64_t *__restrict__ part_keys,
-                                                           float2 *__restrict__ part_ml,
-                                                           uint32_t *__restrict__ err) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  T *slab = reinterpret_cast<T *>(smem);                          // [kSlab][D]
-  float *qs = reinterpret_cast<float *>(smem + kSlab * D * sizeof(T));  // [G][D]
-  uint64_t *keys = reinterpret_cast<uint64_t *>(qs + kMaxG * D);  // [G][kSlab]
-  float *red = reinterpret_cast<float *>(keys + kMaxG * kSlab);   // [8 warps][G]
-  __shared__ uint64_t bar;
-  __shared__ int abort_flag;
-
-  const int G = ds.Hq / ds.Hkv, K = ds.topk;
-  const int p = blockIdx.x, bk = blockIdx.y;  // bk = b*Hkv + hkv
+__global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(DecodeSpec ds,
+                                                                  const T *__restrict__ q,
+                                                                  const T *__restrict__ lmk,
+                                                                  float *__restrict__ scores) {
+  __shared__ __align__(16) float qs[kMaxG * D];  // [G][D], scaled
+  const int G = ds.Hq / ds.Hkv;
+  const int bk = blockIdx.y;
   const int b = bk / ds.Hkv, hkv = bk % ds.Hkv;
-  const int n_c = ds.n_c;
-  const int c0 = p * kSlab;
-  const int n = min(kSlab, n_c - c0);
-  const int tid = threadIdx.x;
-  if (tid == 0) {
-    abort_flag = 0;
-    mbar_init(&bar, 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  if (tid == 0) {
-    const uint32_t bytes = (uint32_t)n * D * sizeof(T);
-    mbar_expect_tx(&bar, bytes);
-    const T *src = lmk + ((size_t)bk * ds.nlmk + c0) * D;
-    // bulk copies of at most 64 KB each
-    for (uint32_t off = 0; off < bytes; off += 65536u)
-      bulk_g2s(reinterpret_cast<unsigned char *>(slab) + off,
-               reinterpret_cast<const unsigned char *>(src) + off, min(65536u, bytes - off), &bar);
-  }
-  for (int i = tid; i < G * D; i += blockDim.x) {
+  for (int i = threadIdx.x; i < G * D; i += kGemvThreads) {
     const int g = i / D, e = i % D;
     qs[i] = to_f(q[((size_t)b * ds.Hq + hkv * G + g) * D + e]) * ds.scale;
   }
   __syncthreads();
-  const bool ok = __syncthreads_and(wait_bar(&bar, 0, &abort_flag));
-  if (!ok && tid == 0) mbar_wait_bounded(&bar, 0);
-  float s[kMaxG];
+  const int c = blockIdx.x * kGemvThreads + threadIdx.x;
+  if (c >= ds.n_c) return;
+  const T *row = lmk + ((size_t)bk * ds.nlmk + c) * D;
+  float a[kMaxG];
 #pragma unroll
-  for (int g = 0; g < kMaxG; ++g) s[g] = -INFINITY;
-  if (ok && tid < n) {
+  for (int g = 0; g < kMaxG; ++g) a[g] = 0.0f;
+  // the row in two halves (registers), each half's loads issued together
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g) s[g] = 0.0f;
-    const T *row = slab + tid * D;
-    for (int cc = 0; cc < D / 8; ++cc) {
-      const int c = (cc + tid) % (D / 8);  // rotated 16-byte column: spreads the banks
-      float f[8];
-      load8<T>(row + c * 8, f);
+  for (int half = 0; half < 2; ++half) {
+    constexpr int H = D / 2;
+    float f[H];
 #pragma unroll
-      for (int g = 0; g < kMaxG; ++g) {
-        if (g < G) {
-          const float4 qa = *reinterpret_cast<const float4 *>(qs + g * D + c * 8);
-          const float4 qb = *reinterpret_cast<const float4 *>(qs + g * D + c * 8 + 4);
-          float a = s[g];
-          a = fmaf(f[0], qa.x, a); a = fmaf(f[1], qa.y, a); a = fmaf(f[2], qa.z, a);
-          a = fmaf(f[3], qa.w, a); a = fmaf(f[4], qb.x, a); a = fmaf(f[5], qb.y, a);
-          a = fmaf(f[6], qb.z, a); a = fmaf(f[7], qb.w, a);
-          s[g] = a;
+    for (int cc = 0; cc < H / 8; ++cc) {
+      float g8[8];
+      ldg8<T>(row + half * H + cc * 8, g8);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) f[cc * 8 + u] = g8[u];
+    }
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) {
+      if (g < G) {
+#pragma unroll
+        for (int e = 0; e < H; e += 4) {
+          const float4 qv = *reinterpret_cast<const float4 *>(qs + g * D + half * H + e);
+          a[g] = fmaf(f[e], qv.x, a[g]);
+          a[g] = fmaf(f[e + 1], qv.y, a[g]);
+          a[g] = fmaf(f[e + 2], qv.z, a[g]);
+          a[g] = fmaf(f[e + 3], qv.w, a[g]);
         }
       }
     }
   }
-  // keys for the per-head sort; slots without a candidate get key 0 (never kept)
-  for (int g = 0; g < G; ++g) keys[g * kSlab + tid] = (tid < n && ok) ? sel_key(s[g], c0 + tid) : 0ull;
-  // per-head (max, sum exp) of the slab
-  const int lane = tid & 31, warp = tid >> 5;
-  for (int g = 0; g < G; ++g) {
-    float m = s[g];
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) red[warp * kMaxG + g] = m;
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g)
+    if (g < G) scores[((size_t)bk * G + g) * ds.n_c + c] = a[g];
+}
+
+// order-preserving 32-bit image of an fp32 score (-0 folded into +0)
+__device__ __forceinline__ uint32_t score_bits(float s) {
+  uint32_t x = __float_as_uint(s + 0.0f);
+  return (x & 0x80000000u) ? ~x : (x | 0x80000000u);
+}
+
+// Block-wide exclusive prefix count of a predicate over the 256 threads, in
+// thread order; *total gets the block's count.  Uses wsum[8] in shared memory.
+__device__ __forceinline__ int block_excl_count(bool pred, int *wsum, int *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t bal = __ballot_sync(0xffffffffu, pred);
+  if (lane == 0) wsum[warp] = __popc(bal);
+  __syncthreads();
+  int before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    const int x = wsum[w];
+    before += w < warp ? x : 0;
+    all += x;
   }
   __syncthreads();
-  float mh[kMaxG];
-  for (int g = 0; g < G; ++g) {
-    float m = -INFINITY;
-    for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w * kMaxG + g]);
-    mh[g] = m;
-  }
+  *total = all;
+  return before + __popc(bal & ((1u << lane) - 1u));
+}
+
+// Exact top-k of one head's landmark logits (s desc, c asc) and their
+// log-sum-exp.  The k-th largest score is found by a radix select on the
+// order-preserving bits (four 8-bit digits, warp-aggregated histograms);
+// the kept chunks are then written in ascending chunk order, the lowest ids
+// among scores equal to the k-th.
+__global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
+                                                          const float *__restrict__ scores,
+                                                          int32_t *__restrict__ sel,
+                                                          float *__restrict__ chunk_w,
+                                                          float *__restrict__ lse_lmk) {
+  __shared__ uint32_t hist[256];
+  __shared__ int wsum[8];
+  __shared__ float red[8];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_need;
+  const int h = blockIdx.x;  // b*Hq + hq
+  const int n = ds.n_c, K = ds.topk;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float *sc = scores + (size_t)h * n;
+  int32_t *srow = sel + (size_t)h * K;
+  float *wrow = chunk_w + (size_t)h * K;
+
+  // log-sum-exp: block maximum, then the sum of exponentials against it
+  float m = -INFINITY;
+  for (int i = tid; i < n; i += 256) m = fmaxf(m, sc[i]);
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[warp] = m;
   __syncthreads();
-  for (int g = 0; g < G; ++g) {
-    float e = (tid < n && ok) ? __expf(s[g] - mh[g]) : 0.0f;
-    for (int o = 16; o; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-    if (lane == 0) red[warp * kMaxG + g] = e;
-  }
+  m = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
   __syncthreads();
-  if (tid < G) {
-    float l = 0.0f;
-    for (int w = 0; w < 8; ++w) l += red[w * kMaxG + tid];
-    part_ml[((size_t)bk * ds.P + p) * G + tid] = make_float2(mh[tid], l);
+  float l = 0.0f;
+  if (n > 0)
+    for (int i = tid; i < n; i += 256) l += __expf(sc[i] - m);
+  for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  if (lane == 0) red[warp] = l;
+  __syncthreads();
+  if (tid == 0 && lse_lmk) {
+    float lt = 0.0f;
+    for (int w = 0; w < 8; ++w) lt += red[w];
+    lse_lmk[h] = n > 0 ? m + __logf(lt) : -INFINITY;
   }
-  // bitonic sort of each head's 256 keys, descending
-  for (int size = 2; size <= kSlab; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      __syncthreads();
-      for (int pr = tid; pr < G * (kSlab / 2); pr += blockDim.x) {
-        const int g = pr / (kSlab / 2), i0 = pr % (kSlab / 2);
-        const int lo = 2 * i0 - (i0 & (stride - 1));
-        const int hi = lo + stride;
-        const bool desc = (lo & size) == 0;
-        uint64_t *kk = keys + g * kSlab;
-        const uint64_t a = kk[lo], c = kk[hi];
-        if ((a < c) == desc) {
-          kk[lo] = c;
-          kk[hi] = a;
+
+  if (n <= K) {
+    // every completed chunk is selected
+    for (int i = tid; i < K; i += 256) {
+      srow[i] = i < n ? i : -1;
+      wrow[i] = i < n ? sc[i] : -INFINITY;
+    }
+    return;
+  }
+  // radix select of the K-th largest key
+  uint32_t prefix = 0;
+  int need = K;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    hist[tid] = 0;
+    __syncthreads();
+    for (int i0 = 0; i0 < n; i0 += 256) {
+      const int i = i0 + tid;
+      uint32_t digit = 256;  // no bin
+      if (i < n) {
+        const uint32_t k = score_bits(sc[i]);
+        if (pass == 0 || (k >> (shift + 8)) == prefix) digit = (k >> shift) & 255u;
+      }
+      const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+      if (digit < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // bins from the top: lane j holds bins 255-8j .. 248-8j
+      uint32_t cnt[8], tot = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        cnt[u] = hist[255 - 8 * lane - u];
+        tot += cnt[u];
+      }
+      uint32_t incl = tot;
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t excl = incl - tot;
+      // the lane whose range holds the need-th largest key
+      if (excl < (uint32_t)need && incl >= (uint32_t)need) {
+        uint32_t cum = excl;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (cum + cnt[u] >= (uint32_t)need && cum < (uint32_t)need) {
+            s_prefix = (prefix << 8) | (uint32_t)(255 - 8 * lane - u);
+            s_need = need - (int)cum;
+          }
+          cum += cnt[u];
         }
       }
     }
+    __syncthreads();
+    prefix = s_prefix;
+    need = s_need;
+    __syncthreads();
   }
-  __syncthreads();
-  for (int i = tid; i < G * K; i += blockDim.x) {
-    const int g = i / K, j = i % K;
-    part_keys[(((size_t)bk * ds.P + p) * G + g) * K + j] = j < kSlab ? keys[g * kSlab + j] : 0ull;
+  // prefix = the K-th largest key T; `need` entries with key T are kept,
+  // the lowest chunk ids first; write in ascending chunk order
+  const uint32_t T = prefix;
+  int base = 0, eq_seen = 0;
+  for (int i0 = 0; i0 < n; i0 += 256) {
+    const int i = i0 + tid;
+    uint32_t k = 0;
+    float v = 0.0f;
+    if (i < n) {
+      v = sc[i];
+      k = score_bits(v);
+    }
+    const bool gt = i < n && k > T, eq = i < n && k == T;
+    int n_eq;
+    const int eq_rank = eq_seen + block_excl_count(eq, wsum, &n_eq);
+    const bool take = gt || (eq && eq_rank < need);
+    int n_take;
+    const int pos = base + block_excl_count(take, wsum, &n_take);
+    if (take && pos < K) {
+      srow[pos] = i;
+      wrow[pos] = v;
+    }
+    base += n_take;
+    eq_seen += n_eq;
   }
-  if (tid == 0 && abort_flag) report(err, DEV_TIMEOUT);
 }
 
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) decode_merge_kernel(DecodeSpec ds,
-                                                           const uint64_t *__restrict__ part_keys,
-                                                           const float2 *__restrict__ part_ml,
-                                                           int32_t *__restrict__ sel,
-                                                           float *__restrict__ chunk_w,
-                                                           float *__restrict__ lse_lmk,
+// The KV head's chunk union: the selections of its G query heads and the own
+// chunk, ascending, with a per-entry mask of the heads that attend it and
+// their logits.
+__global__ void __launch_bounds__(256) decode_union_kernel(DecodeSpec ds,
+                                                           const int32_t *__restrict__ sel,
+                                                           const float *__restrict__ chunk_w,
                                                            int32_t *__restrict__ u_c,
                                                            uint32_t *__restrict__ u_mask,
                                                            float *__restrict__ u_logit,
                                                            int32_t *__restrict__ u_count) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const int G = ds.Hq / ds.Hkv, K = ds.topk, P = ds.P;
+  const int G = ds.Hq / ds.Hkv, K = ds.topk;
   uint64_t *chosen = reinterpret_cast<uint64_t *>(smem);          // [G][K]
   uint32_t *bitmap = reinterpret_cast<uint32_t *>(chosen + G * K);  // [nwords]
   int *prefix = reinterpret_cast<int *>(bitmap + ds.nwords);       // [nwords]
-  int *cursor = prefix + ds.nwords;                                // [G][P]
   __shared__ int total;
   const int bk = blockIdx.x;
   const int b = bk / ds.Hkv, hkv = bk % ds.Hkv;
@@ -219,66 +327,16 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(DecodeSpec ds,
   const int own = ds.own;
 
   for (int i = tid; i < ds.nwords; i += blockDim.x) bitmap[i] = 0;
-  for (int i = tid; i < G * P; i += blockDim.x) cursor[i] = 0;
   __syncthreads();
-  // one warp per head: k-way merge of the P descending slab lists
-  for (int g = warp; g < G; g += blockDim.x / 32) {
-    const uint64_t *lists = part_keys + (size_t)bk * P * G * K;
-    // each lane walks the lists p = lane, lane+32, ...; its candidate is the
-    // best current head among them
-    int *cur = cursor + g * P;
-    int got = 0;
-    for (; got < K; ++got) {
-      uint64_t best = 0;
-      int bestp = -1;
-      for (int pl = lane; pl < P; pl += 32) {
-        if (cur[pl] < K) {
-          const uint64_t x = lists[((size_t)pl * G + g) * K + cur[pl]];
-          if (x > best) { best = x; bestp = pl; }
-        }
-      }
-      uint64_t wbest = best;
-      for (int o = 16; o; o >>= 1) {
-        const uint64_t y = __shfl_xor_sync(0xffffffffu, wbest, o);
-        wbest = y > wbest ? y : wbest;
-      }
-      if (wbest == 0) break;  // no candidate left
-      if (best == wbest && bestp >= 0) ++cur[bestp];  // keys are unique: one lane advances
-      if (lane == 0) chosen[g * K + got] = wbest;
-    }
-    __syncwarp();
-    // ascending chunk order (insertion sort by lane 0; K <= 64)
-    if (lane == 0) {
-      uint64_t *ch = chosen + g * K;
-      for (int i = 1; i < got; ++i) {
-        const uint64_t x = ch[i];
-        int j = i - 1;
-        while (j >= 0 && key_chunk(ch[j]) > key_chunk(x)) { ch[j + 1] = ch[j]; --j; }
-        ch[j + 1] = x;
-      }
-    }
-    __syncwarp();
+  for (int i = tid; i < G * K; i += blockDim.x) {
+    const int g = i / K, j = i % K;
     const size_t hrow = (size_t)b * ds.Hq + hkv * G + g;
-    for (int i = lane; i < K; i += 32) {
-      const bool have = i < got;
-      const uint64_t x = have ? chosen[g * K + i] : 0;
-      sel[hrow * K + i] = have ? key_chunk(x) : -1;
-      chunk_w[hrow * K + i] = have ? key_score(x) : -INFINITY;
-      if (have) atomicOr(&bitmap[key_chunk(x) >> 5], 1u << (key_chunk(x) & 31));
-      if (!have) chosen[g * K + i] = 0;
-    }
-    if (lse_lmk && lane == 0) {
-      float m = -INFINITY;
-      for (int pl = 0; pl < P; ++pl) m = fmaxf(m, part_ml[((size_t)bk * P + pl) * G + g].x);
-      float l = 0.0f;
-      if (m > -INFINITY)
-        for (int pl = 0; pl < P; ++pl) {
-          const float2 ml = part_ml[((size_t)bk * P + pl) * G + g];
-          if (ml.x > -INFINITY) l += ml.y * __expf(ml.x - m);
-        }
-      lse_lmk[hrow] = (m > -INFINITY) ? m + __logf(l) : -INFINITY;
-    }
+    const int c = sel[hrow * K + j];
+    const bool have = c >= 0 && c < ds.n_c;
+    chosen[i] = have ? sel_key(chunk_w[hrow * K + j], c) : 0ull;
+    if (have) atomicOr(&bitmap[c >> 5], 1u << (c & 31));
   }
+  __syncthreads();
   if (tid == 0) atomicOr(&bitmap[own >> 5], 1u << (own & 31));
   __syncthreads();
   // union positions: exclusive prefix of the bitmap popcounts (one warp)
@@ -547,7 +605,7 @@ DecodeSpec decode_spec(int B, int Hq, int Hkv, int N, int d, int topk, float sca
   ds.own = (N - 1) / kC;
   ds.nlmk = N / kC;
   ds.n_c = ds.own;  // completed chunks of the query at N-1 (all of them have a landmark)
-  ds.P = (ds.n_c + kSlab - 1) / kSlab;
+  ds.P = (ds.n_c + kGemvThreads - 1) / kGemvThreads;
   ds.nwords = ((N + kC - 1) / kC + 31) / 32;
   const int G = Hq / Hkv;
   ds.ucap = G * topk + 1;
@@ -561,13 +619,13 @@ size_t decode_workspace_bytes(const DecodeSpec &ds) {
   const int G = ds.Hq / ds.Hkv;
   const size_t BK = (size_t)ds.B * ds.Hkv;
   size_t n = 256;                                          // error word
-  n += al(BK * ds.P * G * ds.topk * sizeof(uint64_t));     // part_keys
-  n += al(BK * ds.P * G * sizeof(float2));                 // part_ml
   n += al(BK * ds.ucap * sizeof(int32_t));                 // u_c
   n += al(BK * ds.ucap * sizeof(uint32_t));                // u_mask
   n += al(BK * ds.ucap * G * sizeof(float));               // u_logit
   n += al(BK * sizeof(int32_t));                           // u_count
-  n += al(BK * ds.Q * G * (2 + ds.d) * sizeof(float));     // attention partials
+  // the landmark logits [B*Hq][n_c] are dead before the attention partials
+  // [B*Hkv][Q][G][2+d] are written: one region holds both
+  n += al(std::max(BK * G * (size_t)ds.n_c, BK * ds.Q * G * (size_t)(2 + ds.d)) * sizeof(float));
   return n;
 }
 
@@ -585,35 +643,32 @@ cudaError_t decode_fwd(const DecodeSpec &ds, bool bf16, const void *q, const voi
     p += al(bytes);
     return r;
   };
-  uint64_t *part_keys = reinterpret_cast<uint64_t *>(take(BK * ds.P * G * ds.topk * 8));
-  float2 *part_ml = reinterpret_cast<float2 *>(take(BK * ds.P * G * sizeof(float2)));
   int32_t *u_c = reinterpret_cast<int32_t *>(take(BK * ds.ucap * 4));
   uint32_t *u_mask = reinterpret_cast<uint32_t *>(take(BK * ds.ucap * 4));
   float *u_logit = reinterpret_cast<float *>(take(BK * ds.ucap * G * 4));
   int32_t *u_count = reinterpret_cast<int32_t *>(take(BK * 4));
-  float *part = reinterpret_cast<float *>(take(BK * ds.Q * G * (2 + ds.d) * 4));
+  float *part = reinterpret_cast<float *>(
+      take(std::max(BK * G * (size_t)ds.n_c, BK * ds.Q * G * (size_t)(2 + ds.d)) * 4));
+  float *scores = part;  // landmark logits, consumed before the partials are written
   const size_t esz = bf16 ? 2 : 4;
   cudaError_t e;
 
   if (ds.P > 0) {
-    const size_t smem = kSlab * ds.d * esz + kMaxG * ds.d * 4 + kMaxG * kSlab * 8 + 8 * kMaxG * 4;
-#define HILS_SCORE(T, DD)                                                                       \
-  do {                                                                                          \
-    auto kern = decode_score_kernel<T, DD>;                                                     \
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e; \
-    kern<<<dim3(ds.P, (unsigned)BK), 256, smem, st>>>(ds, (const T *)q, (const T *)lmk, part_keys, part_ml, err); \
-  } while (0)
-    if (bf16) { if (ds.d == 64) HILS_SCORE(__nv_bfloat16, 64); else HILS_SCORE(__nv_bfloat16, 128); }
-    else { if (ds.d == 64) HILS_SCORE(float, 64); else HILS_SCORE(float, 128); }
-#undef HILS_SCORE
+#define HILS_GEMV(T, DD) \
+  decode_gemv_kernel<T, DD><<<dim3(ds.P, (unsigned)BK), kGemvThreads, 0, st>>>(ds, (const T *)q, (const T *)lmk, scores)
+    if (bf16) { if (ds.d == 64) HILS_GEMV(__nv_bfloat16, 64); else HILS_GEMV(__nv_bfloat16, 128); }
+    else { if (ds.d == 64) HILS_GEMV(float, 64); else HILS_GEMV(float, 128); }
+#undef HILS_GEMV
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++*launches;
   }
+  decode_topk_kernel<<<(unsigned)(ds.B * ds.Hq), 256, 0, st>>>(ds, scores, sel, w, lse_lmk);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  ++*launches;
   {
-    const size_t smem = (size_t)G * ds.topk * 8 + (size_t)ds.nwords * 8 + (size_t)G * ds.P * 4;
-    if ((e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
-    decode_merge_kernel<<<(unsigned)BK, 256, smem, st>>>(ds, part_keys, part_ml, sel, w, lse_lmk,
-                                                         u_c, u_mask, u_logit, u_count);
+    const size_t smem = (size_t)G * ds.topk * 8 + (size_t)ds.nwords * 8;
+    if ((e = cudaFuncSetAttribute(decode_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
+    decode_union_kernel<<<(unsigned)BK, 256, smem, st>>>(ds, sel, w, u_c, u_mask, u_logit, u_count);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++*launches;
   }
