@@ -69,27 +69,6 @@ __device__ __forceinline__ void load8<float>(const float *p, float (&f)[8]) {
   f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
-// 8 consecutive elements through the read-only path, widened to fp32
-template <typename T>
-__device__ __forceinline__ void ldg8(const T *p, float (&f)[8]);
-template <>
-__device__ __forceinline__ void ldg8<__nv_bfloat16>(const __nv_bfloat16 *p, float (&f)[8]) {
-  const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-template <>
-__device__ __forceinline__ void ldg8<float>(const float *p, float (&f)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
-  const float4 b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
-  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-}
-
 // Bounded wait on a single-use barrier (phase 0); sets *abort on timeout.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort) {
   return mbar_wait(bar, parity, abort);
@@ -105,42 +84,53 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(DecodeSpec ds
                                                                   const T *__restrict__ lmk,
                                                                   float *__restrict__ scores) {
   __shared__ __align__(16) float qs[kMaxG * D];  // [G][D], scaled
+  constexpr int kV = 16 / sizeof(T);             // elements per 16-byte load
   const int G = ds.Hq / ds.Hkv;
   const int bk = blockIdx.y;
   const int b = bk / ds.Hkv, hkv = bk % ds.Hkv;
+  const int c = blockIdx.x * kGemvThreads + threadIdx.x;
+  const bool have = c < ds.n_c;
+  // the landmark row's loads go out first, all in flight together, before
+  // the queries are staged
+  uint4 raw[D / kV];
+  const uint4 *row = reinterpret_cast<const uint4 *>(lmk + ((size_t)bk * ds.nlmk + (have ? c : 0)) * D);
+#pragma unroll
+  for (int cc = 0; cc < D / kV; ++cc) raw[cc] = have ? __ldg(row + cc) : make_uint4(0u, 0u, 0u, 0u);
   for (int i = threadIdx.x; i < G * D; i += kGemvThreads) {
     const int g = i / D, e = i % D;
     qs[i] = to_f(q[((size_t)b * ds.Hq + hkv * G + g) * D + e]) * ds.scale;
   }
   __syncthreads();
-  const int c = blockIdx.x * kGemvThreads + threadIdx.x;
-  if (c >= ds.n_c) return;
-  const T *row = lmk + ((size_t)bk * ds.nlmk + c) * D;
+  if (!have) return;
   float a[kMaxG];
 #pragma unroll
   for (int g = 0; g < kMaxG; ++g) a[g] = 0.0f;
-  // the row in two halves (registers), each half's loads issued together
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    constexpr int H = D / 2;
-    float f[H];
+  for (int cc = 0; cc < D / kV; ++cc) {
+    float f[kV];
+    if constexpr (sizeof(T) == 2) {
+      const uint32_t w[4] = {raw[cc].x, raw[cc].y, raw[cc].z, raw[cc].w};
 #pragma unroll
-    for (int cc = 0; cc < H / 8; ++cc) {
-      float g8[8];
-      ldg8<T>(row + half * H + cc * 8, g8);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) f[cc * 8 + u] = g8[u];
+      for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+    } else {
+      f[0] = __uint_as_float(raw[cc].x);
+      f[1] = __uint_as_float(raw[cc].y);
+      f[2] = __uint_as_float(raw[cc].z);
+      f[3] = __uint_as_float(raw[cc].w);
     }
 #pragma unroll
     for (int g = 0; g < kMaxG; ++g) {
       if (g < G) {
 #pragma unroll
-        for (int e = 0; e < H; e += 4) {
-          const float4 qv = *reinterpret_cast<const float4 *>(qs + g * D + half * H + e);
-          a[g] = fmaf(f[e], qv.x, a[g]);
-          a[g] = fmaf(f[e + 1], qv.y, a[g]);
-          a[g] = fmaf(f[e + 2], qv.z, a[g]);
-          a[g] = fmaf(f[e + 3], qv.w, a[g]);
+        for (int u = 0; u < kV; u += 4) {
+          const float4 qv = *reinterpret_cast<const float4 *>(qs + g * D + cc * kV + u);
+          a[g] = fmaf(f[u], qv.x, a[g]);
+          a[g] = fmaf(f[u + 1], qv.y, a[g]);
+          a[g] = fmaf(f[u + 2], qv.z, a[g]);
+          a[g] = fmaf(f[u + 3], qv.w, a[g]);
         }
       }
     }
@@ -156,44 +146,34 @@ __device__ __forceinline__ uint32_t score_bits(float s) {
   return (x & 0x80000000u) ? ~x : (x | 0x80000000u);
 }
 
-// Block-wide exclusive prefix count of a predicate over the 256 threads, in
-// thread order; *total gets the block's count.  Uses wsum[8] in shared memory.
-__device__ __forceinline__ int block_excl_count(bool pred, int *wsum, int *total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t bal = __ballot_sync(0xffffffffu, pred);
-  if (lane == 0) wsum[warp] = __popc(bal);
-  __syncthreads();
-  int before = 0, all = 0;
-#pragma unroll
-  for (int w = 0; w < 8; ++w) {
-    const int x = wsum[w];
-    before += w < warp ? x : 0;
-    all += x;
-  }
-  __syncthreads();
-  *total = all;
-  return before + __popc(bal & ((1u << lane) - 1u));
-}
-
 // Exact top-k of one head's landmark logits (s desc, c asc) and their
 // log-sum-exp.  The k-th largest score is found by a radix select on the
-// order-preserving bits (four 8-bit digits, warp-aggregated histograms);
-// the kept chunks are then written in ascending chunk order, the lowest ids
-// among scores equal to the k-th.
+// order-preserving bits (four 8-bit digits, per-warp histograms); the kept
+// chunks are then written in ascending chunk order, the lowest ids among
+// scores equal to the k-th.
 __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
                                                           const float *__restrict__ scores,
                                                           int32_t *__restrict__ sel,
                                                           float *__restrict__ chunk_w,
-                                                          float *__restrict__ lse_lmk) {
+                                                          float *__restrict__ lse_lmk,
+                                                          int staged) {
+  extern __shared__ __align__(16) float sc_s[];  // the head's logits when staged
+  __shared__ uint32_t hist_w[8 * 256];  // per-warp digit histograms
   __shared__ uint32_t hist[256];
   __shared__ int wsum[8];
   __shared__ float red[8];
-  __shared__ uint32_t s_prefix;
+  __shared__ uint32_t s_prefix, s_bin;
   __shared__ int s_need;
   const int h = blockIdx.x;  // b*Hq + hq
   const int n = ds.n_c, K = ds.topk;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float *sc = scores + (size_t)h * n;
+  if (staged) {
+    // one pass over HBM/L2 with every load in flight; the rest reads shared memory
+    for (int i = tid; i < n; i += 256) sc_s[i] = sc[i];
+    __syncthreads();
+    sc = sc_s;
+  }
   int32_t *srow = sel + (size_t)h * K;
   float *wrow = chunk_w + (size_t)h * K;
 
@@ -227,22 +207,26 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
     }
     return;
   }
-  // radix select of the K-th largest key
+  // radix select of the K-th largest key: per pass a histogram of one 8-bit
+  // digit of the keys that match the digits chosen so far (one histogram per
+  // warp, summed), then warp 0 finds the digit holding the need-th largest
   uint32_t prefix = 0;
   int need = K;
+  uint32_t last_bin = 0;  // keys equal to the final prefix
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    hist[tid] = 0;
+    for (int i = tid; i < 8 * 256; i += 256) hist_w[i] = 0;
     __syncthreads();
-    for (int i0 = 0; i0 < n; i0 += 256) {
-      const int i = i0 + tid;
-      uint32_t digit = 256;  // no bin
-      if (i < n) {
-        const uint32_t k = score_bits(sc[i]);
-        if (pass == 0 || (k >> (shift + 8)) == prefix) digit = (k >> shift) & 255u;
-      }
-      const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-      if (digit < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
+    for (int i = tid; i < n; i += 256) {
+      const uint32_t k = score_bits(sc[i]);
+      if (pass == 0 || (k >> (shift + 8)) == prefix) atomicAdd(&hist_w[warp * 256 + ((k >> shift) & 255u)], 1u);
+    }
+    __syncthreads();
+    {
+      uint32_t sum = 0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) sum += hist_w[w * 256 + tid];
+      hist[tid] = sum;
     }
     __syncthreads();
     if (warp == 0) {
@@ -267,6 +251,7 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
           if (cum + cnt[u] >= (uint32_t)need && cum < (uint32_t)need) {
             s_prefix = (prefix << 8) | (uint32_t)(255 - 8 * lane - u);
             s_need = need - (int)cum;
+            s_bin = cnt[u];
           }
           cum += cnt[u];
         }
@@ -275,32 +260,69 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
     __syncthreads();
     prefix = s_prefix;
     need = s_need;
+    last_bin = s_bin;
     __syncthreads();
   }
-  // prefix = the K-th largest key T; `need` entries with key T are kept,
-  // the lowest chunk ids first; write in ascending chunk order
+  // prefix = the K-th largest key T.  Kept: every key above T and the `need`
+  // lowest chunk ids among the last_bin keys equal to T, written in ascending
+  // chunk order.  Each warp owns a contiguous segment of the chunks; counts
+  // per segment give every warp its output offset, then it writes in order.
   const uint32_t T = prefix;
-  int base = 0, eq_seen = 0;
-  for (int i0 = 0; i0 < n; i0 += 256) {
-    const int i = i0 + tid;
-    uint32_t k = 0;
-    float v = 0.0f;
-    if (i < n) {
-      v = sc[i];
-      k = score_bits(v);
+  const bool all_eq = last_bin == (uint32_t)need;
+  const int seg = (n + 7) / 8;
+  const int lo = warp * seg, hi = min(n, lo + seg);
+  auto key_at = [&](int i) { return score_bits(sc[i]); };
+  int my_eq = 0;
+  if (!all_eq)
+    for (int i0 = lo; i0 < hi; i0 += 32) {
+      const int i = i0 + lane;
+      my_eq += __popc(__ballot_sync(0xffffffffu, i < hi && key_at(i) == T));
     }
-    const bool gt = i < n && k > T, eq = i < n && k == T;
-    int n_eq;
-    const int eq_rank = eq_seen + block_excl_count(eq, wsum, &n_eq);
-    const bool take = gt || (eq && eq_rank < need);
-    int n_take;
-    const int pos = base + block_excl_count(take, wsum, &n_take);
-    if (take && pos < K) {
-      srow[pos] = i;
-      wrow[pos] = v;
+  if (lane == 0) wsum[warp] = my_eq;
+  __syncthreads();
+  int eq_before = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) eq_before += w < warp ? wsum[w] : 0;
+  __syncthreads();
+  // takes per segment
+  int my_take = 0;
+  {
+    int eq_run = eq_before;
+    for (int i0 = lo; i0 < hi; i0 += 32) {
+      const int i = i0 + lane;
+      const uint32_t k = i < hi ? key_at(i) : 0u;
+      const bool gt = i < hi && k > T, eq = i < hi && k == T;
+      const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+      const int rank = eq_run + __popc(eqb & ((1u << lane) - 1u));
+      const bool take = gt || (eq && (all_eq || rank < need));
+      my_take += __popc(__ballot_sync(0xffffffffu, take));
+      eq_run += __popc(eqb);
     }
-    base += n_take;
-    eq_seen += n_eq;
+  }
+  if (lane == 0) wsum[warp] = my_take;
+  __syncthreads();
+  int base = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) base += w < warp ? wsum[w] : 0;
+  {
+    int eq_run = eq_before;
+    for (int i0 = lo; i0 < hi; i0 += 32) {
+      const int i = i0 + lane;
+      const float v = i < hi ? sc[i] : 0.0f;
+      const uint32_t k = i < hi ? score_bits(v) : 0u;
+      const bool gt = i < hi && k > T, eq = i < hi && k == T;
+      const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+      const int rank = eq_run + __popc(eqb & ((1u << lane) - 1u));
+      const bool take = gt || (eq && (all_eq || rank < need));
+      const uint32_t tb = __ballot_sync(0xffffffffu, take);
+      const int pos = base + __popc(tb & ((1u << lane) - 1u));
+      if (take && pos < K) {
+        srow[pos] = i;
+        wrow[pos] = v;
+      }
+      base += __popc(tb);
+      eq_run += __popc(eqb);
+    }
   }
 }
 
@@ -465,15 +487,17 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(DecodeSpec ds, const T
       const int g = pr / kC, j = pr % kC;
       float a = -INFINITY;
       if (((mask >> g) & 1u) && j <= jmax) {
-        a = 0.0f;
+        // four partial sums keep the FMA chains short
+        float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         for (int cc = 0; cc < D / 8; ++cc) {
           const int col = (cc + j) % (D / 8);
           float f[8];
           load8<T>(kt + j * D + col * 8, f);
           const float *qq = qs + g * D + col * 8;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) a = fmaf(f[u], qq[u], a);
+          for (int u = 0; u < 8; ++u) a4[u & 3] = fmaf(f[u], qq[u], a4[u & 3]);
         }
+        a = (a4[0] + a4[1]) + (a4[2] + a4[3]);
       }
       xs[g * kC + j] = a;
     }
@@ -504,7 +528,8 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(DecodeSpec ds, const T
       const int pr = tid + s * 256;
       const int g = pr / e2n, e2 = pr % e2n;
       if (g < G && ((mask >> g) & 1u)) {
-        float o0 = 0.0f, o1 = 0.0f;
+        // two partial sums per output column keep the FMA chains short
+        float o0 = 0.0f, o1 = 0.0f, p0 = 0.0f, p1 = 0.0f;
         for (int j = 0; j <= jmax; ++j) {
           const float pj = xs[g * kC + j];
           float v0, v1;
@@ -517,9 +542,16 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(DecodeSpec ds, const T
             v0 = w.x;
             v1 = w.y;
           }
-          o0 = fmaf(pj, v0, o0);
-          o1 = fmaf(pj, v1, o1);
+          if (j & 1) {
+            p0 = fmaf(pj, v0, p0);
+            p1 = fmaf(pj, v1, p1);
+          } else {
+            o0 = fmaf(pj, v0, o0);
+            o1 = fmaf(pj, v1, o1);
+          }
         }
+        o0 += p0;
+        o1 += p1;
         const float lg = st[g * 4 + 2], l = st[g * 4 + 1];
         float mo = 0.0f, ln = 0.0f;
 #pragma unroll
@@ -662,8 +694,14 @@ cudaError_t decode_fwd(const DecodeSpec &ds, bool bf16, const void *q, const voi
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++*launches;
   }
-  decode_topk_kernel<<<(unsigned)(ds.B * ds.Hq), 256, 0, st>>>(ds, scores, sel, w, lse_lmk);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {
+    // stage the head's logits in shared memory when they fit
+    const size_t tsmem = (size_t)ds.n_c * sizeof(float);
+    const int staged = tsmem <= 160 * 1024 ? 1 : 0;
+    if (staged && (e = cudaFuncSetAttribute(decode_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem)) != cudaSuccess) return e;
+    decode_topk_kernel<<<(unsigned)(ds.B * ds.Hq), 256, staged ? tsmem : 0, st>>>(ds, scores, sel, w, lse_lmk, staged);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   ++*launches;
   {
     const size_t smem = (size_t)G * ds.topk * 8 + (size_t)ds.nwords * 8;
