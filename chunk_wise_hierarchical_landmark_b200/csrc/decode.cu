@@ -69,6 +69,27 @@ __device__ __forceinline__ void load8<float>(const float *p, float (&f)[8]) {
   f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
+// 8 consecutive elements through the read-only path, widened to fp32
+template <typename T>
+__device__ __forceinline__ void ldg8(const T *p, float (&f)[8]);
+template <>
+__device__ __forceinline__ void ldg8<__nv_bfloat16>(const __nv_bfloat16 *p, float (&f)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+template <>
+__device__ __forceinline__ void ldg8<float>(const float *p, float (&f)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
 // Bounded wait on a single-use barrier (phase 0); sets *abort on timeout.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort) {
   return mbar_wait(bar, parity, abort);
@@ -84,53 +105,42 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(DecodeSpec ds
                                                                   const T *__restrict__ lmk,
                                                                   float *__restrict__ scores) {
   __shared__ __align__(16) float qs[kMaxG * D];  // [G][D], scaled
-  constexpr int kV = 16 / sizeof(T);             // elements per 16-byte load
   const int G = ds.Hq / ds.Hkv;
   const int bk = blockIdx.y;
   const int b = bk / ds.Hkv, hkv = bk % ds.Hkv;
-  const int c = blockIdx.x * kGemvThreads + threadIdx.x;
-  const bool have = c < ds.n_c;
-  // the landmark row's loads go out first, all in flight together, before
-  // the queries are staged
-  uint4 raw[D / kV];
-  const uint4 *row = reinterpret_cast<const uint4 *>(lmk + ((size_t)bk * ds.nlmk + (have ? c : 0)) * D);
-#pragma unroll
-  for (int cc = 0; cc < D / kV; ++cc) raw[cc] = have ? __ldg(row + cc) : make_uint4(0u, 0u, 0u, 0u);
   for (int i = threadIdx.x; i < G * D; i += kGemvThreads) {
     const int g = i / D, e = i % D;
     qs[i] = to_f(q[((size_t)b * ds.Hq + hkv * G + g) * D + e]) * ds.scale;
   }
   __syncthreads();
-  if (!have) return;
+  const int c = blockIdx.x * kGemvThreads + threadIdx.x;
+  if (c >= ds.n_c) return;
+  const T *row = lmk + ((size_t)bk * ds.nlmk + c) * D;
   float a[kMaxG];
 #pragma unroll
   for (int g = 0; g < kMaxG; ++g) a[g] = 0.0f;
+  // the row in two halves (registers), each half's loads issued together
 #pragma unroll
-  for (int cc = 0; cc < D / kV; ++cc) {
-    float f[kV];
-    if constexpr (sizeof(T) == 2) {
-      const uint32_t w[4] = {raw[cc].x, raw[cc].y, raw[cc].z, raw[cc].w};
+  for (int half = 0; half < 2; ++half) {
+    constexpr int H = D / 2;
+    float f[H];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-      }
-    } else {
-      f[0] = __uint_as_float(raw[cc].x);
-      f[1] = __uint_as_float(raw[cc].y);
-      f[2] = __uint_as_float(raw[cc].z);
-      f[3] = __uint_as_float(raw[cc].w);
+    for (int cc = 0; cc < H / 8; ++cc) {
+      float g8[8];
+      ldg8<T>(row + half * H + cc * 8, g8);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) f[cc * 8 + u] = g8[u];
     }
 #pragma unroll
     for (int g = 0; g < kMaxG; ++g) {
       if (g < G) {
 #pragma unroll
-        for (int u = 0; u < kV; u += 4) {
-          const float4 qv = *reinterpret_cast<const float4 *>(qs + g * D + cc * kV + u);
-          a[g] = fmaf(f[u], qv.x, a[g]);
-          a[g] = fmaf(f[u + 1], qv.y, a[g]);
-          a[g] = fmaf(f[u + 2], qv.z, a[g]);
-          a[g] = fmaf(f[u + 3], qv.w, a[g]);
+        for (int e = 0; e < H; e += 4) {
+          const float4 qv = *reinterpret_cast<const float4 *>(qs + g * D + half * H + e);
+          a[g] = fmaf(f[e], qv.x, a[g]);
+          a[g] = fmaf(f[e + 1], qv.y, a[g]);
+          a[g] = fmaf(f[e + 2], qv.z, a[g]);
+          a[g] = fmaf(f[e + 3], qv.w, a[g]);
         }
       }
     }
