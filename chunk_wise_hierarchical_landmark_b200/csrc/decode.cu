@@ -492,24 +492,59 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(DecodeSpec ds, const T
     const int jmax = (c == own) ? (t - c * kC) : (kC - 1);
     const T *kt = ks + buf * kC * D;
     const T *vt = vs + buf * kC * D;
-    // logits x[g][j] = scale * <q_g, k_j>
-    for (int pr = tid; pr < G * kC; pr += blockDim.x) {
-      const int g = pr / kC, j = pr % kC;
-      float a = -INFINITY;
-      if (((mask >> g) & 1u) && j <= jmax) {
-        // four partial sums keep the FMA chains short
-        float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        for (int cc = 0; cc < D / 8; ++cc) {
-          const int col = (cc + j) % (D / 8);
-          float f[8];
-          load8<T>(kt + j * D + col * 8, f);
-          const float *qq = qs + g * D + col * 8;
-#pragma unroll
-          for (int u = 0; u < 8; ++u) a4[u & 3] = fmaf(f[u], qq[u], a4[u & 3]);
-        }
-        a = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+    // logits x[g][j] = scale * <q_g, k_j>.  A warp takes one head and 32
+    // keys; each lane holds a D/32 slice of the head's query in registers and
+    // reads the same slice of each key row (a warp reads whole rows, no bank
+    // conflicts), and a reduce-scatter butterfly (31 shuffles) leaves lane l
+    // with the full logit of key l.
+    for (int job = warp; job < 2 * G; job += blockDim.x / 32) {
+      const int g = job >> 1, j0 = (job & 1) * 32;
+      if (!((mask >> g) & 1u)) {
+        xs[g * kC + j0 + lane] = -INFINITY;
+        continue;
       }
-      xs[g * kC + j] = a;
+      constexpr int kPer = D / 32;  // query / key elements per lane
+      float qv[kPer];
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) qv[u] = qs[g * D + lane * kPer + u];
+      float v[32];
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) {
+        const T *kr = kt + (j0 + jj) * D + lane * kPer;
+        float f[kPer];
+        if constexpr (sizeof(T) == 2) {
+          if constexpr (kPer == 4) {
+            const uint2 w = *reinterpret_cast<const uint2 *>(kr);
+            f[0] = __uint_as_float(w.x << 16);
+            f[1] = __uint_as_float(w.x & 0xFFFF0000u);
+            f[2] = __uint_as_float(w.y << 16);
+            f[3] = __uint_as_float(w.y & 0xFFFF0000u);
+          } else {
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(kr);
+            f[0] = __uint_as_float(w << 16);
+            f[1] = __uint_as_float(w & 0xFFFF0000u);
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < kPer; ++u) f[u] = to_f(kr[u]);
+        }
+        float a = 0.0f;
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) a = fmaf(f[u], qv[u], a);
+        v[jj] = a;
+      }
+#pragma unroll
+      for (int sft = 16; sft >= 1; sft >>= 1) {
+        const bool upper = (lane & sft) != 0;
+#pragma unroll
+        for (int i = 0; i < sft; ++i) {
+          const float send = upper ? v[i] : v[i + sft];
+          const float keep = upper ? v[i + sft] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
+        }
+      }
+      const int j = j0 + lane;
+      xs[g * kC + j] = j <= jmax ? v[0] : -INFINITY;
     }
     __syncthreads();
     // per head: m, l over the chunk; probabilities e_j = exp(x_j - m)
