@@ -7,18 +7,18 @@
 //
 // The step is bound by HBM bytes: every landmark key of every (b, kv-head)
 // and the K/V of the chunks the G = Hq/Hkv query heads of a KV head attend.
-// All G heads of a KV head are served from one staged copy of each landmark
-// slab and of each chunk's K/V (bulk asynchronous copies into shared memory),
-// so the union of the heads' chunks crosses HBM once.
+// The landmark rows stream through once for all G heads, and each chunk's
+// K/V is staged once (bulk asynchronous copies into shared memory) for every
+// head that attends it, so the union of the heads' chunks crosses HBM once.
 //
-//   decode_score   grid (P, B*Hkv): slab p of 256 landmarks -> scores of the
-//                  G heads, per-head top-k of the slab (bitonic sort) and
-//                  per-head (max, sum of exp) of the slab
-//   decode_merge   grid (B*Hkv), one warp per head: k-way merge of the P
-//                  sorted slab lists -> sel_idx / chunk_w (ascending chunk
-//                  ids), lse_lmk; then the KV head's chunk union with a
-//                  per-entry head mask and per-head logits
-//   decode_attn    grid (Q, B*Hkv): up to 4 union chunks per CTA, each chunk's
+//   decode_gemv    grid (ceil(n_c/128), B*Hkv): one thread per landmark ->
+//                  the logits of the G heads, into a workspace array
+//   decode_topk    grid (B*Hq): the head's log-sum-exp and exact top-k
+//                  (radix select on the logit bits) -> sel_idx / chunk_w,
+//                  ascending chunk ids, lse_lmk
+//   decode_union   grid (B*Hkv): the KV head's chunk union with a per-entry
+//                  head mask and per-head logits
+//   decode_attn    grid (Q, B*Hkv): up to 16 union chunks per CTA, each chunk's
 //                  K and V staged once; per head an online (max, sum, acc)
 //                  partial over its chunks
 //   decode_combine grid (B*Hq): partials -> out, lse
@@ -36,7 +36,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kGemvThreads = 128; // landmarks per scoring CTA
-constexpr int kChunksPerCta = 4; // union chunks per attention CTA
+constexpr int kChunksPerCta = 16; // union chunks per attention CTA
 constexpr int kMaxG = 8;         // query heads per KV head handled per CTA
 constexpr int kC = 64;
 
