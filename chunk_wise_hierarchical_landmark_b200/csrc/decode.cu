@@ -49,26 +49,6 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       : "memory");
 }
 
-template <typename T>
-__device__ __forceinline__ void load8(const T *p, float (&f)[8]);
-template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *p, float (&f)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4 *>(p);
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-template <>
-__device__ __forceinline__ void load8<float>(const float *p, float (&f)[8]) {
-  const float4 a = reinterpret_cast<const float4 *>(p)[0];
-  const float4 b = reinterpret_cast<const float4 *>(p)[1];
-  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-}
-
 // 8 consecutive elements through the read-only path, widened to fp32
 template <typename T>
 __device__ __forceinline__ void ldg8(const T *p, float (&f)[8]);
@@ -148,6 +128,157 @@ __global__ void __launch_bounds__(kGemvThreads) decode_gemv_kernel(DecodeSpec ds
 #pragma unroll
   for (int g = 0; g < kMaxG; ++g)
     if (g < G) scores[((size_t)bk * G + g) * ds.n_c + c] = a[g];
+}
+
+// Landmark logits on the tensor cores (bf16): per 128-landmark tile one
+// MMA  S = Lmk_tile [128 x d] . Qg^T [d x 16], the G query heads of the KV
+// head zero-padded to 16 rows, scaled after the fp32 accumulation (the same
+// arithmetic as the prefill scoring kernel).  Warp 0 streams the tiles with
+// TMA through a 3-stage ring, warp 1 issues the MMAs into two TMEM
+// accumulators, warps 2-5 (one thread per landmark) write the G logits.
+constexpr int kTcRows = 128;
+constexpr int kTcStages = 3;
+constexpr int kTcN = 16;  // padded head count (UMMA N)
+constexpr int kTcTilesPerCta = 8;
+
+template <int D>
+struct GemvTcLayout {
+  static constexpr int kTileBytes = kTcRows * D * 2;
+  static constexpr int ring = 0;
+  static constexpr int bq = ring + kTcStages * kTileBytes;  // Q^T: [D/64][16 rows][128 B]
+  static constexpr int bars = bq + (D / 64) * kTcN * 128;
+  static constexpr int misc = bars + 16 * 8;
+  static constexpr int total = misc + 16;
+};
+
+struct GemvTcBars {
+  uint64_t full[kTcStages], empty[kTcStages], acc_full[2], acc_empty[2], done;
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    decode_gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_l, DecodeSpec ds,
+                          const __nv_bfloat16 *__restrict__ q, float *__restrict__ scores,
+                          uint32_t *__restrict__ err) {
+  using Lay = GemvTcLayout<D>;
+  // a name of its own: this kernel asks the dynamic window for 1024-byte alignment
+  extern __shared__ __align__(1024) unsigned char smem_tc[];
+  unsigned char *smem = smem_tc;
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) report(err, DEV_BAD_INDEX);
+    return;
+  }
+  GemvTcBars *bars = reinterpret_cast<GemvTcBars *>(smem + Lay::bars);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::misc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::misc + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = ds.Hq / ds.Hkv;
+  const int bk = blockIdx.y, b = bk / ds.Hkv, hkv = bk % ds.Hkv;
+  const int ntiles = (ds.n_c + kTcRows - 1) / kTcRows;
+  const int my_n =
+      ntiles > (int)blockIdx.x ? (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->acc_full[i], 1);
+      mbar_init(&bars->acc_empty[i], kTcRows);
+    }
+    mbar_init(&bars->done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tmap(&tm_l);
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 32);  // two 16-column accumulators
+    tmem_relinquish();
+  }
+  // Q^T tile (K-major, 128-byte swizzle): row g = head g's query, 0 past G
+  for (int i = threadIdx.x; i < kTcN * D; i += blockDim.x) {
+    const int g = i / D, d = i % D;
+    const __nv_bfloat16 val =
+        g < G ? q[((size_t)b * ds.Hq + hkv * G + g) * D + d] : __float2bfloat16(0.0f);
+    const int kb = d >> 6, c = d & 63;
+    const int off = kb * kTcN * 128 + g * 128 + ((((c >> 3) ^ (g & 7))) << 4) + (c & 7) * 2;
+    *reinterpret_cast<__nv_bfloat16 *>(smem + Lay::bq + off) = val;
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < my_n; ++i) {
+        const int tile = blockIdx.x + i * gridDim.x, s = i % kTcStages;
+        if (i >= kTcStages && !mbar_wait(&bars->empty[s], ((i / kTcStages) - 1) & 1, abort_flag))
+          break;
+        mbar_expect_tx(&bars->full[s], Lay::kTileBytes);
+        unsigned char *dst = smem + Lay::ring + s * Lay::kTileBytes;
+        for (int kb = 0; kb < D / 64; ++kb)
+          tma_load_2d(dst + kb * kTcRows * 128, &tm_l, &bars->full[s], kb * 64,
+                      bk * ds.nlmk + tile * kTcRows);
+        ++issued;
+      }
+      for (int i = (issued > kTcStages ? issued - kTcStages : 0); i < issued; ++i)
+        mbar_wait_bounded(&bars->full[i % kTcStages], (i / kTcStages) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kTcRows, kTcN, false, false);
+      const uint32_t bq_addr = smem_u32(smem + Lay::bq);
+      for (int i = 0; i < my_n; ++i) {
+        const int s = i % kTcStages, ab = i & 1;
+        if (!mbar_wait(&bars->full[s], (i / kTcStages) & 1, abort_flag)) break;
+        if (i >= 2 && !mbar_wait(&bars->acc_empty[ab], ((i >> 1) - 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + Lay::ring + s * Lay::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int kb = kk >> 2, kw = kk & 3;
+          const uint64_t ad = smem_desc_sw128(a_addr + kb * kTcRows * 128 + kw * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(bq_addr + kb * kTcN * 128 + kw * 32, 16, 1024);
+          mma_bf16_ss(tmem + ab * kTcN, ad, bd, idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->acc_full[ab]);
+        mma_commit(&bars->empty[s]);
+      }
+      mma_commit(&bars->done);
+      mbar_wait_bounded(&bars->done, 0);
+    }
+  } else {
+    const int r = 32 * (warp & 3) + lane;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    for (int i = 0; i < my_n; ++i) {
+      const int ab = i & 1, tile = blockIdx.x + i * gridDim.x;
+      const bool ok = mbar_wait(&bars->acc_full[ab], (i >> 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      float v[16];
+      tmem_ld16(tmem + ab * kTcN + lane_off, v);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars->acc_empty[ab]);
+      const int c = tile * kTcRows + r;
+      if (c < ds.n_c) {
+#pragma unroll
+        for (int g = 0; g < kTcN; ++g)
+          if (g < G) scores[((size_t)bk * G + g) * ds.n_c + c] = v[g] * ds.scale;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) report(err, DEV_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
+  }
 }
 
 // order-preserving 32-bit image of an fp32 score (-0 folded into +0)
@@ -730,7 +861,23 @@ cudaError_t decode_fwd(const DecodeSpec &ds, bool bf16, const void *q, const voi
   const size_t esz = bf16 ? 2 : 4;
   cudaError_t e;
 
-  if (ds.P > 0) {
+  if (ds.P > 0 && bf16 && G <= kTcN) {
+    CUtensorMap tl;
+    if ((e = make_tmap_bf16(&tl, lmk, (uint64_t)BK * ds.nlmk, ds.d, kTcRows)) != cudaSuccess) return e;
+    const int ntiles = (ds.n_c + kTcRows - 1) / kTcRows;
+    const dim3 grid((unsigned)std::min(ntiles, kTcTilesPerCta), (unsigned)BK);
+#define HILS_GEMV_TC(DD)                                                                        \
+  do {                                                                                          \
+    auto kern = decode_gemv_tc_kernel<DD>;                                                      \
+    const size_t smem = GemvTcLayout<DD>::total;                                                \
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e; \
+    kern<<<grid, 192, smem, st>>>(tl, ds, (const __nv_bfloat16 *)q, scores, err);               \
+  } while (0)
+    if (ds.d == 64) HILS_GEMV_TC(64); else HILS_GEMV_TC(128);
+#undef HILS_GEMV_TC
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ++*launches;
+  } else if (ds.P > 0) {
 #define HILS_GEMV(T, DD) \
   decode_gemv_kernel<T, DD><<<dim3(ds.P, (unsigned)BK), kGemvThreads, 0, st>>>(ds, (const T *)q, (const T *)lmk, scores)
     if (bf16) { if (ds.d == 64) HILS_GEMV(__nv_bfloat16, 64); else HILS_GEMV(__nv_bfloat16, 128); }
