@@ -45,6 +45,14 @@ def test_decode_small(N, dtype, d):
     check_decode(w)
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 2), (6, 3)])
+def test_decode_group_sizes(Hq, Hkv):
+    """G = Hq / Hkv of 1, 8 (the most one decode CTA serves) and 2 with an
+    odd head count."""
+    w = W.DECODE_512K.with_(B=2, Hq=Hq, Hkv=Hkv, L=3000 + Hq, topk=16, seed=400 + Hq)
+    check_decode(w)
+
+
 def test_decode_equals_last_prefill_row():
     """The decode step equals row N-1 of a prefill over the same cache."""
     w = W.PREFILL_128K.with_(Hq=8, Hkv=2, L=1000, topk=8)
