@@ -31,7 +31,7 @@ def _outputs(w, dev):
 
 @pytest.mark.parametrize("w", [
     W.DECODE_512K.with_(B=2, L=3000, topk=16),
-    W.DECODE_512K.with_(B=16, L=524288),          # the full decode workload (26.5 MB of scratch)
+    W.DECODE_512K.with_(B=16, L=524288),          # the full decode workload (17.6 MB of scratch)
 ], ids=["small", "full"])
 def test_noalloc_matches_workspace_decode_twice(w):
     dev = torch.device("cuda")
@@ -56,7 +56,7 @@ def test_noalloc_matches_workspace_decode_twice(w):
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
-    p = hb.make_params(B=64, Hq=32, Hkv=8, L=524288, d=128, topk=64)  # needs ~106 MB of scratch
+    p = hb.make_params(B=64, Hq=32, Hkv=8, L=524288, d=128, topk=64)  # needs ~70 MB of scratch
     fake = ctypes.c_void_p(1 << 20)
     rc = hb.lib().hils_decode_fwd_noalloc(ctypes.byref(p), fake, fake, fake, fake, fake, fake,
                                          None, fake, fake, None)
