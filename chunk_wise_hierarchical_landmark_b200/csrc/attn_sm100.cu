@@ -14,13 +14,13 @@
 //   warp 0     TMA producer: Q tile once, then K_c / V_c of every union chunk
 //              into a 2-stage ring;
 //   warp 1     TMEM owner and MMA issuer (one thread): S = Q K_c^T into TMEM,
-//              then O += P_c V_c and the row sums of P_c (against an all-ones
-//              tile), both reading P from tensor memory;
+//              then O += P_c V_c reading P from tensor memory;
 //   warps 2-5  one thread per row (TMEM lane): chunk softmax, P -> tensor
-//              memory (bf16, two per column), epilogue.
-// S and P are single-buffered: the MMA computes S for the next chunk while
-// the rows turn the current S into P, and P·V for a chunk while the rows work
-// on the next S.
+//              memory (bf16, two per column, over the chunk's own S), the
+//              running sum of the rounded P, epilogue.
+// S is double-buffered: while the rows turn S_j into P_j, S_{j+1} is ready
+// in the other buffer, and S_{j+2} is computed into this one as soon as
+// P_j·V_j has read P_j.
 //
 // Processing order: the tile's own chunks first (later one first), then the
 // rest of the union ascending.  After its own chunk a row knows its largest
@@ -30,9 +30,9 @@
 //   P_j = exp(x_j - M)                               (own chunk)
 // and O = sum_c P_c V_c needs no rescaling.  P is rounded to bf16 for the
 // tensor core; the output is normalised by the sum of the ROUNDED
-// probabilities, which the tensor core accumulates alongside O, so the
-// weights applied to V sum to one exactly: out = O / sum_j bf16(P_j).  lse
-// stays the fp32 value M + log(sum_c exp(s_c - M)).
+// probabilities (accumulated in fp32 by the row threads from the bf16 values
+// they store), so the weights applied to V sum to one: out = O / sum_j
+// bf16(P_j).  lse stays the fp32 value M + log(sum_c exp(s_c - M)).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -58,21 +58,23 @@ struct Layout {
   static constexpr int q = 0;
   static constexpr int k0 = q + kQBytes;
   static constexpr int v0 = k0 + kStages * kKVBytes;
-  static constexpr int ones = v0 + kStages * kKVBytes;  // 16 x 64 bf16 ones (B of the row-sum MMA)
-  static constexpr int bars = ones + 16 * 128;
-  static constexpr int misc = bars + 16 * 8;
+  static constexpr int bars = v0 + kStages * kKVBytes;
+  static constexpr int misc = bars + 24 * 8;
   static constexpr int bitmap = misc + 64;
   static constexpr int fixed = bitmap;  // + bitmap words
-  // TMEM columns: S [0,64), P [64,96) (bf16 pairs), row sums [96,112), O [128,128+D)
-  static constexpr uint32_t kSCol = 0, kPCol = 64, kSumCol = 96, kOCol = 128, kTmemCols = 256;
+  // TMEM columns: S buffers [0,64) and [64,128) (P over the first 32 columns
+  // of its own S buffer, bf16 pairs), O [128,128+D)
+  static constexpr uint32_t kSCol = 0, kOCol = 128, kTmemCols = 256;
 };
 
 // K and V have their own barriers: a K slot frees when its QK^T is done, a V
-// slot only when its PV is, so K can be fetched further ahead.
+// slot only when its PV is, so K can be fetched further ahead.  S buffer b:
+// s_full (QK^T done), p_full (the rows stored P), p_free (PV read P).
 struct Bars {
-  uint64_t q, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages], s_full,
-      s_free, p_full, p_free, o_full, done;
+  uint64_t q, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages], s_full[2],
+      p_full[2], p_free[2], o_full, done;
 };
+static_assert(sizeof(Bars) <= 24 * 8, "barrier area");
 
 struct ChunkIter {
   const uint32_t *bm;
@@ -101,6 +103,17 @@ struct ChunkIter {
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// acc_lo += low bf16 of w, acc_hi += high bf16 of w (each widened exactly
+// to fp32, then one fp32 addition)
+__device__ __forceinline__ void add_bf16x2_f32(float &acc_lo, float &acc_hi, uint32_t w) {
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\t"
+      "add.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(acc_lo), "+f"(acc_hi)
+      : "r"(w));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -150,10 +163,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
-    mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->s_free, kRows);
-    mbar_init(&bars->p_full, kRows);
-    mbar_init(&bars->p_free, 1);
+    for (int b2 = 0; b2 < 2; ++b2) {
+      mbar_init(&bars->s_full[b2], 1);
+      mbar_init(&bars->p_full[b2], kRows);
+      mbar_init(&bars->p_free[b2], 1);
+    }
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->done, 1);
     *abort_flag = 0;
@@ -169,8 +183,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     tmem_relinquish();
   }
   for (int i = threadIdx.x; i < nwords; i += kThreads) bitmap[i] = 0;
-  for (int i = threadIdx.x; i < 16 * 128 / 4; i += kThreads)
-    reinterpret_cast<uint32_t *>(smem + Lay::ones)[i] = 0x3F803F80u;  // bf16 1.0 pairs
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -269,9 +281,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   const int n_steps = *n_steps_slot;
 
-  const uint32_t s_tmem = tmem + Lay::kSCol;
-  const uint32_t p_tmem = tmem + Lay::kPCol;
-  const uint32_t sum_tmem = tmem + Lay::kSumCol;
+  const uint32_t s_tmem = tmem + Lay::kSCol;  // buffer b at s_tmem + 64 b
   const uint32_t o_tmem = tmem + Lay::kOCol;
   unsigned char *q_s = smem + Lay::q;
   const int kv_row0 = (b * rs.Hkv + hkv) * L;
@@ -329,13 +339,31 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kRows, kChunk, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kRows, D, false, true);
-      constexpr uint32_t idesc_sum = idesc_bf16_f32(kRows, 16, false, false);
-      const uint32_t ones_addr = smem_u32(smem + Lay::ones);
       const uint32_t q_addr = smem_u32(q_s);
+      // S_j = Q K_j^T into S buffer j & 1, once K_j has landed and PV_{j-2}
+      // has read P_{j-2} from that buffer
+      auto qk = [&](int j) -> bool {
+        const int s = j % kStages, b2 = j & 1;
+        if (!mbar_wait(&bars->k_full[s], (j / kStages) & 1, abort_flag)) return false;
+        if (j >= 2 && !mbar_wait(&bars->p_free[b2], ((j >> 1) - 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + Lay::k0 + s * Lay::kKVBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int kb = kk >> 2, kw = kk & 3;
+          const uint64_t a = smem_desc_sw128(q_addr + kb * kRows * 128 + kw * 32, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(k_addr + kb * kChunk * 128 + kw * 32, 16, 1024);
+          mma_bf16_ss(s_tmem + 64 * b2, a, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->s_full[b2]);
+        mma_commit(&bars->k_empty[s]);
+        return true;
+      };
+      // O += P_j V_j, P_j read from the first 32 columns of S buffer j & 1
       auto pv = [&](int j) -> bool {
-        const int s = j % kStages;
+        const int s = j % kStages, b2 = j & 1;
         if (!mbar_wait(&bars->v_full[s], (j / kStages) & 1, abort_flag)) return false;
-        if (!mbar_wait(&bars->p_full, j & 1, abort_flag)) return false;
+        if (!mbar_wait(&bars->p_full[b2], (j >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(smem + Lay::v0 + s * Lay::kKVBytes);
 #pragma unroll
@@ -344,38 +372,19 @@ __global__ void __launch_bounds__(kThreads, 2)
           // B = V [64 keys x D] MN-major: 16 keys = 16 rows of 128 bytes;
           // the D axis is split into 64-wide blocks 64*128 bytes apart
           const uint64_t bdesc = smem_desc_sw128(v_addr + kk * 16 * 128, kChunk * 128, 1024);
-          mma_bf16_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        // row sums of the rounded P: P [128 x 64] times ones [64 x 16]
-#pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk) {
-          const uint64_t bdesc = smem_desc_sw128(ones_addr + kk * 32, 16, 1024);
-          mma_bf16_ts(sum_tmem, p_tmem + kk * 8, bdesc, idesc_sum, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(o_tmem, s_tmem + 64 * b2 + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&bars->v_empty[s]);
-        mma_commit(&bars->p_free);
+        mma_commit(&bars->p_free[b2]);
         return true;
       };
       bool ok = mbar_wait(&bars->q, 0, abort_flag);
-      for (int i = 0; ok && i < n_steps; ++i) {
-        const int s = i % kStages;
-        if (!mbar_wait(&bars->k_full[s], (i / kStages) & 1, abort_flag)) { ok = false; break; }
-        // S is single-buffered: the rows must have read the previous S
-        if (i >= 1 && !mbar_wait(&bars->s_free, (i - 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + Lay::k0 + s * Lay::kKVBytes);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int kb = kk >> 2, kw = kk & 3;
-          const uint64_t a = smem_desc_sw128(q_addr + kb * kRows * 128 + kw * 32, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(k_addr + kb * kChunk * 128 + kw * 32, 16, 1024);
-          mma_bf16_ss(s_tmem, a, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars->s_full);
-        mma_commit(&bars->k_empty[s]);
-        if (i >= 1 && !pv(i - 1)) { ok = false; break; }
+      if (ok) ok = qk(0);
+      if (ok && n_steps > 1) ok = qk(1);
+      for (int j = 0; ok && j < n_steps; ++j) {
+        ok = pv(j);
+        if (ok && j + 2 < n_steps) ok = qk(j + 2);
       }
-      if (ok) ok = pv(n_steps - 1);
       if (ok) mma_commit(&bars->o_full);
       // all issued tensor-core work must finish before TMEM is released
       mma_commit(&bars->done);
@@ -400,21 +409,22 @@ __global__ void __launch_bounds__(kThreads, 2)
     ChunkIter it;
     it.init(bitmap, c0, n_own);
     bool ok = true;
+    // sum of the rounded probabilities this row stores (four partial sums)
+    float rsum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     for (int i = 0; i < n_steps; ++i) {
       const int c = it.next();
-      ok = mbar_wait(&bars->s_full, i & 1, abort_flag);
+      const uint32_t sb = s_tmem + 64 * (i & 1) + lane_off;
+      ok = mbar_wait(&bars->s_full[i & 1], (i >> 1) & 1, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       float x[64];
       {
         float (&x0)[32] = *reinterpret_cast<float (*)[32]>(&x[0]);
         float (&x1)[32] = *reinterpret_cast<float (*)[32]>(&x[32]);
-        tmem_ld32(s_tmem + lane_off, x0);
-        tmem_ld32(s_tmem + lane_off + 32, x1);
+        tmem_ld32(sb, x0);
+        tmem_ld32(sb + 32, x1);
         tmem_wait_ld();
       }
-      tc_fence_before();
-      mbar_arrive(&bars->s_free);
 
       // does this row attend chunk c, and with which logit?
       int kind = 0;  // 0 none, 1 own, 2 selected
@@ -474,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           M2 = fmaxf(lse2_own, wmax2);
           sc = ex2_approx(m2 - M2);
         } else if (kind == 2) {
-          sc = ex2_approx(logit2 - M2) / l;
+          sc = __fdividef(ex2_approx(logit2 - M2), l);  // l in [1, 64]
         } else {
           sc = 0.0f;
         }
@@ -483,29 +493,25 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int j = 0; j < 32; ++j) {
           const float2 pj = __fmul2_rn(make_float2(x[2 * j], x[2 * j + 1]), scv);
           pk[j] = pack_bf16(pj.x, pj.y);
+          add_bf16x2_f32(rsum[2 * (j & 1)], rsum[2 * (j & 1) + 1], pk[j]);
         }
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) pk[j] = 0u;
       }
-      // P is single-buffered: the previous chunk's PV product must be done
-      if (i >= 1) {
-        ok = mbar_wait(&bars->p_free, (i - 1) & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      }
+      // P over the S just read (this buffer is the rows' until p_full)
       __syncwarp();  // tcgen05.st is warp-collective
-      tmem_st32(p_tmem + lane_off, pk);
+      tmem_st32(sb, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->p_full);
+      mbar_arrive(&bars->p_full[i & 1]);
     }
     // ---------------------------------------------------------- epilogue
     if (ok) ok = mbar_wait(&bars->o_full, 0, abort_flag);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const float lsum = ex2_approx(lse2_own - M2) + sumsel * ex2_approx(wmax2 - M2);
-      const float lsum_rounded = tmem_ld1(sum_tmem + lane_off);
-      tmem_wait_ld();
+      const float lsum_rounded = (rsum[0] + rsum[2]) + (rsum[1] + rsum[3]);
       const float inv = 1.0f / lsum_rounded;
       __nv_bfloat16 *orow = out + row * D;
 #pragma unroll
