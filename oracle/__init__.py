@@ -18,6 +18,12 @@ which follows the pages on HiLS attention step by step:
   inside the selected chunks) and section "Hardware-efficient kernel": the
   union of the chunks of M adjacent queries.
 
+``gather_pages`` turns a paged KV cache (one chunk of every KV head per page,
+as an inference engine's attention backend receives it; the same page's
+section "Converting existing models" has HiLS served as such a backend) back
+into the dense cache it describes; ``decode_paged`` is the decode step on that
+dense cache.
+
 Every entry point is pinned in ``tests/test_oracle_pins.py`` against closed
 forms, hand-derived values and brute force; none is "parity unpinned".
 
@@ -167,6 +173,14 @@ class Oracle:
         h = np.arange(p.B * p.Hq, dtype=np.int64) if heads is None else heads
         return self.rows(p, q, k, v, lmk, h, nthreads=nthreads, decode=True)
 
+    def decode_paged(self, p: Problem, q, k_pages, v_pages, page_table, lmk, heads=None,
+                     nthreads: int = 0) -> dict:
+        """Decode step over a paged cache: the dense-cache decode of the caches
+        that ``gather_pages`` rebuilds from the pages and the table."""
+        k = gather_pages(k_pages, page_table, p.L)
+        v = gather_pages(v_pages, page_table, p.L)
+        return self.decode(p, q, k, v, lmk, heads, nthreads)
+
     def scores(self, p: Problem, q, lmk, rows, nthreads: int = 0,
                decode: bool = False) -> np.ndarray:
         """Landmark logits of every completed chunk for the rows (numbered as in
@@ -197,6 +211,29 @@ class Oracle:
         return u[:n].copy()
 
 
+def gather_pages(pages, page_table, L: int) -> np.ndarray:
+    """Dense cache [B, Hkv, L, d] from a paged one.
+
+    pages [num_pages, Hkv, C, d] (fp32, or bf16 as raw bits / a bf16 tensor);
+    page_table [B, max_pages] integers.  Token t = c*C + r (r < C) of sequence
+    b and KV head h is row r of KV head h of page page_table[b, c]; only the
+    ceil(L/C) first entries of a table row are read, and rows r with
+    c*C + r >= L are not.  Returns numpy (uint16 bits for bf16 input)."""
+    pg, _ = _as_array(pages)
+    tab = np.asarray(page_table.cpu() if hasattr(page_table, "cpu") else page_table)
+    num_pages, Hkv, C, d = pg.shape
+    B = tab.shape[0]
+    out = np.empty((B, Hkv, L, d), pg.dtype)
+    for b in range(B):
+        for c in range(-(-L // C)):
+            page = int(tab[b, c])
+            if not 0 <= page < num_pages:
+                raise ValueError(f"page table entry ({b}, {c}) = {page} outside the pool")
+            n = min(C, L - c * C)
+            out[b, :, c * C:c * C + n, :] = pg[page, :, :n, :]
+    return out
+
+
 _default = None
 
 
@@ -222,3 +259,7 @@ def union(*a, **kw):
 
 def scores(*a, **kw):
     return default().scores(*a, **kw)
+
+
+def decode_paged(*a, **kw):
+    return default().decode_paged(*a, **kw)

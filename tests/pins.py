@@ -380,6 +380,49 @@ def pin_union_is_set_union(orc):
             assert got.tolist() == sorted(want), (head, g)
 
 
+def pin_paged_decode_is_dense_decode(orc):
+    """A paged cache is another layout of the dense cache: the decode step
+    over pages in shuffled order (with unused pages, unused table columns and
+    the tail of a partial last page all NaN) equals the decode over the dense
+    cache exactly; two sequences sharing every page equal two sequences with
+    identical dense caches."""
+    rng = _rng(37)
+    B, Hq, Hkv, N, d, C, topk = 2, 4, 2, 70, 8, 8, 3
+    npg = -(-N // C)
+    p = Problem(B=B, Hq=Hq, Hkv=Hkv, L=N, d=d, C=C, topk=topk, scale=1 / math.sqrt(d))
+    q = _f32(B, Hq, d, rng=rng)
+    k = _f32(B, Hkv, N, d, rng=rng)
+    v = _f32(B, Hkv, N, d, rng=rng)
+    lmk = _f32(B, Hkv, N // C, d, rng=rng)
+    num_pages = B * npg + 3
+    perm = rng.permutation(num_pages)[:B * npg]
+    table = np.full((B, npg + 2), -1, np.int64)
+    kp = np.full((num_pages, Hkv, C, d), np.nan, np.float32)
+    vp = np.full((num_pages, Hkv, C, d), np.nan, np.float32)
+    for b in range(B):
+        for c in range(npg):
+            page = int(perm[b * npg + c])
+            table[b, c] = page
+            n = min(C, N - c * C)
+            # the page holds [Hkv][C][d]: head-major, the chunk's tokens in order
+            kp[page, :, :n] = k[b, :, c * C:c * C + n]
+            vp[page, :, :n] = v[b, :, c * C:c * C + n]
+    dense = orc.decode(p, q, k, v, lmk)
+    paged = orc.decode_paged(p, q, kp, vp, table, lmk)
+    for key in ("sel", "w", "out", "lse", "lse_lmk", "wfin"):
+        assert np.array_equal(dense[key], paged[key]), key
+    # shared pages: sequence 1 reads sequence 0's pages
+    shared = table.copy()
+    shared[1] = table[0]
+    k2, v2, lmk2 = k.copy(), v.copy(), lmk.copy()
+    k2[1], v2[1], lmk2[1] = k[0], v[0], lmk[0]
+    dense2 = orc.decode(p, q, k2, v2, lmk2)
+    paged2 = orc.decode_paged(p, q, kp, vp, shared, lmk2)
+    for key in ("sel", "out", "lse"):
+        assert np.array_equal(dense2[key], paged2[key]), key
+    assert np.isfinite(paged["out"]).all()
+
+
 ALL_PINS = [
     pin_landmark_logit_and_normaliser,
     pin_topk_planted_ties,
@@ -393,4 +436,5 @@ ALL_PINS = [
     pin_decode_is_last_prefill_row,
     pin_bf16_bits_widen_exactly,
     pin_union_is_set_union,
+    pin_paged_decode_is_dense_decode,
 ]
