@@ -37,7 +37,8 @@ class Params(ctypes.Structure):
 
 _lib = None
 EXPORTS = ["hils_workspace_size", "hils_select", "hils_union_capacity", "hils_union",
-           "hils_attn_fwd", "hils_prefill", "hils_decode_fwd", "hils_decode_fwd_noalloc",
+           "hils_attn_fwd", "hils_prefill", "hils_decode_fwd", "hils_decode_fwd_paged",
+           "hils_decode_fwd_noalloc",
            "hils_status_string", "hils_last_error", "hils_launch_count"]
 
 
@@ -59,9 +60,10 @@ def lib():
         L.hils_attn_fwd.argtypes = [PP, P, P, P, P, P, P, P, P, P, SZ, P]
         L.hils_prefill.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.hils_decode_fwd.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.hils_decode_fwd_paged.argtypes = [PP, P, P, P, I64, P, I, P, P, P, P, P, P, P, SZ, P]
         L.hils_decode_fwd_noalloc.argtypes = [PP, P, P, P, P, P, P, P, P, P, P]
         for f in ("hils_select", "hils_union", "hils_attn_fwd", "hils_prefill", "hils_decode_fwd",
-                  "hils_decode_fwd_noalloc"):
+                  "hils_decode_fwd_paged", "hils_decode_fwd_noalloc"):
             getattr(L, f).restype = I
         L.hils_status_string.argtypes = [I]
         L.hils_status_string.restype = ctypes.c_char_p
@@ -150,6 +152,16 @@ def hils_decode_fwd(p: Params, q, k_cache, v_cache, lmk_k, sel_idx, chunk_w, lse
                                  _ptr(out), _ptr(lse), *_ws_args(ws), _stream(stream)))
 
 
+def hils_decode_fwd_paged(p: Params, q, k_pages, v_pages, page_table, lmk_k, sel_idx, chunk_w,
+                          lse_lmk, out, lse, ws=None, stream=None):
+    """k_pages / v_pages [num_pages, Hkv, C, d]; page_table [B, max_pages] int32."""
+    _check(lib().hils_decode_fwd_paged(ctypes.byref(p), _ptr(q), _ptr(k_pages), _ptr(v_pages),
+                                       int(k_pages.shape[0]), _ptr(page_table),
+                                       int(page_table.shape[1]), _ptr(lmk_k), _ptr(sel_idx),
+                                       _ptr(chunk_w), _ptr(lse_lmk), _ptr(out), _ptr(lse),
+                                       *_ws_args(ws), _stream(stream)))
+
+
 def hils_decode_fwd_noalloc(p: Params, q, k_cache, v_cache, lmk_k, sel_idx, chunk_w, lse_lmk,
                             out, lse, stream=None):
     _check(lib().hils_decode_fwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache),
@@ -217,6 +229,25 @@ def decode(q, k_cache, v_cache, lmk_k, topk, scale=None, debug_checks=False):
     lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
     hils_decode_fwd(p, q, k_cache, v_cache, lmk_k, sel, w, lse_lmk, out, lse,
                     workspace(p, HILS_OP_DECODE, dev))
+    return dict(out=out, lse=lse, sel_idx=sel, chunk_w=w, lse_lmk=lse_lmk)
+
+
+def decode_paged(q, k_pages, v_pages, page_table, lmk_k, N, topk, scale=None,
+                 debug_checks=False):
+    """One decode step over a paged cache (q [B,Hq,d]; pages [num_pages,Hkv,64,d];
+    page_table [B, max_pages] int32; N tokens per sequence): returns
+    dict(out, lse, sel_idx, chunk_w, lse_lmk)."""
+    B, Hq, d = q.shape
+    Hkv = k_pages.shape[1]
+    p = make_params(B, Hq, Hkv, N, d, topk, 64, 64, scale, q.dtype, debug_checks)
+    dev = q.device
+    sel = torch.empty((B, Hq, topk), dtype=torch.int32, device=dev)
+    w = torch.empty((B, Hq, topk), dtype=torch.float32, device=dev)
+    lse_lmk = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    hils_decode_fwd_paged(p, q, k_pages, v_pages, page_table, lmk_k, sel, w, lse_lmk, out, lse,
+                          workspace(p, HILS_OP_DECODE, dev))
     return dict(out=out, lse=lse, sel_idx=sel, chunk_w=w, lse_lmk=lse_lmk)
 
 

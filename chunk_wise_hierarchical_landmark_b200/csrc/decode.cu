@@ -28,6 +28,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "paged.h"
 #include "sm100.cuh"
 
 namespace hils {
@@ -552,6 +553,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) decode_attn_kernel(DecodeSpec ds, const T *__restrict__ q,
                                                           const T *__restrict__ kc,
                                                           const T *__restrict__ vc,
+                                                          const PagedKV pg,
                                                           const int32_t *__restrict__ u_c,
                                                           const uint32_t *__restrict__ u_mask,
                                                           const float *__restrict__ u_logit,
@@ -592,9 +594,22 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(DecodeSpec ds, const T
     const int c = u_c[(size_t)bk * cap + i];
     const int rows = min(kC, ds.N - c * kC);
     const uint32_t bytes = (uint32_t)rows * D * sizeof(T);
+    size_t off = (kvbase + (size_t)c * kC) * D;  // element offset of the chunk's [rows][D] slab
+    if (pg.table) {
+      // paged: the chunk is page table[b][c], its KV head hkv at [page][hkv][C][D]
+      const long long page = pg.table[(size_t)b * pg.max_pages + c];
+      if (page < 0 || page >= pg.num_pages) {
+        // no copy for an entry outside the pool: complete the phase without
+        // bytes (the chunk's logits are then unspecified) and report it
+        report(err, DEV_BAD_INDEX);
+        mbar_expect_tx(&bars[buf], 0);
+        return;
+      }
+      off = ((size_t)page * ds.Hkv + hkv) * kC * D;
+    }
     mbar_expect_tx(&bars[buf], 2 * bytes);
-    bulk_g2s(ks + buf * kC * D, kc + (kvbase + (size_t)c * kC) * D, bytes, &bars[buf]);
-    bulk_g2s(vs + buf * kC * D, vc + (kvbase + (size_t)c * kC) * D, bytes, &bars[buf]);
+    bulk_g2s(ks + buf * kC * D, kc + off, bytes, &bars[buf]);
+    bulk_g2s(vs + buf * kC * D, vc + off, bytes, &bars[buf]);
   };
   if (tid == 0 && i0 < i1) issue(i0, 0);
 
@@ -839,10 +854,11 @@ size_t decode_workspace_bytes(const DecodeSpec &ds) {
 
 size_t decode_max_g() { return kMaxG; }
 
-cudaError_t decode_fwd(const DecodeSpec &ds, bool bf16, const void *q, const void *k,
-                       const void *v, const void *lmk, int32_t *sel, float *w, float *lse_lmk,
-                       void *out, float *lse, void *ws, uint32_t *err, cudaStream_t st,
-                       int *launches) {
+// The five launches of one decode step; pages.table == nullptr: dense caches.
+static cudaError_t decode_run(const DecodeSpec &ds, bool bf16, const void *q, const void *k,
+                              const void *v, const PagedKV &pages, const void *lmk, int32_t *sel,
+                              float *w, float *lse_lmk, void *out, float *lse, void *ws,
+                              uint32_t *err, cudaStream_t st, int *launches) {
   const int G = ds.Hq / ds.Hkv;
   const size_t BK = (size_t)ds.B * ds.Hkv;
   unsigned char *p = static_cast<unsigned char *>(ws) + 256;
@@ -908,7 +924,7 @@ cudaError_t decode_fwd(const DecodeSpec &ds, bool bf16, const void *q, const voi
   do {                                                                                          \
     auto kern = decode_attn_kernel<T, DD>;                                                      \
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e; \
-    kern<<<dim3(ds.Q, (unsigned)BK), 256, smem, st>>>(ds, (const T *)q, (const T *)k, (const T *)v, u_c, u_mask, u_logit, u_count, part, err); \
+    kern<<<dim3(ds.Q, (unsigned)BK), 256, smem, st>>>(ds, (const T *)q, (const T *)k, (const T *)v, pages, u_c, u_mask, u_logit, u_count, part, err); \
   } while (0)
     if (bf16) { if (ds.d == 64) HILS_ATTN(__nv_bfloat16, 64); else HILS_ATTN(__nv_bfloat16, 128); }
     else { if (ds.d == 64) HILS_ATTN(float, 64); else HILS_ATTN(float, 128); }
@@ -926,6 +942,22 @@ cudaError_t decode_fwd(const DecodeSpec &ds, bool bf16, const void *q, const voi
     ++*launches;
   }
   return cudaSuccess;
+}
+
+cudaError_t decode_fwd(const DecodeSpec &ds, bool bf16, const void *q, const void *k,
+                       const void *v, const void *lmk, int32_t *sel, float *w, float *lse_lmk,
+                       void *out, float *lse, void *ws, uint32_t *err, cudaStream_t st,
+                       int *launches) {
+  return decode_run(ds, bf16, q, k, v, PagedKV{nullptr, 0, 0}, lmk, sel, w, lse_lmk, out, lse, ws,
+                    err, st, launches);
+}
+
+cudaError_t decode_fwd_paged(const DecodeSpec &ds, bool bf16, const void *q, const void *k_pages,
+                             const void *v_pages, const PagedKV &pages, const void *lmk,
+                             int32_t *sel, float *w, float *lse_lmk, void *out, float *lse,
+                             void *ws, uint32_t *err, cudaStream_t st, int *launches) {
+  return decode_run(ds, bf16, q, k_pages, v_pages, pages, lmk, sel, w, lse_lmk, out, lse, ws, err,
+                    st, launches);
 }
 
 }  // namespace hils

@@ -9,6 +9,7 @@
 
 #include "../../include/hils.h"
 #include "kernels.h"
+#include "paged.h"
 
 #define HILS_API extern "C" __attribute__((visibility("default")))
 
@@ -227,15 +228,14 @@ HILS_API hils_status hils_prefill(const hils_params *p, const void *q, const voi
   return hils_attn_fwd(p, q, k, v, sel_idx, chunk_w, out, lse, nullptr, ws, ws_bytes, stream);
 }
 
-HILS_API hils_status hils_decode_fwd(const hils_params *p, const void *q, const void *k_cache,
-                                     const void *v_cache, const void *lmk_k, int32_t *sel_idx,
-                                     float *chunk_w, float *lse_lmk, void *out, float *lse,
-                                     void *ws, size_t ws_bytes, void *stream) {
-  hils_status s = check_params(p);
-  if (s != HILS_OK) return s;
-  NEED(q);
-  NEED(k_cache);
-  NEED(v_cache);
+namespace {
+
+// The decode step over dense caches (pages.table == nullptr) or paged ones.
+hils_status decode_impl(const hils_params *p, const void *q, const void *k, const void *v,
+                        const hils::PagedKV &pages, const void *lmk_k, int32_t *sel_idx,
+                        float *chunk_w, float *lse_lmk, void *out, float *lse, void *ws,
+                        size_t ws_bytes, void *stream) {
+  hils_status s;
   NEED(sel_idx);
   NEED(chunk_w);
   NEED(out);
@@ -252,11 +252,54 @@ HILS_API hils_status hils_decode_fwd(const hils_params *p, const void *q, const 
   uint32_t *err = nullptr;
   if ((s = debug_begin(p, ws, ws_bytes, &err, st)) != HILS_OK) return s;
   int n = 0;
-  cudaError_t e = hils::decode_fwd(ds, p->dtype == HILS_BF16, q, k_cache, v_cache, lmk_k, sel_idx,
-                                   chunk_w, lse_lmk, out, lse, ws, err, st, &n);
+  cudaError_t e =
+      pages.table ? hils::decode_fwd_paged(ds, p->dtype == HILS_BF16, q, k, v, pages, lmk_k,
+                                           sel_idx, chunk_w, lse_lmk, out, lse, ws, err, st, &n)
+                  : hils::decode_fwd(ds, p->dtype == HILS_BF16, q, k, v, lmk_k, sel_idx, chunk_w,
+                                     lse_lmk, out, lse, ws, err, st, &n);
   g_launches += n;
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return debug_end(err, st);
+}
+
+}  // namespace
+
+HILS_API hils_status hils_decode_fwd(const hils_params *p, const void *q, const void *k_cache,
+                                     const void *v_cache, const void *lmk_k, int32_t *sel_idx,
+                                     float *chunk_w, float *lse_lmk, void *out, float *lse,
+                                     void *ws, size_t ws_bytes, void *stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  NEED(q);
+  NEED(k_cache);
+  NEED(v_cache);
+  return decode_impl(p, q, k_cache, v_cache, hils::PagedKV{nullptr, 0, 0}, lmk_k, sel_idx,
+                     chunk_w, lse_lmk, out, lse, ws, ws_bytes, stream);
+}
+
+HILS_API hils_status hils_decode_fwd_paged(const hils_params *p, const void *q,
+                                           const void *k_pages, const void *v_pages,
+                                           int64_t num_pages, const int32_t *page_table,
+                                           int max_pages_per_seq, const void *lmk_k,
+                                           int32_t *sel_idx, float *chunk_w, float *lse_lmk,
+                                           void *out, float *lse, void *ws, size_t ws_bytes,
+                                           void *stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  NEED(q);
+  NEED(k_pages);
+  NEED(v_pages);
+  NEED(page_table);
+  const int pages_needed = (p->L + p->chunk - 1) / p->chunk;
+  if (max_pages_per_seq < pages_needed)
+    return fail(HILS_ERR_INVALID_ARG, "max_pages_per_seq %d below the %d pages of N=%d",
+                max_pages_per_seq, pages_needed, p->L);
+  if (num_pages < 1) return fail(HILS_ERR_INVALID_ARG, "num_pages must be >= 1");
+  if ((int64_t)p->B * max_pages_per_seq >= (int64_t)1 << 31)
+    return fail(HILS_ERR_UNSUPPORTED, "B * max_pages_per_seq must be below 2^31");
+  return decode_impl(p, q, k_pages, v_pages,
+                     hils::PagedKV{page_table, max_pages_per_seq, (long long)num_pages}, lmk_k,
+                     sel_idx, chunk_w, lse_lmk, out, lse, ws, ws_bytes, stream);
 }
 
 HILS_API const char *hils_status_string(hils_status s) {

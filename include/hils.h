@@ -159,6 +159,31 @@ hils_status hils_decode_fwd(const hils_params *p, const void *q, const void *k_c
                             size_t ws_bytes, void *stream);
 
 /*
+ * The decode step of hils_decode_fwd over a paged KV cache, the form an
+ * inference engine's attention backend is handed (molayo1419.me, "Converting
+ * existing models": serving runs HiLS as an attention backend of an SGLang
+ * fork; the page layout below is this library's).  A page holds one chunk
+ * (C = p->chunk tokens) of every KV head:
+ *   k_pages, v_pages [num_pages, Hkv, C, d] in (dtype); a page of a partial
+ *            last chunk holds its N - C*(ceil(N/C)-1) tokens first
+ *   page_table [B, max_pages_per_seq] int32 in (device): page of chunk c of
+ *            sequence b; entries c < ceil(N/C) are read, the rest ignored
+ *   lmk_k    [B,Hkv,N/C,d] in: the landmark keys stay a dense per-sequence
+ *            array (one row per chunk, 1/C of the cache)
+ * Everything else (q, outputs, workspace, N = p->L) is as in hils_decode_fwd;
+ * the results equal hils_decode_fwd on the dense caches the table describes.
+ * Pages may be shared or in any order.  An entry outside [0, num_pages) is
+ * never dereferenced: that chunk's attention output is unspecified and, with
+ * p->debug_checks, the call returns HILS_ERR_DEVICE_CHECK.
+ */
+hils_status hils_decode_fwd_paged(const hils_params *p, const void *q, const void *k_pages,
+                                  const void *v_pages, int64_t num_pages,
+                                  const int32_t *page_table, int max_pages_per_seq,
+                                  const void *lmk_k, int32_t *sel_idx, float *chunk_w,
+                                  float *lse_lmk, void *out, float *lse, void *ws,
+                                  size_t ws_bytes, void *stream);
+
+/*
  * Allocation-free variant of hils_decode_fwd.  The paper has no counterpart:
  * this is a deployment aid.  It is for callers that cannot pass a workspace
  * because they cannot allocate device memory -- e.g. a serving framework that

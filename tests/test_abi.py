@@ -100,3 +100,18 @@ def test_decode_workspace_size(lib):
     rc = lib.hils_decode_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
                              FAKE, None, 0, None)
     assert rc == 3   # workspace too small, rejected before any launch
+
+
+def test_paged_decode_rejects_bad_tables(lib):
+    """hils_decode_fwd_paged: a table narrower than the pages of N, an empty
+    pool or a missing table are refused before any launch."""
+    p = _params(L=1000)  # 1000 tokens: 16 pages of 64
+
+    def call(num_pages, table, max_pages):
+        return lib.hils_decode_fwd_paged(ctypes.byref(p), FAKE, FAKE, FAKE, num_pages, table,
+                                         max_pages, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE,
+                                         1 << 20, None)
+    assert call(16, FAKE, 15) == 1
+    assert call(0, FAKE, 16) == 1
+    assert call(16, None, 16) == 1
+    assert call(16, MISALIGNED, 16) == 1

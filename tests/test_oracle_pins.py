@@ -1,7 +1,8 @@
 """The CPU oracle against its pins (closed forms, hand values, brute force).
 
 Parity status: every oracle entry point (prefill rows in landmark, given and
-exact-mass modes; decode; union) is pinned here; none is unpinned.  The pages
+exact-mass modes; decode; decode over a paged cache; union) is pinned here;
+none is unpinned.  The pages
 print no worked numeric example, so the pins are closed forms and hand-derived
 values listed in tests/pins.py with the passage each one follows.
 """
