@@ -11,8 +11,11 @@
 // K/V is staged once (bulk asynchronous copies into shared memory) for every
 // head that attends it, so the union of the heads' chunks crosses HBM once.
 //
-//   decode_gemv    grid (ceil(n_c/128), B*Hkv): one thread per landmark ->
-//                  the logits of the G heads, into a workspace array
+//   decode_gemv_tc grid (min(ceil(n_c/128), 8), B*Hkv), bf16 and G <= 16:
+//                  per 128-landmark tile one tcgen05.mma (M = 128 landmarks,
+//                  N = 16 padded heads) -> the logits of the G heads, into a
+//                  workspace array (decode_gemv: the same on the CUDA cores,
+//                  one thread per landmark, for fp32 or G > 16)
 //   decode_topk    grid (B*Hq): the head's log-sum-exp and exact top-k
 //                  (radix select on the logit bits) -> sel_idx / chunk_w,
 //                  ascending chunk ids, lse_lmk
@@ -20,7 +23,9 @@
 //                  head mask and per-head logits
 //   decode_attn    grid (Q, B*Hkv): up to 16 union chunks per CTA, each chunk's
 //                  K and V staged once; per head an online (max, sum, acc)
-//                  partial over its chunks
+//                  partial over its chunks.  With a page table the chunk's
+//                  [64][d] slab of KV head hkv is read from its page
+//                  ([num_pages][Hkv][64][d] pools) instead of the dense cache
 //   decode_combine grid (B*Hq): partials -> out, lse
 #include <cuda_bf16.h>
 

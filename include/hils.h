@@ -164,8 +164,9 @@ hils_status hils_decode_fwd(const hils_params *p, const void *q, const void *k_c
  * existing models": serving runs HiLS as an attention backend of an SGLang
  * fork; the page layout below is this library's).  A page holds one chunk
  * (C = p->chunk tokens) of every KV head:
- *   k_pages, v_pages [num_pages, Hkv, C, d] in (dtype); a page of a partial
- *            last chunk holds its N - C*(ceil(N/C)-1) tokens first
+ *   k_pages, v_pages [num_pages, Hkv, C, d] in (dtype), both of num_pages
+ *            pages; a page of a partial last chunk holds its
+ *            N - C*(ceil(N/C)-1) tokens first
  *   page_table [B, max_pages_per_seq] int32 in (device): page of chunk c of
  *            sequence b; entries c < ceil(N/C) are read, the rest ignored
  *   lmk_k    [B,Hkv,N/C,d] in: the landmark keys stay a dense per-sequence
