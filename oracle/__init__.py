@@ -24,6 +24,10 @@ section "Converting existing models" has HiLS served as such a backend) back
 into the dense cache it describes; ``decode_paged`` is the decode step on that
 dense cache.
 
+``hope`` is the hierarchical positional encoding of the same page, section
+"Engineering details" (HoPE): rotary position embedding on the dimensions
+that fall inside the pre-training window, no positional encoding on the rest.
+
 Every entry point is pinned in ``tests/test_oracle_pins.py`` against closed
 forms, hand-derived values and brute force; none is "parity unpinned".
 
@@ -231,6 +235,40 @@ def gather_pages(pages, page_table, L: int) -> np.ndarray:
                 raise ValueError(f"page table entry ({b}, {c}) = {page} outside the pool")
             n = min(C, L - c * C)
             out[b, :, c * C:c * C + n, :] = pg[page, :, :n, :]
+    return out
+
+
+def hope(x, positions, n_rope_pairs: int, base: float = 10000.0) -> np.ndarray:
+    """HoPE applied to x [..., n, d] at integer positions [n], in fp64.
+
+    Dimensions pair up as (i, i + d/2) (the rotate-half convention); pair i
+    has angular frequency theta_i = base ** (-2 i / d), so the wavelength
+    grows with i.  Pairs i < n_rope_pairs (the short wavelengths, inside the
+    pre-training window) are rotated by the angle t * theta_i:
+        x'_i       = x_i cos - x_{i+d/2} sin
+        x'_{i+d/2} = x_i sin + x_{i+d/2} cos
+    and the other pairs are left as they are (NoPE).  Returns fp64; bf16
+    input (raw bits or a bf16 tensor) is widened exactly first."""
+    a, bf16 = _as_array(x)
+    if bf16:
+        a = (a.astype(np.uint32) << 16).view(np.float32)
+    a = a.astype(np.float64)
+    d = a.shape[-1]
+    half = d // 2
+    if not 0 <= n_rope_pairs <= half:
+        raise ValueError("n_rope_pairs must lie in [0, d/2]")
+    t = np.asarray(positions, dtype=np.float64).reshape(-1)
+    if t.shape[0] != a.shape[-2]:
+        raise ValueError("one position per row")
+    out = a.copy()
+    for i in range(n_rope_pairs):
+        theta = float(base) ** (-2.0 * i / d)
+        ang = t * theta
+        c, s = np.cos(ang)[:, None], np.sin(ang)[:, None]
+        xi = a[..., :, i:i + 1]
+        xj = a[..., :, i + half:i + half + 1]
+        out[..., :, i:i + 1] = xi * c - xj * s
+        out[..., :, i + half:i + half + 1] = xi * s + xj * c
     return out
 
 

@@ -423,6 +423,52 @@ def pin_paged_decode_is_dense_decode(orc):
     assert np.isfinite(paged["out"]).all()
 
 
+def pin_hope_rotation_properties(orc):
+    """HoPE [KR "Engineering details", HoPE]: on the rotated pairs a rotary
+    embedding, on the others the identity.  Checked against what rotations
+    fix: norms are kept; position 0 and n_rope_pairs = 0 are the identity;
+    the NoPE half of the pairs is untouched; rotating by t1 then by t2 equals
+    rotating by t1 + t2; the dot product of a rotated query and key depends
+    on their positions only through t - s; one pair at one position equals a
+    hand-computed 2-d rotation."""
+    from oracle import hope
+    rng = _rng(41)
+    d, n = 16, 9
+    x = rng.standard_normal((2, n, d))
+    pos = rng.integers(0, 5000, size=n)
+    y = hope(x.astype(np.float32), pos, 5, 500.0)
+    x32 = x.astype(np.float32).astype(np.float64)
+    assert np.allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x32, axis=-1), rtol=1e-12)
+    assert np.array_equal(hope(x32.astype(np.float32), np.zeros(n), 8, 500.0), x32)
+    assert np.array_equal(hope(x32.astype(np.float32), pos, 0, 500.0), x32)
+    nope = [i for i in range(d // 2) if i >= 5]
+    for i in nope:
+        assert np.array_equal(y[..., i], x32[..., i]) and np.array_equal(y[..., i + d // 2], x32[..., i + d // 2])
+    # group property, with the rotation written out as a matrix per pair
+    t1, t2 = 1234, 777
+    def rot(v, t, pairs, base):
+        out = v.copy()
+        for i in range(pairs):
+            th = base ** (-2.0 * i / d) * t
+            m = np.array([[math.cos(th), -math.sin(th)], [math.sin(th), math.cos(th)]])
+            u = np.stack([v[..., i], v[..., i + d // 2]], -1) @ m.T
+            out[..., i], out[..., i + d // 2] = u[..., 0], u[..., 1]
+        return out
+    v = rng.standard_normal((n, d)).astype(np.float32)
+    a1 = hope(v, np.full(n, t1 + t2), 6, 10000.0)
+    a2 = rot(rot(v.astype(np.float64), t1, 6, 10000.0), t2, 6, 10000.0)
+    assert np.allclose(a1, a2, atol=1e-9)
+    # relative positions: <R(t) q, R(s) k> is a function of t - s
+    q = rng.standard_normal((1, d)).astype(np.float32)
+    k = rng.standard_normal((1, d)).astype(np.float32)
+    dots = [float((hope(q, [t], 8, 10000.0) @ hope(k, [s], 8, 10000.0).T)[0, 0])
+            for t, s in ((50, 20), (1030, 1000), (900030, 900000))]
+    assert np.allclose(dots, dots[0], atol=1e-8)
+    # hand value: d = 4, pair 0 has theta 1; x = (1, 0, 0, 0) at position t -> (cos t, 0, sin t, 0)
+    h = hope(np.array([[1.0, 0.0, 0.0, 0.0]], np.float32), [3], 1, 10000.0)
+    assert np.allclose(h, [[math.cos(3.0), 0.0, math.sin(3.0), 0.0]], atol=1e-15)
+
+
 ALL_PINS = [
     pin_landmark_logit_and_normaliser,
     pin_topk_planted_ties,
@@ -437,4 +483,5 @@ ALL_PINS = [
     pin_bf16_bits_widen_exactly,
     pin_union_is_set_union,
     pin_paged_decode_is_dense_decode,
+    pin_hope_rotation_properties,
 ]
