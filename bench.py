@@ -9,9 +9,10 @@ synthetic batch: landmark scoring + inter-chunk normaliser + top-k
 (hils_select), then the chunk union, intra-chunk attention and fusion
 (hils_attn_fwd, which builds each tile's union itself).  Default workload:
 the 512K-token 7B-shaped prefill (B=1, 32/8 heads, d=128, k=64, M=128).
-The 128K prefill, the B=16 x 512K decode step and the same decode step over
-a paged KV cache (hils_decode_fwd_paged, shuffled page pool) are timed as
-extra lines inside the same JSON object ("workloads").
+The 128K prefill, the B=16 x 512K decode step, the same decode step over a
+paged KV cache (hils_decode_fwd_paged, shuffled page pool) and the HoPE
+pre-pass over the 512K q and k (hils_hope) are timed as extra lines inside
+the same JSON object ("workloads").
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
 cuda synchronize, CUDA events on the launching stream, max over ranks.
@@ -387,6 +388,36 @@ def bench_decode(hb, synth, w, steps, warmup, seed_offset, paged=False):
     return res
 
 
+def bench_hope(hb, w, steps, warmup, train_len=65536, base=500000.0):
+    """The HoPE pre-pass (hils_hope) over q and k of workload w, in place:
+    the pairs whose wavelength fits train_len are rotated.  HBM-bound; the
+    algorithmic bytes are the rotated elements read and written once."""
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev).manual_seed(w.seed + 23)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q = torch.randn((w.B, w.Hq, w.L, w.d), generator=g, device=dev).to(dt)
+    k = torch.randn((w.B, w.Hkv, w.L, w.d), generator=g, device=dev).to(dt)
+    npairs = hb.rope_pairs_for(w.d, base, train_len)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hb.hils_hope(q, npairs, 0, base, stream)
+        hb.hils_hope(k, npairs, 0, base, stream)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    nbytes = 2.0 * 2 * npairs * (w.Hq + w.Hkv) * w.B * w.L * q.element_size()
+    return dict(ms=ms, bytes=nbytes, npairs=npairs)
+
+
 def union_stats(hb, sel, w):
     """Chunk-union size per group of M rows and adjacent-query overlap."""
     u_off, _ = hb.union(sel, M=w.M)
@@ -522,6 +553,18 @@ def run_ours(args):
             "hbm_frac": pgbs / peaks["hbm_gbs"],
             "pool": f"{r3['paged_pages']} pages of 64 tokens x {w3.Hkv} KV heads, random order",
             "equal_to_dense": r3["paged_equal"]}
+        del r3
+        torch.cuda.empty_cache()
+        try:
+            r4 = bench_hope(hb, w, max(5, args.steps), 3)
+            hgbs = r4["bytes"] / (r4["ms"] * 1e-3) / 1e9
+            extra["hope_prepass_" + w.name] = {
+                "ms_per_step": r4["ms"], "rotated_pairs": r4["npairs"],
+                "split": "pairs with wavelength <= 65536 tokens at base 500000 (q and k, in place)",
+                "algorithmic_bytes": r4["bytes"], "achieved_gbs": hgbs,
+                "hbm_frac": hgbs / peaks["hbm_gbs"]}
+        except Exception as e:  # an extra entry must not cost the main line
+            extra["hope_prepass_" + w.name] = {"error": str(e)[:200]}
         line["workloads"] = extra
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, res["host_inputs"])

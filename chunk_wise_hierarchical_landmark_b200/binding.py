@@ -9,6 +9,7 @@ libhils.so is missing or fails to load, every call raises.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 
 import torch
@@ -38,7 +39,7 @@ class Params(ctypes.Structure):
 _lib = None
 EXPORTS = ["hils_workspace_size", "hils_select", "hils_union_capacity", "hils_union",
            "hils_attn_fwd", "hils_prefill", "hils_decode_fwd", "hils_decode_fwd_paged",
-           "hils_decode_fwd_noalloc",
+           "hils_decode_fwd_noalloc", "hils_hope",
            "hils_status_string", "hils_last_error", "hils_launch_count"]
 
 
@@ -62,8 +63,9 @@ def lib():
         L.hils_decode_fwd.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.hils_decode_fwd_paged.argtypes = [PP, P, P, P, I64, P, I, P, P, P, P, P, P, P, SZ, P]
         L.hils_decode_fwd_noalloc.argtypes = [PP, P, P, P, P, P, P, P, P, P, P]
+        L.hils_hope.argtypes = [P, I, I, I, I, I, I, I, ctypes.c_double, P]
         for f in ("hils_select", "hils_union", "hils_attn_fwd", "hils_prefill", "hils_decode_fwd",
-                  "hils_decode_fwd_paged", "hils_decode_fwd_noalloc"):
+                  "hils_decode_fwd_paged", "hils_decode_fwd_noalloc", "hils_hope"):
             getattr(L, f).restype = I
         L.hils_status_string.argtypes = [I]
         L.hils_status_string.restype = ctypes.c_char_p
@@ -167,6 +169,28 @@ def hils_decode_fwd_noalloc(p: Params, q, k_cache, v_cache, lmk_k, sel_idx, chun
     _check(lib().hils_decode_fwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                          _ptr(lmk_k), _ptr(sel_idx), _ptr(chunk_w), _ptr(lse_lmk),
                                          _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def hils_hope(x, n_rope_pairs: int, pos0: int = 0, base: float = 10000.0, stream=None):
+    """HoPE in place on x [B,H,L,d] (or a decode query [B,H,d], one position)."""
+    if x.dim() == 3:
+        B, H, d = x.shape
+        L = 1
+    else:
+        B, H, L, d = x.shape
+    dt = HILS_BF16 if x.dtype == torch.bfloat16 else HILS_F32
+    _check(lib().hils_hope(_ptr(x), dt, B, H, L, d, int(pos0), int(n_rope_pairs), float(base),
+                           _stream(stream)))
+
+
+def rope_pairs_for(d: int, base: float, train_len: int) -> int:
+    """One split rule for HoPE: the pairs whose wavelength 2*pi*base^(2i/d)
+    fits in the pre-training length get RoPE (they are the first ones, as the
+    wavelength grows with i)."""
+    n = 0
+    while n < d // 2 and 2.0 * math.pi * base ** (2.0 * n / d) <= train_len:
+        n += 1
+    return n
 
 
 def launch_count() -> int:

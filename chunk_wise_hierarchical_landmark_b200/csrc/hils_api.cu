@@ -9,6 +9,7 @@
 
 #include "../../include/hils.h"
 #include "kernels.h"
+#include "hope.h"
 #include "paged.h"
 
 #define HILS_API extern "C" __attribute__((visibility("default")))
@@ -300,6 +301,26 @@ HILS_API hils_status hils_decode_fwd_paged(const hils_params *p, const void *q,
   return decode_impl(p, q, k_pages, v_pages,
                      hils::PagedKV{page_table, max_pages_per_seq, (long long)num_pages}, lmk_k,
                      sel_idx, chunk_w, lse_lmk, out, lse, ws, ws_bytes, stream);
+}
+
+HILS_API hils_status hils_hope(void *x, int dtype, int B, int H, int L, int d, int pos0,
+                               int n_rope_pairs, double base, void *stream) {
+  NEED(x);
+  if (dtype != HILS_F32 && dtype != HILS_BF16) return fail(HILS_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (B < 1 || H < 1 || L < 1) return fail(HILS_ERR_INVALID_ARG, "B, H and L must be >= 1");
+  if (d != 64 && d != 128) return fail(HILS_ERR_UNSUPPORTED, "d=%d (supported: 64, 128)", d);
+  if (n_rope_pairs < 0 || n_rope_pairs > d / 2)
+    return fail(HILS_ERR_INVALID_ARG, "n_rope_pairs=%d outside [0, d/2]", n_rope_pairs);
+  if (pos0 < 0 || (int64_t)pos0 + L - 1 >= (int64_t)1 << 31)
+    return fail(HILS_ERR_INVALID_ARG, "positions pos0 .. pos0+L-1 must lie in [0, 2^31)");
+  if (!std::isfinite(base) || !(base > 1.0)) return fail(HILS_ERR_INVALID_ARG, "base must be finite and > 1");
+  if ((int64_t)B * H > (1 << 16) - 1) return fail(HILS_ERR_UNSUPPORTED, "B*H above 65535");
+  int n = 0;
+  cudaError_t e = hils::hope_apply(x, dtype == HILS_BF16, B * H, L, d, pos0, n_rope_pairs, base,
+                                   static_cast<cudaStream_t>(stream), &n);
+  g_launches += n;
+  if (e != cudaSuccess) return cuda_fail(e, "hope launch");
+  return HILS_OK;
 }
 
 HILS_API const char *hils_status_string(hils_status s) {

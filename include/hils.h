@@ -205,6 +205,25 @@ hils_status hils_decode_fwd_noalloc(const hils_params *p, const void *q, const v
                                     float *chunk_w, float *lse_lmk, void *out, float *lse,
                                     void *stream);
 
+/*
+ * HoPE, the positional encoding of the pages (molayo1419.me, "Engineering
+ * details", HoPE): rotary position embedding on the dimensions inside the
+ * pre-training window, none (NoPE) on the rest.  Applied in place to q or k
+ * before hils_prefill / hils_decode_fwd (a decode query at pos0 = N-1; keys
+ * as they enter the cache); the landmark keys are left to the caller.
+ *   x      [B, H, L, d] in/out, dtype HILS_F32 or HILS_BF16; row (b, h, t)
+ *          has position pos0 + t
+ *   n_rope_pairs  number of rotated pairs, 0..d/2: dimensions pair up as
+ *          (i, i + d/2) and pair i < n_rope_pairs turns by the angle
+ *          (pos0 + t) * base^(-2i/d); the other pairs are not touched.  The
+ *          pages give no split rule: the caller picks it (e.g. the pairs
+ *          whose wavelength 2*pi*base^(2i/d) fits the pre-training length)
+ *   base   > 1
+ * Asynchronous on `stream`; invalid arguments are refused before the launch.
+ */
+hils_status hils_hope(void *x, int dtype, int B, int H, int L, int d, int pos0,
+                      int n_rope_pairs, double base, void *stream);
+
 /* Static description of a status code. */
 const char *hils_status_string(hils_status s);
 

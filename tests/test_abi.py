@@ -115,3 +115,26 @@ def test_paged_decode_rejects_bad_tables(lib):
     assert call(0, FAKE, 16) == 1
     assert call(16, None, 16) == 1
     assert call(16, MISALIGNED, 16) == 1
+
+
+@pytest.mark.parametrize("kw", [dict(n_rope_pairs=65), dict(n_rope_pairs=-1), dict(base=1.0),
+                                dict(base=float("nan")), dict(d=96), dict(L=0), dict(dtype=7),
+                                dict(pos0=-1), dict(pos0=(1 << 31) - 10, L=20)])
+def test_hope_rejects_bad_arguments(lib, kw):
+    """hils_hope validates before any launch."""
+    a = dict(dtype=hb.HILS_BF16, B=1, H=2, L=16, d=128, pos0=0, n_rope_pairs=8, base=10000.0)
+    a.update(kw)
+    rc = lib.hils_hope(FAKE, a["dtype"], a["B"], a["H"], a["L"], a["d"], a["pos0"],
+                       a["n_rope_pairs"], a["base"], None)
+    assert rc in (1, 2), lib.hils_last_error()
+    assert lib.hils_hope(None, hb.HILS_BF16, 1, 1, 1, 64, 0, 1, 10000.0, None) == 1
+
+
+def test_rope_pairs_for_matches_its_definition():
+    """The split helper counts exactly the pairs whose wavelength fits."""
+    import math
+    for d in (64, 128):
+        for base in (10000.0, 500000.0):
+            for train in (1, 6, 4096, 65536, 10 ** 12):
+                want = sum(1 for i in range(d // 2) if 2 * math.pi * base ** (2 * i / d) <= train)
+                assert hb.rope_pairs_for(d, base, train) == want
