@@ -28,6 +28,9 @@ dense cache.
 "Engineering details" (HoPE): rotary position embedding on the dimensions
 that fall inside the pre-training window, no positional encoding on the rest.
 
+``oracle.backward`` (plain PyTorch fp64) states the forward a second time and
+differentiates it with autograd: the reference for a backward pass.
+
 Every entry point is pinned in ``tests/test_oracle_pins.py`` against closed
 forms, hand-derived values and brute force; none is "parity unpinned".
 
