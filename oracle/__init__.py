@@ -28,6 +28,11 @@ dense cache.
 "Engineering details" (HoPE): rotary position embedding on the dimensions
 that fall inside the pre-training window, no positional encoding on the rest.
 
+``qcal_query`` and ``Oracle.rows_qcal`` follow the Q-Cal item of the same
+section: a low-rank offset W_up W_down h added to the query for the chunk
+scores only (selection and chunk logits); attention inside the chunks keeps
+the plain query.
+
 ``oracle.backward`` (plain PyTorch fp64) states the forward a second time and
 differentiates it with autograd: the reference for a backward pass.
 
@@ -188,6 +193,19 @@ class Oracle:
         v = gather_pages(v_pages, page_table, p.L)
         return self.decode(p, q, k, v, lmk, heads, nthreads)
 
+    def rows_qcal(self, p: Problem, q, k, v, lmk, qs, rows, nthreads: int = 0) -> dict:
+        """Prefill rows with a separate scoring query qs [B,Hq,L,d] (fp32):
+        landmark scores, top-k, chunk logits and lse_lmk come from qs; the
+        attention inside the chunks and the own chunk's logit from q.  Two
+        calls of the same oracle: landmark mode on qs, then given mode on q
+        with that selection and those logits (all inputs widened to fp32)."""
+        k32, v32, l32, q32 = (_widen32(a) for a in (k, v, lmk, q))
+        sc = self.rows(p, _widen32(qs), k32, v32, l32, rows, nthreads=nthreads)
+        res = self.rows(p, q32, k32, v32, l32, rows, mode="given", sel_in=sc["sel"],
+                        w_in=sc["w"], nthreads=nthreads)
+        res["lse_lmk"] = sc["lse_lmk"]
+        return res
+
     def scores(self, p: Problem, q, lmk, rows, nthreads: int = 0,
                decode: bool = False) -> np.ndarray:
         """Landmark logits of every completed chunk for the rows (numbered as in
@@ -216,6 +234,25 @@ class Oracle:
         if n < 0:
             raise ValueError("union capacity exceeded")
         return u[:n].copy()
+
+
+def _widen32(x) -> np.ndarray:
+    """fp32 copy of fp32 / bf16 input (bf16 widens exactly)."""
+    a, bf16 = _as_array(x)
+    if bf16:
+        a = (a.astype(np.uint32) << 16).view(np.float32)
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def qcal_query(q, h, w_down, w_up) -> np.ndarray:
+    """Q-Cal scoring query: q_t + W_up[hq] (W_down h_t) for every head and
+    position, formed in fp64 and rounded once to fp32.
+    q [B,Hq,L,d] (fp32 / bf16), h [B,L,D] hidden states, w_down [r,D] (shared
+    by the heads), w_up [Hq,d,r]."""
+    qa = _widen32(q).astype(np.float64)
+    z = np.einsum("rD,bLD->bLr", np.asarray(w_down, np.float64), np.asarray(h, np.float64))
+    dq = np.einsum("hdr,bLr->bhLd", np.asarray(w_up, np.float64), z)
+    return (qa + dq).astype(np.float32)
 
 
 def gather_pages(pages, page_table, L: int) -> np.ndarray:

@@ -55,17 +55,18 @@ def causal_attention(q, k, v, scale):
     return np.exp(X - lse[:, None]) @ v, lse
 
 
-def all_selected_closed_form(q, k, v, lmk, C, scale):
+def all_selected_closed_form(q, k, v, lmk, C, scale, qs=None):
     """HiLS output when every completed chunk is selected, written as ONE
     masked softmax over keys ([MC]: inter-chunk softmax times intra-chunk
     softmax): key j of a completed chunk c gets logit
     scale*<q,k_j> + s_c - lse_c with s_c = scale*<q, lmk_c> and lse_c the
     log-sum-exp of chunk c's token logits; own-chunk keys (j <= t) keep their
-    token logit.  q, k, v [L, d], lmk [L//C, d] fp64 for one head."""
+    token logit.  q, k, v [L, d], lmk [L//C, d] fp64 for one head; qs, when
+    given, replaces q in the landmark logits s_c only (Q-Cal)."""
     L = q.shape[0]
     nfull = L // C
     X = scale * q @ k.T                                # [L, L]
-    S = scale * q @ lmk.T                              # [L, nfull]
+    S = scale * (q if qs is None else qs) @ lmk.T      # [L, nfull]
     chunk_lse = _lse(X[:, :nfull * C].reshape(L, nfull, C), axis=2) if nfull else np.zeros((L, 0))
     t = np.arange(L)[:, None]
     j = np.arange(L)[None, :]
@@ -469,6 +470,55 @@ def pin_hope_rotation_properties(orc):
     assert np.allclose(h, [[math.cos(3.0), 0.0, math.sin(3.0), 0.0]], atol=1e-15)
 
 
+def pin_qcal_scoring_query(orc):
+    """Q-Cal [KR "Engineering details", Q-Cal]: the offset W_up W_down h
+    changes the query of the chunk scores only.  A hand value of the offset;
+    no offset reproduces the plain oracle; with every chunk selected the
+    output is the dense closed form whose chunk logits use the calibrated
+    query and whose token logits use the plain one; an offset along one
+    landmark makes k = 1 pick that chunk on every row that can."""
+    from oracle import qcal_query
+    # hand value: D = 2, r = 1, d = 2, h_t = (1, 1): z = 1 + 2 = 3, dq = (3*3, 4*3)
+    qs = qcal_query(np.zeros((1, 1, 1, 2), np.float32), np.ones((1, 1, 2)), [[1.0, 2.0]],
+                    [[[3.0], [4.0]]])
+    assert np.array_equal(qs.reshape(-1), np.array([9.0, 12.0], np.float32))
+    rng = _rng(43)
+    B, Hq, Hkv, L, d, C, D, r = 1, 4, 2, 45, 8, 4, 12, 3
+    q = _f32(B, Hq, L, d, rng=rng)
+    k = _f32(B, Hkv, L, d, rng=rng)
+    v = _f32(B, Hkv, L, d, rng=rng)
+    lmk = _f32(B, Hkv, L // C, d, rng=rng, scale=0.7)
+    h = rng.standard_normal((B, L, D))
+    wd = rng.standard_normal((r, D)) * 0.3
+    wu = rng.standard_normal((Hq, d, r)) * 0.3
+    rows = np.arange(B * Hq * L)
+    p = Problem(B=B, Hq=Hq, Hkv=Hkv, L=L, d=d, C=C, topk=3, scale=1 / math.sqrt(d))
+    plain = orc.rows(p, q, k, v, lmk, rows)
+    same = orc.rows_qcal(p, q, k, v, lmk, qcal_query(q, h, wd, 0 * wu), rows)
+    for key in ("sel", "w", "out", "lse", "lse_lmk"):
+        assert np.array_equal(plain[key], same[key]), key
+    pa = Problem(B=B, Hq=Hq, Hkv=Hkv, L=L, d=d, C=C, topk=L // C + 1, scale=1 / math.sqrt(d))
+    qs = qcal_query(q, h, wd, wu)
+    res = orc.rows_qcal(pa, q, k, v, lmk, qs, rows)
+    for hq in range(Hq):
+        g = hq // (Hq // Hkv)
+        o, lse = all_selected_closed_form(q[0, hq].astype(float), k[0, g].astype(float),
+                                          v[0, g].astype(float), lmk[0, g].astype(float), C,
+                                          pa.scale, qs=qs[0, hq].astype(float))
+        sl = slice(hq * L, (hq + 1) * L)
+        assert np.allclose(res["out"][sl], o, rtol=0, atol=1e-11), hq
+        assert np.allclose(res["lse"][sl], lse, rtol=0, atol=1e-11), hq
+    star = 2
+    pull = qs.copy()
+    for hq in range(Hq):
+        pull[0, hq] += 40.0 * lmk[0, hq // (Hq // Hkv), star] / np.linalg.norm(lmk[0, hq // (Hq // Hkv), star])
+    p1 = Problem(B=B, Hq=Hq, Hkv=Hkv, L=L, d=d, C=C, topk=1, scale=1 / math.sqrt(d))
+    got = orc.rows_qcal(p1, q, k, v, lmk, pull, rows)
+    t = rows % L
+    can = t // C > star
+    assert (got["sel"][can, 0] == star).all()
+
+
 ALL_PINS = [
     pin_landmark_logit_and_normaliser,
     pin_topk_planted_ties,
@@ -484,4 +534,5 @@ ALL_PINS = [
     pin_union_is_set_union,
     pin_paged_decode_is_dense_decode,
     pin_hope_rotation_properties,
+    pin_qcal_scoring_query,
 ]
