@@ -99,3 +99,65 @@ def backward(p, q, k, v, lmk, dout, dlse=None) -> dict:
     g = [torch.zeros_like(x) if gi is None else gi for x, gi in zip(xs, g)]
     return {"dq": g[0].numpy(), "dk": g[1].numpy(), "dv": g[2].numpy(), "dlmk": g[3].numpy(),
             "out": out.detach().numpy(), "lse": lse.detach().numpy(), "sel": sels}
+
+
+def backward_explicit(p, q, k, v, lmk, dout, dlse=None) -> dict:
+    """The same gradients from explicit formulas (numpy fp64, one row at a
+    time), in the quantities a kernel forms per (row, attended chunk):
+
+      P_j   = w_c p_{c,j}        the fused weight of key j of chunk c
+                                 (p: softmax inside the chunk, w: fusion)
+      dP_j  = <dout, v_j>        g_c = sum_j p_{c,j} dP_j = <dout, a_c>
+      D     = <dout, out>        (the row's output-gradient dot product)
+      dv_j += P_j dout
+      dx_j  = P_j (dP_j - g_c)                  token logit x_j = scale <q, k_j>
+            + p_{own,j} w_own (g_own - D + dlse)   (own chunk: through l_own)
+      ds_c  = w_c (g_c - D + dlse)                chunk logit s_c of a selected c
+      dq   += scale (sum_j dx_j k_j + sum_c ds_c lmk_c)
+      dk_j += scale dx_j q,   dlmk_c += scale ds_c q
+    The selection is the forward's (no gradient through the choice)."""
+    q, k, v, lmk = (_f64(a).numpy() for a in (q, k, v, lmk))
+    dout = np.asarray(dout, np.float64)
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    C, scale = p.C, p.scale
+    dq, dk, dv, dl = (np.zeros_like(a) for a in (q, k, v, lmk))
+    for b in range(B):
+        for hq in range(Hq):
+            hk = hq // G
+            for t in range(L):
+                qt, dot = q[b, hq, t], dout[b, hq, t]
+                dls = 0.0 if dlse is None else float(np.asarray(dlse)[b, hq, t])
+                oc = t // C
+                s = scale * (lmk[b, hk, :oc] @ qt) if oc else np.zeros(0)
+                pick = select(torch.from_numpy(s), p.topk)
+                spans = [(c * C, c * C + C) for c in pick] + [(oc * C, t + 1)]
+                pc, ac = [], []
+                for j0, j1 in spans:
+                    x = scale * (k[b, hk, j0:j1] @ qt)
+                    e = np.exp(x - x.max())
+                    pc.append(e / e.sum())
+                    ac.append(pc[-1] @ v[b, hk, j0:j1])
+                x_own = scale * (k[b, hk, oc * C:t + 1] @ qt)
+                logits = np.array([s[c] for c in pick] + [x_own.max() + np.log(np.exp(x_own - x_own.max()).sum())])
+                w = np.exp(logits - logits.max())
+                w /= w.sum()
+                out = sum(wi * ai for wi, ai in zip(w, ac))
+                D = float(dot @ out)
+                for i, (j0, j1) in enumerate(spans):
+                    dP = v[b, hk, j0:j1] @ dot
+                    g = float(pc[i] @ dP)
+                    P = w[i] * pc[i]
+                    dv[b, hk, j0:j1] += P[:, None] * dot[None, :]
+                    dx = P * (dP - g)
+                    if i == len(spans) - 1:  # own chunk: its logit is l_own
+                        dx = dx + pc[i] * w[i] * (g - D + dls)
+                    else:
+                        ds = w[i] * (g - D + dls)
+                        c = pick[i]
+                        dq[b, hq, t] += scale * ds * lmk[b, hk, c]
+                        dl[b, hk, c] += scale * ds * qt
+                    dq[b, hq, t] += scale * (dx @ k[b, hk, j0:j1])
+                    dk[b, hk, j0:j1] += scale * dx[:, None] * qt[None, :]
+    return {"dq": dq, "dk": dk, "dv": dv, "dlmk": dl}

@@ -130,3 +130,21 @@ def test_unused_inputs_get_no_gradient():
             assert not r["dk"][0, 0, c * C:(c + 1) * C].any(), c
             assert not r["dv"][0, 0, c * C:(c + 1) * C].any(), c
     assert len(chosen) < L // C  # the case is not vacuous
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,d,C,topk,with_dlse", [(1, 2, 1, 40, 4, 8, 2, True),
+                                                            (2, 4, 2, 37, 8, 4, 3, False),
+                                                            (1, 2, 2, 19, 4, 4, 8, True)])
+def test_explicit_formulas_equal_autograd(B, Hq, Hkv, L, d, C, topk, with_dlse):
+    """The per-chunk backward formulas (the quantities a kernel would form)
+    give autograd's gradients: GQA, a ragged last chunk, k >= n_c, with and
+    without an lse gradient."""
+    p = oracle.Problem(B=B, Hq=Hq, Hkv=Hkv, L=L, d=d, C=C, topk=topk, scale=1 / math.sqrt(d))
+    q, k, v, lmk = inputs(B, Hq, Hkv, L, d, C, seed=L + 1)
+    rng = np.random.default_rng(L + 2)
+    dout = rng.standard_normal((B, Hq, L, d))
+    dlse = rng.standard_normal((B, Hq, L)) if with_dlse else None
+    a = ob.backward(p, q, k, v, lmk, dout, dlse)
+    e = ob.backward_explicit(p, q, k, v, lmk, dout, dlse)
+    for key in ("dq", "dk", "dv", "dlmk"):
+        assert np.abs(a[key] - e[key]).max() <= 1e-12, key
