@@ -7,7 +7,6 @@ a fixed 32 MiB array inside the library.  This file is collected last so
 that a failure here does not hide the results of the other tests."""
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
