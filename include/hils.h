@@ -32,7 +32,8 @@
  *   selected landmark logits plus the own-chunk logit.
  *   Pointers: every array argument is a DEVICE pointer owned by the caller,
  *   16-byte aligned.  The library allocates no device memory and keeps no
- *   state other than cached device attributes and a launch counter.
+ *   state other than cached device attributes, a launch counter and the
+ *   fixed scratch array of hils_decode_fwd_noalloc (module memory, below).
  *   Streams: every call is asynchronous on `stream` (a cudaStream_t passed as
  *   void*; NULL = legacy default stream).  Argument and shape errors are
  *   returned before anything is launched.  A launch failure returns
