@@ -1,9 +1,11 @@
 """The pins catch plausible mistakes: each test compiles a copy of the oracle
-with one planted mistake (on the CPU, in a temporary directory) and requires
-at least one pin of tests/pins.py to fail on it."""
+with one planted mistake (on the CPU, in a temporary directory), or swaps one
+of the oracle's Python functions for a broken version, and requires a pin of
+tests/pins.py to fail on it."""
 import os
 import shutil
 
+import numpy as np
 import pytest
 
 import oracle
@@ -51,3 +53,89 @@ def test_mutant_is_caught(tmp_path, name, old, new):
             failed.append(pin.__name__)
     assert failed, f"planted mistake {name} passed every pin"
     shutil.rmtree(tmp_path, ignore_errors=True)
+
+
+# ---------------------------------------------------------------------------
+# The Python parts of the oracle (paged-cache gather, HoPE, Q-Cal): each
+# planted mistake replaces one function for the duration of the test, and
+# the pin written for that function must fail.
+
+def _gather_ignores_table(pages, page_table, L):
+    pg, _ = oracle._as_array(pages)
+    tab = np.asarray(page_table)
+    num_pages, Hkv, C, d = pg.shape
+    B, npg = tab.shape[0], -(-L // C)
+    out = np.empty((B, Hkv, L, d), pg.dtype)
+    for b in range(B):
+        for c in range(npg):
+            n = min(C, L - c * C)
+            out[b, :, c * C:c * C + n] = pg[b * npg + c, :, :n]
+    return out
+
+
+def _gather_token_major_pages(pages, page_table, L):
+    pg, _ = oracle._as_array(pages)
+    tab = np.asarray(page_table)
+    num_pages, Hkv, C, d = pg.shape
+    flat = pg.reshape(num_pages, C, Hkv, d)
+    out = np.empty((tab.shape[0], Hkv, L, d), pg.dtype)
+    for b in range(tab.shape[0]):
+        for c in range(-(-L // C)):
+            n = min(C, L - c * C)
+            out[b, :, c * C:c * C + n] = flat[int(tab[b, c])].transpose(1, 0, 2)[:, :n]
+    return out
+
+
+def _hope_variant(kind):
+    def hope(x, positions, n_rope_pairs, base=10000.0):
+        a, bf16 = oracle._as_array(x)
+        a = a.astype(np.float64)
+        d = a.shape[-1]
+        half = d // 2
+        t = np.asarray(positions, dtype=np.float64).reshape(-1)
+        out = a.copy()
+        for i in range(n_rope_pairs):
+            theta = base ** ((-1.0 if kind == "frequency_exponent" else -2.0) * i / d)
+            j = half - 1 - i if kind == "last_pairs_rotated" else i
+            p0, p1 = (2 * i, 2 * i + 1) if kind == "interleaved_pairs" else (j, j + half)
+            s = np.sin(t * theta)[:, None] * (-1.0 if kind == "sign" else 1.0)
+            c = np.cos(t * theta)[:, None]
+            xi, xj = a[..., :, p0:p0 + 1], a[..., :, p1:p1 + 1]
+            out[..., :, p0:p0 + 1] = xi * c - xj * s
+            out[..., :, p1:p1 + 1] = xi * s + xj * c
+        return out
+    return hope
+
+
+def _qcal_everywhere(self, p, q, k, v, lmk, qs, rows, nthreads=0):
+    k32, v32, l32 = (oracle._widen32(a) for a in (k, v, lmk))
+    return self.rows(p, oracle._widen32(qs), k32, v32, l32, rows)
+
+
+def _qcal_ignored(self, p, q, k, v, lmk, qs, rows, nthreads=0):
+    return self.rows(p, q, k, v, lmk, rows)
+
+
+PY_MUTANTS = [
+    ("gather_ignores_table", oracle, "gather_pages", _gather_ignores_table,
+     pins.pin_paged_decode_is_dense_decode),
+    ("gather_token_major_pages", oracle, "gather_pages", _gather_token_major_pages,
+     pins.pin_paged_decode_is_dense_decode),
+    ("hope_frequency_exponent", oracle, "hope", _hope_variant("frequency_exponent"),
+     pins.pin_hope_rotation_properties),
+    ("hope_last_pairs_rotated", oracle, "hope", _hope_variant("last_pairs_rotated"),
+     pins.pin_hope_rotation_properties),
+    ("hope_interleaved_pairs", oracle, "hope", _hope_variant("interleaved_pairs"),
+     pins.pin_hope_rotation_properties),
+    ("hope_sign", oracle, "hope", _hope_variant("sign"), pins.pin_hope_rotation_properties),
+    ("qcal_query_used_for_attention", oracle.Oracle, "rows_qcal", _qcal_everywhere,
+     pins.pin_qcal_scoring_query),
+    ("qcal_query_ignored", oracle.Oracle, "rows_qcal", _qcal_ignored, pins.pin_qcal_scoring_query),
+]
+
+
+@pytest.mark.parametrize("name,owner,attr,bad,pin", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_python_mutant_is_caught(monkeypatch, name, owner, attr, bad, pin):
+    monkeypatch.setattr(owner, attr, bad)
+    with pytest.raises((AssertionError, ValueError, IndexError)):
+        pin(oracle.default())
