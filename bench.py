@@ -67,6 +67,63 @@ def prefill_work(w: W.Workload) -> dict:
             "candidates": float(n_c.sum() * heads)}
 
 
+def select_executed_flop(w: W.Workload) -> float:
+    """Tensor-core FLOPs the scoring kernel executes over all heads: each
+    128-row tile multiplies its Q tile [128 x d] by ceil(n / 64) landmark
+    tiles of 64 rows, n = the completed chunks of the tile's last row (the
+    rows before it use a triangle of that), plus one 64-row tile of seed
+    landmarks when n > 0."""
+    ntiles = -(-w.L // 128)
+    t_last = np.minimum(np.arange(ntiles, dtype=np.int64) * 128 + 127, w.L - 1)
+    n = np.minimum(t_last // w.C, w.L // w.C)
+    mma_tiles = -(-n // 64) + (n > 0)
+    return float(mma_tiles.sum() * 2 * 128 * 64 * w.d * w.B * w.Hq)
+
+
+def attn_executed_flop(w: W.Workload, tile_union_sizes) -> float:
+    """Tensor-core FLOPs the attention kernel executes: every 128-row tile
+    runs S = Q K^T (2*128*64*d) and O += P V (2*128*64*d) for each chunk of
+    its union (own chunks included), whichever of its rows selected it."""
+    return float(np.asarray(tile_union_sizes, dtype=np.float64).sum() * 4 * 128 * 64 * w.d)
+
+
+def near_tie_sample(w: W.Workload, q, lmk, sel, n_rows=384, seed=0) -> dict:
+    """Sampled check of the selection of the timed run: for n_rows rows the
+    landmark logits of all completed chunks are formed on the host in fp64
+    (plain torch matmul, rounded to fp32 where the kernel decides), ranked by
+    (logit desc, chunk asc), and compared with the GPU's sel_idx.  A near-tie
+    row has its k-th and (k+1)-th logits within 1e-4 * max(1, |s_k|)."""
+    G = w.Hq // w.Hkv
+    rng = np.random.default_rng(seed)
+    rows = rng.integers(0, w.B * w.Hq * w.L, size=n_rows)
+    near = mism = outside = 0
+    for r in rows.tolist():
+        bh, t = divmod(r, w.L)
+        b, hq = divmod(bh, w.Hq)
+        n_c = min(t // w.C, w.L // w.C)
+        got = sel[b, hq, t].cpu().numpy()
+        if n_c == 0:
+            continue
+        qv = q[b, hq, t].double().cpu()
+        lk = lmk[b, hq // G, :n_c].double().cpu()
+        s = ((lk @ qv) * w.scale).float().double().numpy()
+        order = np.lexsort((np.arange(n_c), -s))
+        want = np.sort(order[:w.topk])
+        is_near = False
+        if n_c > w.topk:
+            sk, sk1 = s[order[w.topk - 1]], s[order[w.topk]]
+            is_near = abs(sk - sk1) < 1e-4 * max(1.0, abs(sk))
+        near += int(is_near)
+        g = got[got >= 0]
+        if not np.array_equal(np.sort(g), want):
+            mism += 1
+            outside += int(not is_near)
+    return {"rows": int(n_rows), "near_ties": near, "index_mismatches": mism,
+            "mismatches_outside_near_ties": outside,
+            "how": "logits of all completed chunks in fp64 on the host (torch), ranked "
+                   "(logit desc, chunk asc); rows sampled uniformly over (b, head, position)"}
+
+
 def decode_bytes(w: W.Workload, sel: torch.Tensor) -> float:
     """Algorithmic HBM bytes of one decode step: every landmark key of every
     (b, hkv), plus the K and V of the union of chunks the G query heads of a
@@ -309,7 +366,7 @@ def bench_prefill(hb, synth, w, steps, warmup, ws, rank, seed_offset, e2e=True, 
         a.record(s_in)
         s_cmp.wait_stream(s_in)
         s_out.wait_stream(s_in)
-        n_e2e = max(1, min(steps, 3))
+        n_e2e = max(1, steps)
         for _ in range(n_e2e):
             e2e_step()
         s_out.wait_stream(s_in)
@@ -322,6 +379,7 @@ def bench_prefill(hb, synth, w, steps, warmup, ws, rank, seed_offset, e2e=True, 
         res["d2h"] = ho.numel() * ho.element_size() + hlse.numel() * hlse.element_size()
         res["host_inputs"] = (hq, hk, hv, hl)
     res["sel"] = sel
+    res["inputs"] = (q, lmk)
     return res
 
 
@@ -417,6 +475,12 @@ def bench_hope(hb, w, steps, warmup, train_len=65536, base=500000.0):
     return dict(ms=ms, bytes=nbytes, npairs=npairs)
 
 
+def tile_union_sizes(hb, sel):
+    """Union size of every 128-row tile (the unit the attention kernel walks)."""
+    u_off, _ = hb.union(sel, M=128)
+    return (u_off[1:] - u_off[:-1]).cpu().numpy()
+
+
 def union_stats(hb, sel, w):
     """Chunk-union size per group of M rows and adjacent-query overlap."""
     u_off, _ = hb.union(sel, M=w.M)
@@ -473,6 +537,8 @@ def run_ours(args):
     from chunk_wise_hierarchical_landmark_b200 import synth
     hb.lib()
     w = W.BY_NAME[args.workload]
+    if w.decode:
+        return run_decode_line(hb, synth, w, args, ws, rank)
     res = bench_prefill(hb, synth, w, args.steps, args.warmup, ws, rank, seed_offset=rank)
     ms = max_over_ranks(res["ms"], ws)
     e2e_ms = max_over_ranks(res["e2e_ms"], ws)
@@ -484,9 +550,18 @@ def run_ours(args):
         "hils_select": {"ms": res["sel_ms"], "flop": work["score_flop"]},
         "hils_attn_fwd": {"ms": res["attn_ms"], "flop": work["attn_flop"]},
     }
+    # executed tensor-core work: the scoring kernel's MMA tiles, and the
+    # attention kernel's per-tile unions (from the timed run's selection)
+    sizes = tile_union_sizes(hb, res["sel"])
+    kernels["hils_select"]["exec_flop"] = select_executed_flop(w)
+    kernels["hils_attn_fwd"]["exec_flop"] = attn_executed_flop(w, sizes)
     dom = max(kernels, key=lambda kname: kernels[kname]["ms"])
     peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     achieved = kernels[dom]["flop"] / (kernels[dom]["ms"] * 1e-3) / 1e12
+    achieved_exec = kernels[dom]["exec_flop"] / (kernels[dom]["ms"] * 1e-3) / 1e12
+    alg_total = work["score_flop"] + work["attn_flop"]
+    exec_total = kernels["hils_select"]["exec_flop"] + kernels["hils_attn_fwd"]["exec_flop"]
+    kstep = res["sel_ms"] + res["attn_ms"]
     line = {
         "metric": "HiLS fwd query-tokens/s (prefill, 512K tokens, 7B-shaped GQA 32/8, d=128)",
         "value": qtok / (ms * 1e-3),
@@ -507,11 +582,24 @@ def run_ours(args):
                    "parallelism": f"independent batch per GPU x{ws}"},
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": achieved / peak,
+                     "achieved_executed": achieved_exec, "frac_executed": achieved_exec / peak,
+                     "algorithmic_over_executed": kernels[dom]["flop"] / kernels[dom]["exec_flop"],
                      "peak_source": f"{peak_src} bf16 dense, sustained",
                      "traffic": load_traffic(dom, w.name)},
-        "kernels": {kn: {"ms": round(kv["ms"], 3), "algorithmic_tflops": round(kv["flop"] / (kv["ms"] * 1e-3) / 1e12, 3),
-                         "share": round(kv["ms"] / (res["sel_ms"] + res["attn_ms"]), 3)}
+        "kernels": {kn: {"ms": round(kv["ms"], 3),
+                         "algorithmic_tflops": round(kv["flop"] / (kv["ms"] * 1e-3) / 1e12, 3),
+                         "executed_tflops": round(kv["exec_flop"] / (kv["ms"] * 1e-3) / 1e12, 3),
+                         "frac_algorithmic": round(kv["flop"] / (kv["ms"] * 1e-3) / 1e12 / peak, 4),
+                         "frac_executed": round(kv["exec_flop"] / (kv["ms"] * 1e-3) / 1e12 / peak, 4),
+                         "algorithmic_over_executed": round(kv["flop"] / kv["exec_flop"], 4),
+                         "share": round(kv["ms"] / kstep, 3)}
                     for kn, kv in kernels.items()},
+        "step_fraction": {"algorithmic_tflops": alg_total / (kstep * 1e-3) / 1e12,
+                          "executed_tflops": exec_total / (kstep * 1e-3) / 1e12,
+                          "frac_algorithmic": alg_total / (kstep * 1e-3) / 1e12 / peak,
+                          "frac_executed": exec_total / (kstep * 1e-3) / 1e12 / peak,
+                          "tile_union_mean": round(float(sizes.mean()), 2)},
+        "selection_check": near_tie_sample(w, *res["inputs"], res["sel"], seed=w.seed),
         "e2e": {"value": qtok / (e2e_ms * 1e-3), "unit": "query-tokens/s",
                 "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
                 "pipeline": f"{w.B * w.Hkv} (b, kv-head) groups, one hils_prefill call each; "
@@ -525,18 +613,33 @@ def run_ours(args):
             extra["union"] = union_stats(hb, res["sel"], w)
         except Exception as e:  # statistics only
             extra["union"] = {"error": str(e)[:200]}
-        del res["sel"]
-        w2 = W.PREFILL_128K
-        r2 = bench_prefill(hb, synth, w2, max(3, args.steps), 3, ws, rank, rank, e2e=False,
-                           clocks=False)
-        wk2 = prefill_work(w2)
-        extra[w2.name] = {"value": w2.B * w2.L * ws / (max_over_ranks(r2["ms"], ws) * 1e-3),
-                          "unit": "query-tokens/s", "ms_per_step": r2["ms"],
-                          "select_ms": r2["sel_ms"], "attn_ms": r2["attn_ms"],
-                          "attn_tflops": wk2["attn_flop"] / (r2["attn_ms"] * 1e-3) / 1e12,
-                          "select_tflops": wk2["score_flop"] / (r2["sel_ms"] * 1e-3) / 1e12}
-        del r2
+        del res["sel"], res["inputs"]
         torch.cuda.empty_cache()
+        # the other prefill configurations: 128K 7B-shaped, 32K small model,
+        # and the tiny fp32 one (CUDA-core kernels: no tensor-core fraction)
+        for w2 in (W.PREFILL_128K, W.SMALL_32K, W.TINY_F32):
+            r2 = bench_prefill(hb, synth, w2, max(5, args.steps), 3, ws, rank, rank, e2e=False,
+                               clocks=False)
+            wk2 = prefill_work(w2)
+            ent = {"value": w2.B * w2.L * ws / (max_over_ranks(r2["ms"], ws) * 1e-3),
+                   "unit": "query-tokens/s", "ms_per_step": r2["ms"],
+                   "select_ms": r2["sel_ms"], "attn_ms": r2["attn_ms"],
+                   "dtype": w2.dtype,
+                   "attn_tflops": wk2["attn_flop"] / (r2["attn_ms"] * 1e-3) / 1e12,
+                   "select_tflops": wk2["score_flop"] / (r2["sel_ms"] * 1e-3) / 1e12}
+            if w2.dtype == "bf16":
+                sz2 = tile_union_sizes(hb, r2["sel"])
+                ex_s, ex_a = select_executed_flop(w2), attn_executed_flop(w2, sz2)
+                ent["attn_executed_tflops"] = ex_a / (r2["attn_ms"] * 1e-3) / 1e12
+                ent["select_executed_tflops"] = ex_s / (r2["sel_ms"] * 1e-3) / 1e12
+                ent["frac_algorithmic"] = (wk2["attn_flop"] + wk2["score_flop"]) / (r2["ms"] * 1e-3) / 1e12 / peak
+                ent["frac_executed"] = (ex_a + ex_s) / (r2["ms"] * 1e-3) / 1e12 / peak
+                ent["tile_union_mean"] = round(float(sz2.mean()), 2)
+                ent["selection_check"] = near_tie_sample(w2, *r2["inputs"], r2["sel"], n_rows=128,
+                                                         seed=w2.seed)
+            extra[w2.name] = ent
+            del r2
+            torch.cuda.empty_cache()
         w3 = W.DECODE_512K
         r3 = bench_decode(hb, synth, w3, max(5, args.steps), 3, rank, paged=True)
         gbs = r3["bytes"] / (r3["ms"] * 1e-3) / 1e9
@@ -567,6 +670,31 @@ def run_ours(args):
         line["workloads"] = extra
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, res["host_inputs"])
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_decode_line(hb, synth, w, args, ws, rank):
+    """A decode workload as the main line (used for profiler captures of the
+    decode kernels on a reduced batch): step = one hils_decode_fwd call."""
+    peaks, peak_src = load_peaks()
+    n0 = hb.launch_count()
+    r = bench_decode(hb, synth, w, args.steps, args.warmup, rank)
+    launches = hb.launch_count() - n0
+    ms = max_over_ranks(r["ms"], ws)
+    gbs = r["bytes"] / (r["ms"] * 1e-3) / 1e9
+    line = {"metric": "HiLS decode query-tokens/s", "value": w.B * ws / (ms * 1e-3),
+            "unit": "query-tokens/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded; per-rank seed offset)",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.L,
+                       "d": w.d, "chunk": w.C, "topk": w.topk},
+            "roofline": {"bound": "hbm", "kernel": "hils_decode_fwd", "achieved": gbs,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                         "peak_source": f"{peak_src} HBM copy", "traffic": None},
+            "gpu_launches": launches}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:
@@ -627,11 +755,12 @@ def main():
     ap.add_argument("--hq", type=int, default=None,
                     help="override the query-head count (smaller cases for profiler captures)")
     ap.add_argument("--hkv", type=int, default=None, help="override the KV-head count")
+    ap.add_argument("--batch", type=int, default=None, help="override the batch size")
     args = ap.parse_args()
-    if args.hq or args.hkv:
+    if args.hq or args.hkv or args.batch:
         base = W.BY_NAME[args.workload]
-        w = base.with_(Hq=args.hq or base.Hq, Hkv=args.hkv or base.Hkv)
-        w = w.with_(name=f"{base.name}_hq{w.Hq}_hkv{w.Hkv}")
+        w = base.with_(Hq=args.hq or base.Hq, Hkv=args.hkv or base.Hkv, B=args.batch or base.B)
+        w = w.with_(name=f"{base.name}_b{w.B}_hq{w.Hq}_hkv{w.Hkv}")
         W.BY_NAME[w.name] = w
         args.workload = w.name
     if args.impl == "reference":

@@ -18,8 +18,13 @@
 //    race on it and must be serialised by the caller;
 //  - the first call on a device looks the array's device address up with
 //    cudaGetSymbolAddress (which can load the library's module on that
-//    device); make that first call before any stream capture.
+//    device); make that first call before any stream capture.  The address
+//    is tied to the device's context: when the context changes (a
+//    cudaDeviceReset, or a primary context released and created again), the
+//    module is loaded anew and the next call looks the address up again.
 // No cudaMalloc, cudaFree or allocating library routine is called here.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "../../include/hils.h"
@@ -32,10 +37,40 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void *g_scratch_addr[kMaxDevices];  // device address of g_decode_scratch, per device
+void *g_scratch_addr[kMaxDevices];          // device address of g_decode_scratch, per device
+unsigned long long g_scratch_ctx[kMaxDevices];  // id of the context it was resolved in
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// Unique id of the calling thread's current context (0 if it cannot be read;
+// then the cached address is trusted as it is).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void *f1 = nullptr, *f2 = nullptr;
+    cudaDriverEntryPointQueryResult r1, r2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &r1) == cudaSuccess &&
+        r1 == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &r2) == cudaSuccess &&
+        r2 == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(f2);
+    looked_up = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx &&
+      get_id(ctx, &id) == CUDA_SUCCESS)
+    return id;
+  return 0;
+}
 
 // Device address of the scratch array on the current device (set-up on the
-// first call per device).  Returns nullptr and fills *e on failure.
+// first call per device, and again whenever the device's context changed).
+// Returns nullptr and fills *e on failure.
 void *scratch_on_current_device(cudaError_t *e) {
   int dev = -1;
   *e = cudaGetDevice(&dev);
@@ -45,11 +80,18 @@ void *scratch_on_current_device(cudaError_t *e) {
     return nullptr;
   }
   std::lock_guard<std::mutex> lock(g_mu);
+  // cudaGetSymbolAddress makes the device's primary context current, so the
+  // context is read after it on the first call
+  if (g_scratch_addr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (ctx != 0 && ctx != g_scratch_ctx[dev]) g_scratch_addr[dev] = nullptr;
+  }
   if (!g_scratch_addr[dev]) {
     void *ptr = nullptr;
     *e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
     if (*e != cudaSuccess) return nullptr;
     g_scratch_addr[dev] = ptr;
+    g_scratch_ctx[dev] = current_context_id();
   }
   *e = cudaSuccess;
   return g_scratch_addr[dev];

@@ -75,7 +75,11 @@ typedef struct {
   int d;          /* head dimension */
   int chunk;      /* C, tokens per chunk */
   int topk;       /* k, chunks selected per query */
-  int M;          /* adjacent queries per group for the chunk union */
+  int M;          /* adjacent queries per group of hils_union (16, 32, 64
+                     or 128).  The prefill kernels do not read it: they
+                     always load the union of a 128-row tile (the tensor
+                     core's full-rate M), so their results do not depend
+                     on it */
   float scale;    /* softmax scale of token and landmark logits (1/sqrt(d)) */
   int dtype;      /* hils_dtype of q, k, v, lmk_k and out */
   int debug_checks; /* 0 or 1, see above */
@@ -196,7 +200,10 @@ hils_status hils_decode_fwd_paged(const hils_params *p, const void *q, const voi
  * (held on every GPU that loads the library until the process exits); shapes
  * that need more scratch return HILS_ERR_WORKSPACE before any launch.  The
  * first call on a device looks the array up (cudaGetSymbolAddress, which may
- * load the library's module there): make it before any stream capture.  All
+ * load the library's module there): make it before any stream capture.  The
+ * address belongs to the device's context; after the context changes (e.g.
+ * cudaDeviceReset) the next call looks it up again, so that call too should
+ * come before any stream capture.  All
  * calls share the array and it keeps the last call's contents (each call
  * writes every scratch entry it reads); calls that overlap on the GPU race
  * and must be serialised by the caller.  Nothing here allocates.

@@ -45,3 +45,42 @@ def test_traffic_record_follows_its_sources(tmp_path, monkeypatch):
     path.write_text(json.dumps(rec))
     assert bench.load_traffic("hils_attn_fwd", "wl") is None
 
+
+def test_select_executed_flop_counts_mma_tiles():
+    w = W.PREFILL_128K.with_(B=1, Hq=2, Hkv=1, L=64 * 300 + 5, d=64, topk=4)
+    want = 0
+    for t0 in range(0, w.L, 128):
+        t_last = min(t0 + 127, w.L - 1)
+        n = min(t_last // w.C, w.L // w.C)
+        tiles = -(-n // 64) + (1 if n > 0 else 0)
+        want += tiles * 2 * 128 * 64 * w.d
+    assert bench.select_executed_flop(w) == want * w.B * w.Hq
+
+
+def test_near_tie_sample_flags_a_wrong_selection():
+    """The bench's sampled selection check agrees with the oracle's top-k and
+    counts a planted wrong index outside any near-tie."""
+    import numpy as np
+    import oracle
+    from chunk_wise_hierarchical_landmark_b200 import synth
+    w = W.PREFILL_128K.with_(Hq=2, Hkv=1, L=640, topk=3)
+    q, k, v, lmk = synth.make_inputs(w, "cpu")
+    p = oracle.Problem(w.B, w.Hq, w.Hkv, w.L, w.d, w.C, w.topk, w.scale)
+    rows = np.arange(w.B * w.Hq * w.L)
+    ref = oracle.rows(p, q, k, v, lmk, rows)
+    sel = torch.from_numpy(np.ascontiguousarray(ref["sel"])).reshape(w.B, w.Hq, w.L, w.topk)
+    st = bench.near_tie_sample(w, q, lmk, sel, n_rows=200, seed=3)
+    assert st["index_mismatches"] == st["mismatches_outside_near_ties"] == 0
+    # plant a wrong chunk in every sampled row that has more than k candidates
+    rs = np.random.default_rng(3).integers(0, w.B * w.Hq * w.L, size=200)
+    bad = sel.clone()
+    planted = 0
+    for r in set(rs.tolist()):
+        bh, t = divmod(r, w.L)
+        if t // w.C > w.topk:
+            row = bad[0, bh, t]
+            unused = [c for c in range(t // w.C) if c not in row.tolist()]
+            row[0] = unused[0]
+            planted += 1
+    st = bench.near_tie_sample(w, q, lmk, bad, n_rows=200, seed=3)
+    assert planted > 0 and st["index_mismatches"] >= planted - st["near_ties"]

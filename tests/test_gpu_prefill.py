@@ -97,13 +97,14 @@ def test_deterministic():
 
 
 def test_group_size_does_not_change_results():
-    """M only changes which chunk tiles are loaded together."""
+    """The prefill kernels always walk 128-row tiles; M only sets the groups
+    hils_union reports.  Every output is therefore bit-identical across M."""
     w = W.PREFILL_128K.with_(Hq=4, Hkv=1, L=2048)
     q, k, v, lmk = (x.cuda() for x in synth.make_inputs(w, "cpu"))
-    outs = [gpu_prefill(q, k, v, lmk, w.with_(M=m)) for m in (16, 64, 128)]
+    outs = [gpu_prefill(q, k, v, lmk, w.with_(M=m)) for m in (16, 32, 64, 128)]
     for o in outs[1:]:
-        assert torch.equal(o["sel"], outs[0]["sel"])
-        assert (o["out"].float() - outs[0]["out"].float()).abs().max().item() <= 2 ** -7
+        for key in ("sel", "w", "lse_lmk", "out", "lse"):
+            assert torch.equal(o[key], outs[0][key]), key
 
 
 def test_union_matches_oracle():

@@ -28,14 +28,18 @@ def _outputs(w, dev):
     )
 
 
-@pytest.mark.parametrize("w", [
-    W.DECODE_512K.with_(B=2, L=3000, topk=16),
-    W.DECODE_512K.with_(B=16, L=524288),          # the full decode workload (17.6 MB of scratch)
-], ids=["small", "full"])
-def test_noalloc_matches_workspace_decode_twice(w):
+@pytest.mark.parametrize("w,debug", [
+    (W.DECODE_512K.with_(B=2, L=3000, topk=16), False),
+    (W.DECODE_512K.with_(B=2, Hq=8, Hkv=2, L=2500, d=64, topk=8, dtype="f32"), False),
+    # debug mode: the error word sits at the start of the library's array
+    (W.DECODE_512K.with_(B=2, L=3000, topk=16), True),
+    (W.DECODE_512K.with_(B=16, L=524288), False),  # the full decode workload (17.6 MB of scratch)
+], ids=["small", "small_f32", "small_debug", "full"])
+def test_noalloc_matches_workspace_decode_twice(w, debug):
     dev = torch.device("cuda")
     q, k, v, lmk = synth.make_inputs(w, "cuda")
-    p = hb.make_params(w.B, w.Hq, w.Hkv, w.L, w.d, w.topk, w.M, w.C, w.scale, q.dtype)
+    p = hb.make_params(w.B, w.Hq, w.Hkv, w.L, w.d, w.topk, w.M, w.C, w.scale, q.dtype,
+                       debug_checks=debug)
     ref = _outputs(w, dev)
     hb.hils_decode_fwd(p, q, k, v, lmk, ref["sel"], ref["w"], ref["lse_lmk"], ref["out"],
                        ref["lse"], hb.workspace(p, hb.HILS_OP_DECODE, dev))
