@@ -69,15 +69,17 @@ def prefill_work(w: W.Workload) -> dict:
 
 def select_executed_flop(w: W.Workload) -> float:
     """Tensor-core FLOPs the scoring kernel executes over all heads: each
-    128-row tile multiplies its Q tile [128 x d] by ceil(n / 64) landmark
-    tiles of 64 rows, n = the completed chunks of the tile's last row (the
-    rows before it use a triangle of that), plus one 64-row tile of seed
-    landmarks when n > 0."""
+    128-row tile multiplies its Q tile [128 x d] by one 64-row tile of seed
+    landmarks when n > 0, n = the completed chunks of the tile's last row,
+    and, when n > k (some candidate is not a seed), by ceil(n / 64) landmark
+    tiles of 64 rows with one extra K = 16 step each (the masking step), the
+    rows before the last using a triangle of that."""
     ntiles = -(-w.L // 128)
     t_last = np.minimum(np.arange(ntiles, dtype=np.int64) * 128 + 127, w.L - 1)
     n = np.minimum(t_last // w.C, w.L // w.C)
-    mma_tiles = -(-n // 64) + (n > 0)
-    return float(mma_tiles.sum() * 2 * 128 * 64 * w.d * w.B * w.Hq)
+    seed = (n > 0).astype(np.int64) * w.d
+    scan = np.where(n > w.topk, -(-n // 64), 0) * (w.d + 16)
+    return float((seed + scan).sum() * 2 * 128 * 64 * w.B * w.Hq)
 
 
 def attn_executed_flop(w: W.Workload, tile_union_sizes) -> float:

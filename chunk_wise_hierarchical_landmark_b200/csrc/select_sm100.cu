@@ -4,33 +4,39 @@
 // t the logits s_c = scale * <q_t, lmk_c> of its completed chunks c < t/C,
 // their log-sum-exp, and the k best by (s desc, c asc).
 //
-// One CTA = 128 query rows of one (b, hq); two CTAs share an SM.  6 warps:
+// One CTA = 128 query rows of one (b, hq); two CTAs share an SM.  10 warps:
 //   warp 0     TMA producer: the Q tile into the landmark ring (staging), then
-//              64-landmark tiles of the row block's KV head into a 2-stage ring;
-//   warp 1     TMEM owner, MMA issuer: the seed scores, then S = Q Lmk^T
-//              (128 x 64 fp32) per landmark tile into one of two TMEM buffers,
-//              with Q as the A operand in tensor memory;
-//   warps 2-5  one thread per row (TMEM lane): copy the row's q into tensor
-//              memory, stage the seed landmarks, start the row's top-k from
-//              the seeds, then per 32-candidate block an online log-sum-exp
-//              (base 2) and, when the block's best score can enter, the
-//              insertion of its qualifying candidates (staged in shared memory,
-//              one per lane per step, so the 32 rows of a warp insert
-//              together).  The row's best k keys live in shared memory (8
-//              groups of 8 slots, group minima in registers).
+//              64-landmark tiles of the row block's KV head into a 2-stage
+//              ring, each with a small bias tile (below) written beside it;
+//   warp 1     TMEM owner, MMA issuer: the seed scores, then per landmark tile
+//              S = Q Lmk^T + bias (128 x 64 fp32) into one of two TMEM
+//              buffers, with Q as the A operand in tensor memory;
+//   warps 2-9  two threads per row: warps 2-5 (the row's "owner") read columns
+//              [0, 32) of every score tile, warps 6-9 columns [32, 64).  Each
+//              keeps an online log-sum-exp (base 2) of its half; the row's
+//              best k keys live in shared memory and only the owner changes
+//              them: the other thread posts the candidates that beat the
+//              row's threshold into a 4-entry mailbox the owner drains once
+//              per tile.
 // Seeds.  Every row's top-k starts from k chunks (the seeds) whose scores an
 // extra MMA computes first: the k-th best seed bounds the row's k-th best
 // score from below (the seeds are candidates too), so the result stays exact
-// and the scan only inserts what beats that bound; seeds are masked out of
-// the scan, and since kept chunks are then not all earlier than the scan
-// position, equal scores are resolved on the full key.  The row tiles run in
+// and the scan only inserts what beats that bound.  The row tiles run in
 // kLevels launches: tiles of level 0 start from the chunks 0..k-1 (where a
 // plain scan starts), tiles of later levels from the selection of the last
 // row of a tile an earlier level finished (1, 2, 4, ... tiles before them),
 // which adjacent queries largely share.
-// The hot loop is kept small (one 32-candidate block per iteration, the rare
-// paths not unrolled): the kernel is bound by instruction issue, and code
-// that does not fit the instruction caches stalls it.
+// Masking on the tensor core.  The seeds (already counted, in the top-k and
+// in the log-sum-exp, from their own MMA) and the chunks a row may not see
+// (the tile's first own chunk for its first 64 rows, and every column past
+// the tile's last candidate) are pushed to -1e30 by one more K = 16 step of
+// the scoring MMA: A = [1, (row < 64)] per row (8 TMEM columns), B = per
+// landmark column [-1e30 if a seed or beyond the candidates, -1e30 if the
+// boundary chunk] (written by the producer while the tile's TMA is in
+// flight, and only for tiles that hold a seed or the boundary).  For every
+// other column that step adds exact zeros, so the scores are unchanged; the
+// row threads then need no per-block masks, and blocks holding seeds no
+// longer pass the top-k prefilter.
 // The candidate scores never leave the chip.
 #include <cuda_bf16.h>
 
@@ -45,10 +51,15 @@ using namespace sm100;
 
 constexpr int kRows = 128;
 constexpr int kTile = 64;     // landmarks per MMA tile (UMMA N)
-constexpr int kStages = 2;
-constexpr int kSBufs = 3;     // score tiles in tensor memory
-constexpr int kThreads = 192;
+constexpr int kStages = 2;    // landmark ring
+constexpr int kSBufs = 2;     // score tiles in tensor memory
+constexpr int kRowThreads = 2 * kRows;
+constexpr int kThreads = 64 + kRowThreads;
 constexpr int kMaxK = 64;
+constexpr int kMbox = 4;      // mailbox entries per row
+constexpr uint32_t kDone = 0x80000000u;
+// a score below this (unscaled) was pushed down by the masking step
+constexpr float kMaskedBelow = -1.0e29f;
 // Row tiles run in kLevels launches (levels): with P = 2^(kLevels-1), level 0
 // takes the tiles P*i unseeded and level j >= 1 the tiles at offset P/2^j in
 // periods of P/2^(j-1), each seeded by the tile offset positions earlier
@@ -72,22 +83,30 @@ struct SelLayout {
   static constexpr int kQBytes = kRows * D * 2;
   static constexpr int kLBytes = kTile * D * 2;
   static_assert(kStages * kLBytes == kQBytes, "the landmark ring stages the Q tile");
-  static constexpr int l0 = 0;                               // landmark ring / Q staging
-  static constexpr int heap = l0 + kStages * kLBytes;        // [kMaxK][128] uint64 slots
-  static constexpr int stage = heap + kMaxK * kRows * 8;     // [32][128] fp32 candidate staging
-  static constexpr int bars = stage + 32 * kRows * 4;
+  static constexpr int l0 = 0;                               // landmark ring / Q / seed staging
+  static constexpr int bias = l0 + kStages * kLBytes;        // [64 rows][128 B], 128-byte swizzle
+  static constexpr int heap = bias + kTile * 128;            // [kMaxK][128] uint64 slots
+  static constexpr int mbox = heap + kMaxK * kRows * 8;      // [kMbox][128] uint64 keys
+  static constexpr int tail = mbox + kMbox * kRows * 8;      // [128] posted count (+ done bit)
+  static constexpr int head = tail + kRows * 4;              // [128] drained count
+  static constexpr int thr = head + kRows * 4;               // [128] prefilter bound
+  static constexpr int lsep = thr + kRows * 4;               // [128] (m2, l) of the second half
+  static constexpr int bars = lsep + kRows * 8;
   static constexpr int misc = bars + 16 * 8;
   static constexpr int seeds = misc + 32;                     // [kMaxK] int seed chunk ids
   static constexpr int total = seeds + kMaxK * 4;
-  // TMEM columns: Q [0, D/2) as bf16 pairs, S0..S2 [64, 256)
-  static constexpr uint32_t kQCol = 0, kSCol = 64, kTmemCols = 256;
+  static_assert(bias % 1024 == 0, "swizzled tiles are 1024-byte aligned");
+  // TMEM columns: Q [0, D/2) as bf16 pairs, the masking A operand [64, 72),
+  // score buffers [128, 192) and [192, 256)
+  static constexpr uint32_t kQCol = 0, kBiasCol = 64, kSCol = 128, kTmemCols = 256;
   static_assert(kSCol + kSBufs * kTile <= kTmemCols, "score tiles fit the allocation");
 };
 
 struct SelBars {
-  uint64_t q_smem, q_tmem, l_full[kStages], l_empty[kStages], s_full[kSBufs], s_empty[kSBufs], done,
-      seed_ready, seed_full, seed_read;
+  uint64_t q_smem, q_tmem, l_full[kStages], l_empty[kStages], s_full[kSBufs], s_empty[kSBufs],
+      seed_ready, seed_full, seed_read, seed_done, done;
 };
+static_assert(sizeof(SelBars) <= 16 * 8, "barrier area");
 
 // Per-row top-k: kMaxK key slots in shared memory (slot i of the row at
 // h[i * 128]) in 8 groups of 8, each group's minimum (key and position) kept
@@ -167,6 +186,20 @@ __device__ __forceinline__ float prefilter(float thr, float inv_scale) {
   if (isinf(thr)) return thr;
   const float u = thr * inv_scale;
   return u - fabsf(u) * 0x1p-20f - 0x1p-100f;
+}
+
+// a[j] for a j known only at run time, by a tree of selects (no local memory)
+__device__ __forceinline__ float pick32(const float (&a)[32], int j) {
+  float b16[16], b8[8], b4[4], b2[2];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) b16[i] = (j & 16) ? a[i + 16] : a[i];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) b8[i] = (j & 8) ? b16[i + 8] : b16[i];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) b4[i] = (j & 4) ? b8[i + 4] : b8[i];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) b2[i] = (j & 2) ? b4[i + 2] : b4[i];
+  return (j & 1) ? b2[1] : b2[0];
 }
 
 // Writes a row's first cnt kept keys in slot order (ids, logits; -1 / -inf
@@ -265,6 +298,57 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// The two threads of every row (warps 2-9) meet here.
+__device__ __forceinline__ void rows_sync() {
+  __syncwarp();
+  asm volatile("bar.sync 1, %0;" ::"n"(kRowThreads) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_vol(const uint32_t *p) { return *reinterpret_cast<const volatile uint32_t *>(p); }
+__device__ __forceinline__ void st_vol(uint32_t *p, uint32_t v) { *reinterpret_cast<volatile uint32_t *>(p) = v; }
+__device__ __forceinline__ float ld_volf(const float *p) { return *reinterpret_cast<const volatile float *>(p); }
+__device__ __forceinline__ void st_volf(float *p, float v) { *reinterpret_cast<volatile float *>(p) = v; }
+
+// Online log-sum-exp (base 2) of one 32-candidate block with block maximum
+// bm (unscaled); c2 = scale * log2(e).  Blocks whose every entry was masked
+// (bm below kMaskedBelow) add nothing.
+__device__ __forceinline__ void lse_block(const float (&a)[32], float bm, float c2, float &m2,
+                                          float &l) {
+  if (!(bm > kMaskedBelow)) return;
+  const float bm2 = bm * c2;
+  if (bm2 > m2) {
+    l *= ex2_approx(m2 - bm2);
+    m2 = bm2;
+  }
+  // pairs of candidates through packed f32x2 FMA and add
+  const float2 c2v = make_float2(c2, c2), nm2 = make_float2(-m2, -m2);
+  float2 ps[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float2 y = __ffma2_rn(make_float2(a[2 * j], a[2 * j + 1]), c2v, nm2);
+    ps[j & 1] = __fadd2_rn(ps[j & 1], make_float2(ex2_approx(y.x), ex2_approx(y.y)));
+  }
+  l += (ps[0].x + ps[1].x) + (ps[0].y + ps[1].y);
+}
+
+__device__ __forceinline__ float block_max(const float (&a)[32]) {
+  // a tree of three-input maxima (32 -> 11 -> 4 -> 1)
+  float y[11];
+#pragma unroll
+  for (int j = 0; j < 10; ++j) y[j] = max3f(a[3 * j], a[3 * j + 1], a[3 * j + 2]);
+  y[10] = fmaxf(a[30], a[31]);
+  return max3f(max3f(y[0], y[1], y[2]), max3f(y[3], y[4], y[5]),
+               max3f(y[6], y[7], max3f(y[8], y[9], y[10])));
+}
+
+// bit j set where a[j] >= u
+__device__ __forceinline__ uint32_t ge_mask(const float (&a)[32], float u) {
+  uint32_t mq[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int j = 0; j < 32; ++j) mq[j >> 3] |= a[j] >= u ? (1u << j) : 0u;
+  return (mq[0] | mq[1]) | (mq[2] | mq[3]);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
     select_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -285,7 +369,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::misc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::misc + 4);
   volatile int *nseed_slot = reinterpret_cast<volatile int *>(smem + Lay::misc + 8);
+  volatile int *bias_flag = reinterpret_cast<volatile int *>(smem + Lay::misc + 16);  // [kStages]
   int *seed_list = reinterpret_cast<int *>(smem + Lay::seeds);
+  uint32_t *tail_s = reinterpret_cast<uint32_t *>(smem + Lay::tail);
+  uint32_t *head_s = reinterpret_cast<uint32_t *>(smem + Lay::head);
+  float *thr_s = reinterpret_cast<float *>(smem + Lay::thr);
+  float2 *lsep_s = reinterpret_cast<float2 *>(smem + Lay::lsep);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
@@ -304,21 +393,26 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_smem, 1);
-    mbar_init(&bars->q_tmem, kRows);
+    mbar_init(&bars->q_tmem, kRowThreads);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->l_full[s], 1);
+      mbar_init(&bars->l_full[s], 2);  // the TMA's bytes + the masking operand
       mbar_init(&bars->l_empty[s], 1);
     }
     for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->s_empty[i], kRows);
+      mbar_init(&bars->s_empty[i], kRowThreads);
     }
-    mbar_init(&bars->done, 1);
-    mbar_init(&bars->seed_ready, kRows);
+    mbar_init(&bars->seed_ready, kRowThreads);
     mbar_init(&bars->seed_full, 1);
-    mbar_init(&bars->seed_read, kRows);
+    mbar_init(&bars->seed_read, kRowThreads);
+    mbar_init(&bars->seed_done, 1);
+    mbar_init(&bars->done, 1);
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  if (threadIdx.x < kRows) {
+    tail_s[threadIdx.x] = 0u;
+    head_s[threadIdx.x] = 0u;
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_q);
@@ -363,45 +457,101 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const int ns = *nseed_slot;
+  // every candidate a seed (a short prefix): nothing left to scan
+  const int n_scan = ns < n_cand ? n_ltiles : 0;
   const uint32_t tmem = *tmem_slot;
   const uint32_t q_tmem = tmem + Lay::kQCol;
+  const uint32_t bias_tmem = tmem + Lay::kBiasCol;
   const uint32_t s_tmem0 = tmem + Lay::kSCol;  // score tile sb at s_tmem0 + sb * kTile
   const uint32_t seed_tmem = s_tmem0 + (kSBufs - 1) * kTile;  // free until tile kSBufs - 1
+  unsigned char *seed_stage = smem + Lay::l0 + (kStages - 1) * Lay::kLBytes;
   const int lrow0 = (b * rs.Hkv + hkv) * nlmk;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && n_ltiles > 0) {
-      mbar_expect_tx(&bars->q_smem, Lay::kQBytes);
-      for (int kb = 0; kb < D / 64; ++kb)
-        tma_load_2d(smem + Lay::l0 + kb * kRows * 128, &tm_q, &bars->q_smem, kb * 64, bh * L + t0);
-      // the ring holds the Q tile until the row threads have moved it to TMEM
-      const bool ok = mbar_wait(&bars->q_tmem, 0, abort_flag);
-      int issued = 0;
-      for (int i = 0; ok && i < n_ltiles; ++i) {
-        const int s = i % kStages;
-        if (i >= kStages && !mbar_wait(&bars->l_empty[s], ((i / kStages) - 1) & 1, abort_flag))
-          break;
-        mbar_expect_tx(&bars->l_full[s], Lay::kLBytes);
-        unsigned char *ls = smem + Lay::l0 + s * Lay::kLBytes;
+    if (n_ltiles > 0) {
+      if (lane == 0) {
+        mbar_expect_tx(&bars->q_smem, Lay::kQBytes);
         for (int kb = 0; kb < D / 64; ++kb)
-          tma_load_2d(ls + kb * kTile * 128, &tm_l, &bars->l_full[s], kb * 64, lrow0 + i * kTile);
-        ++issued;
+          tma_load_2d(smem + Lay::l0 + kb * kRows * 128, &tm_q, &bars->q_smem, kb * 64, bh * L + t0);
       }
-      for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-        mbar_wait_bounded(&bars->l_full[i % kStages], (i / kStages) & 1);
-      mbar_wait_bounded(&bars->q_smem, 0);
+      // the ring holds the Q tile until the row threads have moved it to TMEM
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->q_tmem, 0, abort_flag));
+      const __nv_bfloat16 negb = __float2bfloat16_rn(-1.0e30f);
+      const uint32_t neg = (uint32_t)__bfloat16_as_ushort(negb);
+      int issued = 0;
+      int cur = 0;  // seeds below tile i's columns have been passed
+      for (int i = 0; ok && i < n_scan; ++i) {
+        const int s = i % kStages;
+        bool w = true;
+        if (i >= kStages) w = mbar_wait(&bars->l_empty[s], ((i / kStages) - 1) & 1, abort_flag);
+        // the seed tile sits in the last ring stage until the seed MMA is done
+        if (w && i == kStages - 1) w = mbar_wait(&bars->seed_done, 0, abort_flag);
+        if (!__all_sync(0xffffffffu, w)) break;
+        // the landmark tile first (arrival 1 of 2, with its bytes) ...
+        if (lane == 0) {
+          mbar_expect_tx(&bars->l_full[s], Lay::kLBytes);
+          unsigned char *ls = smem + Lay::l0 + s * Lay::kLBytes;
+          for (int kb = 0; kb < D / 64; ++kb)
+            tma_load_2d(ls + kb * kTile * 128, &tm_l, &bars->l_full[s], kb * 64, lrow0 + i * kTile);
+        }
+        ++issued;
+        // ... then, while it is in flight, the seeds among its columns (the
+        // ascending seed list walked 32 entries at a time) ...
+        const int c0 = i * kTile;
+        uint32_t m_lo = 0u, m_hi = 0u;
+        for (;;) {
+          const int idx = cur + lane;
+          const int c = idx < ns ? seed_list[idx] : INT_MAX;
+          const bool in = c < c0 + kTile;
+          const uint32_t bal = __ballot_sync(0xffffffffu, in);
+          const int rel = c - c0;
+          m_lo |= __reduce_or_sync(0xffffffffu, in && rel < 32 ? (1u << rel) : 0u);
+          m_hi |= __reduce_or_sync(0xffffffffu, in && rel >= 32 ? (1u << (rel - 32)) : 0u);
+          cur += __popc(bal);
+          if (bal != 0xffffffffu) break;
+        }
+        // ... and, for a tile that holds seeds or the row boundary (the last
+        // one), its masking operand, K-slice s of the swizzled bias tile:
+        // element 0 = -1e30 for seeds and columns past the candidates,
+        // element 1 = -1e30 for the boundary chunk (first 64 rows only)
+        const bool need = (m_lo | m_hi) != 0u || i == n_ltiles - 1;
+        if (need) {
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int rr = lane + 32 * u;
+            const int c = c0 + rr;
+            const bool seed = ((u ? m_hi : m_lo) >> lane) & 1u;
+            const uint32_t e0 = (seed || c >= n_cand) ? neg : 0u;
+            const uint32_t e1 = (c == n_lo) ? neg : 0u;
+            unsigned char *row = smem + Lay::bias + (rr >> 3) * 1024 + (rr & 7) * 128;
+            *reinterpret_cast<uint4 *>(row + (((2 * s) ^ (rr & 7)) << 4)) = make_uint4(e0 | (e1 << 16), 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(row + (((2 * s + 1) ^ (rr & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          bias_flag[s] = need ? 1 : 0;
+          mbar_arrive(&bars->l_full[s]);  // arrival 2 of 2
+        }
+      }
+      if (lane == 0) {
+        for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+          mbar_wait_bounded(&bars->l_full[i % kStages], (i / kStages) & 1);
+        mbar_wait_bounded(&bars->q_smem, 0);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_ltiles > 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kRows, kTile, false, false);
       bool ok = mbar_wait(&bars->q_tmem, 0, abort_flag);
-      // seed scores: S1 = Q * seeds^T (the seed landmark rows, staged by the rows)
+      // seed scores: Q * seeds^T (the seed landmark rows, staged by the rows)
       ok = ok && mbar_wait(&bars->seed_ready, 0, abort_flag);
       tc_fence_after();
       if (ok) {
-        const uint32_t sd_addr = smem_u32(smem + Lay::stage);
+        const uint32_t sd_addr = smem_u32(seed_stage);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int kb = kk >> 2, kw = kk & 3;
@@ -409,20 +559,26 @@ __global__ void __launch_bounds__(kThreads, 2)
           mma_bf16_ts(seed_tmem, q_tmem + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars->seed_full);
+        mma_commit(&bars->seed_done);
       }
-      for (int i = 0; ok && i < n_ltiles; ++i) {
+      const uint32_t bias_addr = smem_u32(smem + Lay::bias);
+      for (int i = 0; ok && i < n_scan; ++i) {
         const int s = i % kStages, sb = i % kSBufs;
         if (!mbar_wait(&bars->l_full[s], (i / kStages) & 1, abort_flag)) break;
         if (i >= kSBufs && !mbar_wait(&bars->s_empty[sb], ((i / kSBufs) - 1) & 1, abort_flag)) break;
         if (i == kSBufs - 1 && !mbar_wait(&bars->seed_read, 0, abort_flag)) break;
         tc_fence_after();
         const uint32_t l_addr = smem_u32(smem + Lay::l0 + s * Lay::kLBytes);
+        const uint32_t d_tmem = s_tmem0 + sb * kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int kb = kk >> 2, kw = kk & 3;
           const uint64_t bd = smem_desc_sw128(l_addr + kb * kTile * 128 + kw * 32, 16, 1024);
-          mma_bf16_ts((s_tmem0 + sb * kTile), q_tmem + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
+          mma_bf16_ts(d_tmem, q_tmem + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
         }
+        // the masking step, on tiles that need one: S += [1, row < 64] * bias_s^T
+        if (bias_flag[s])
+          mma_bf16_ts(d_tmem, bias_tmem, smem_desc_sw128(bias_addr + s * 32, 16, 1024), idesc, 1u);
         mma_commit(&bars->s_full[sb]);
         mma_commit(&bars->l_empty[s]);
       }
@@ -431,19 +587,25 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   } else {
     // ---------------------------------------------------------- row threads
-    const int r = 32 * (warp & 3) + lane;
+    const int h = (warp - 2) >> 2;         // 0: owner, columns [0, 32); 1: columns [32, 64)
+    const int r = 32 * (warp & 3) + lane;  // TMEM lane == tile row
+    const int rt = r + kRows * h;
     const int t = t0 + r;
     const bool valid = t < L;
     const int n_c = valid ? min(t / C, nlmk) : 0;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     uint64_t *slots = reinterpret_cast<uint64_t *>(smem + Lay::heap) + r;
-    float *stage = reinterpret_cast<float *>(smem + Lay::stage) + r;
+    uint64_t *mbox = reinterpret_cast<uint64_t *>(smem + Lay::mbox) + r;
     const float c2 = rs.scale * kLog2e;
     const float sc = rs.scale;
+    const float inv_sc = 1.0f / sc;
     const bool want_lse = lse_lmk != nullptr;
     float m2 = -INFINITY, l = 0.0f;
-    // rows with at most k candidates keep all of them (no search)
+    // rows with at most k candidates keep all of them (no search); with
+    // seeds, the first `cnt` seeds are the row's starting set (all of them
+    // are candidates of the row)
     const int cnt = n_c <= K ? n_c : K;
+    const bool search = n_c > K;
     TopK tk;
     tk.thr = INFINITY;
     tk.mn = ~0ull;
@@ -454,14 +616,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     bool ok = true;
     if (n_ltiles > 0) {
       // q row -> tensor memory (A operand of the scoring MMA): the row's
-      // 128-byte lines of the swizzled staging tile, two bf16 per column
+      // 128-byte lines of the swizzled staging tile, two bf16 per column;
+      // the owner also writes the masking operand [1, row < 64, 0, ...]
       ok = mbar_wait(&bars->q_smem, 0, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
-#pragma unroll
-        for (int kb = 0; kb < D / 64; ++kb) {
+        if (h < D / 64) {
           uint32_t w[32];
-          const unsigned char *line = smem + Lay::l0 + kb * kRows * 128 + r * 128;
+          const unsigned char *line = smem + Lay::l0 + h * kRows * 128 + r * 128;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const uint4 v4 = *reinterpret_cast<const uint4 *>(line + ((j ^ (r & 7)) << 4));
@@ -470,25 +632,32 @@ __global__ void __launch_bounds__(kThreads, 2)
             w[4 * j + 2] = v4.z;
             w[4 * j + 3] = v4.w;
           }
-          tmem_st32(q_tmem + lane_off + kb * 32, w);
+          tmem_st32(q_tmem + lane_off + h * 32, w);
+        }
+        if (h == 0) {
+          const __nv_bfloat162 p01 = __floats2bfloat162_rn(1.0f, r < kTile ? 1.0f : 0.0f);
+          uint32_t w8[8] = {*reinterpret_cast<const uint32_t *>(&p01), 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+          tmem_st8(bias_tmem + lane_off, w8);
         }
         tmem_wait_st();
       }
       tc_fence_before();
       mbar_arrive(&bars->q_tmem);
-      // stage the seed landmark rows (128-byte swizzled, as a TMA tile would
-      // be); rows past the seed count are zero
+      // stage the seed landmark rows into the last ring stage (128-byte
+      // swizzled, as a TMA tile would be) once every row has read its Q
+      // line out of it; rows past the seed count are zero
+      rows_sync();
       if (ok) {
         constexpr int kPieces = D / 8;  // 16-byte pieces per row
 #pragma unroll 1
-        for (int pc = r; pc < kTile * kPieces; pc += kRows) {
+        for (int pc = rt; pc < kTile * kPieces; pc += kRowThreads) {
           const int sr = pc / kPieces, col = pc % kPieces, kb = col >> 3, j = col & 7;
           uint4 v4 = make_uint4(0u, 0u, 0u, 0u);
           if (sr < ns)
             v4 = *reinterpret_cast<const uint4 *>(
                 reinterpret_cast<const unsigned char *>(lmk_raw) +
                 ((size_t)(lrow0 + seed_list[sr]) * D + kb * 64 + j * 8) * 2);
-          *reinterpret_cast<uint4 *>(smem + Lay::stage + kb * kTile * 128 + sr * 128 +
+          *reinterpret_cast<uint4 *>(seed_stage + kb * kTile * 128 + sr * 128 +
                                      ((j ^ (sr & 7)) << 4)) = v4;
         }
       }
@@ -497,119 +666,172 @@ __global__ void __launch_bounds__(kThreads, 2)
       ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->seed_full, 0, abort_flag));
       if (ok) {
         tc_fence_after();
-        float sa[2][32];
-        tmem_ld32(seed_tmem + lane_off, sa[0]);
-        tmem_ld32(seed_tmem + lane_off + 32, sa[1]);
+        float sa[32];
+        tmem_ld32(seed_tmem + lane_off + 32 * h, sa);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&bars->seed_read);
-        // the row's starting set: the first `cnt` seeds (all seeds when the
-        // row has more than k candidates)
+        // this thread's half of the starting set, and its log-sum-exp
 #pragma unroll
-        for (int j = 0; j < kMaxK; ++j)
-          if (j < cnt) slots[j * kRows] = sel_key(sa[j >> 5][j & 31] * sc, seed_list[j]);
-        if (n_c > K) tk.build(slots, K);
+        for (int j = 0; j < 32; ++j) {
+          const int jj = 32 * h + j;
+          if (jj < cnt) slots[jj * kRows] = sel_key(sa[j] * sc, seed_list[jj]);
+          sa[j] = jj < cnt ? sa[j] : -INFINITY;
+        }
+        if (want_lse) {
+          const float bm = block_max(sa);
+          if (bm > -INFINITY) lse_block(sa, bm, c2, m2, l);
+        }
       }
     }
-    const float inv_sc = 1.0f / sc;
-    float thr_u = prefilter(tk.thr, inv_sc);
-    int sp = 0;  // cursor into the ascending seed list
-    int next_seed = ns > 0 ? seed_list[0] : INT_MAX;
-    for (int i = 0; ok && i < n_ltiles; ++i) {
+    rows_sync();  // both halves of every row's starting set are in place
+    if (h == 0) {
+      if (ok && search) tk.build(slots, K);
+      st_volf(&thr_s[r], prefilter(tk.thr, inv_sc));
+    }
+    rows_sync();
+    float thr_u = thr_s[r];
+    uint32_t mb = 0;  // owner: keys drained; other half: keys posted
+    // owner: insert what the other half posted so far; returns the raw tail
+    auto drain = [&]() -> uint32_t {
+      const uint32_t tv = ld_vol(&tail_s[r]);
+      const uint32_t tl = tv & ~kDone;
+      while (mb != tl) {
+        __threadfence_block();
+        const uint64_t key = reinterpret_cast<volatile uint64_t *>(mbox)[(mb % kMbox) * kRows];
+        ++mb;
+        __threadfence_block();
+        st_vol(&head_s[r], mb);
+        if (key > tk.mn) {
+          tk.replace(slots, key, K);
+          thr_u = prefilter(tk.thr, inv_sc);
+          st_volf(&thr_s[r], thr_u);
+        }
+      }
+      return tv;
+    };
+    for (int i = 0; ok && i < n_scan; ++i) {
       const int sb = i % kSBufs;
-      ok = mbar_wait(&bars->s_full[sb], (i / kSBufs) & 1, abort_flag);
+      const uint32_t par = (i / kSBufs) & 1;
+      if (h == 0) {
+        // The owner keeps draining while it waits: the other half may be a
+        // tile behind, waiting for mailbox room, and the next score tile
+        // needs that half to release the one before.
+        bool got = mbar_try_wait(&bars->s_full[sb], par);
+        if (!got) {
+          const uint64_t w0 = globaltimer();
+          for (uint32_t it = 1;; ++it) {
+            drain();
+            if (mbar_try_wait(&bars->s_full[sb], par)) { got = true; break; }
+            if ((it & 63u) == 0) {
+              if (*abort_flag) break;
+              if (globaltimer() - w0 > kWaitLimitNs) { *abort_flag = 1; break; }
+            }
+          }
+        }
+        ok = got;
+      } else {
+        ok = mbar_wait(&bars->s_full[sb], par, abort_flag);
+      }
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-#pragma unroll 1
-      for (int blk = 0; blk < 2; ++blk) {
-        const int cb = i * kTile + blk * 32;
-        float a[32];
-        tmem_ld32((s_tmem0 + sb * kTile) + lane_off + blk * 32, a);
-        tmem_wait_ld();
-        if (blk == 1) {
-          tc_fence_before();
-          mbar_arrive(&bars->s_empty[sb]);
-        }
-        if (cb >= n_cand) break;
-        const int nv = max(0, min(32, n_c - cb));
-        if (cb + 32 > n_lo) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) a[j] = j < nv ? a[j] : -INFINITY;
-        }
-        // block maximum: a tree of three-input maxima (32 -> 11 -> 4 -> 1)
-        float y[11];
-#pragma unroll
-        for (int j = 0; j < 10; ++j) y[j] = max3f(a[3 * j], a[3 * j + 1], a[3 * j + 2]);
-        y[10] = fmaxf(a[30], a[31]);
-        const float bm = max3f(max3f(y[0], y[1], y[2]), max3f(y[3], y[4], y[5]),
-                               max3f(y[6], y[7], max3f(y[8], y[9], y[10])));
-        if (want_lse && nv > 0) {
-          const float bm2 = bm * c2;
-          if (bm2 > m2) {
-            l *= ex2_approx(m2 - bm2);
-            m2 = bm2;
-          }
-          // pairs of candidates through packed f32x2 FMA and add
-          const float2 c2v = make_float2(c2, c2), nm2 = make_float2(-m2, -m2);
-          float2 ps[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float2 y = __ffma2_rn(make_float2(a[2 * j], a[2 * j + 1]), c2v, nm2);
-            ps[j & 1] = __fadd2_rn(ps[j & 1], make_float2(ex2_approx(y.x), ex2_approx(y.y)));
-          }
-          l += (ps[0].x + ps[1].x) + (ps[0].y + ps[1].y);
-        }
-        // candidates that may enter the top-k; seeds are already kept
-        const bool pass = bm >= thr_u;
-        if (!__any_sync(0xffffffffu, pass)) continue;
-        uint32_t mask = 0;
-        if (pass) {
-          uint32_t mq[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-          for (int j = 0; j < 32; ++j) mq[j >> 3] |= a[j] >= thr_u ? (1u << j) : 0u;
-          mask = (mq[0] | mq[1]) | (mq[2] | mq[3]);
-        }
-        // the seeds in this block, the same for every row: all lanes walk the
-        // ascending seed list together (seeds of skipped blocks are passed over)
-        while (next_seed < cb + 32) {
-          if (next_seed >= cb) mask &= ~(1u << (next_seed - cb));
-          ++sp;
-          next_seed = sp < ns ? seed_list[sp] : INT_MAX;
-        }
-        if (!__any_sync(0xffffffffu, mask != 0)) continue;
+      float a[32];
+      tmem_ld32(s_tmem0 + sb * kTile + lane_off + 32 * h, a);
+      if (h == 0)
+        drain();  // the other half's candidates since the last tile
+      else
+        thr_u = ld_volf(&thr_s[r]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars->s_empty[sb]);
+      const int cb = i * kTile + 32 * h;
+      const float bm = block_max(a);
+      if (want_lse) lse_block(a, bm, c2, m2, l);
+      // candidates that may enter the top-k (seeds and masked columns sit at -1e30)
+      const bool pass = bm >= thr_u;
+      if (!__any_sync(0xffffffffu, pass)) continue;
+      uint32_t mask = pass ? ge_mask(a, thr_u) : 0u;
+      const bool single = __popc(mask) == 1;  // then it is the block maximum
+      // one candidate per lane per iteration: the lanes insert together
+      while (__any_sync(0xffffffffu, mask != 0)) {
         if (mask) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) stage[j * kRows] = a[j];
-        }
-        // one candidate per lane per iteration: the lanes insert together
-        while (__any_sync(0xffffffffu, mask != 0)) {
-          if (mask) {
-            const int j = __ffs(mask) - 1;
-            mask &= mask - 1;
-            const uint64_t key = sel_key(stage[j * kRows] * sc, cb + j);
+          const int j = __ffs(mask) - 1;
+          mask &= mask - 1;
+          const float v = single ? bm : pick32(a, j);
+          const uint64_t key = sel_key(v * sc, cb + j);
+          if (h == 0) {
             if (key > tk.mn) {
               tk.replace(slots, key, K);
               thr_u = prefilter(tk.thr, inv_sc);
+              st_volf(&thr_s[r], thr_u);
+            }
+          } else {
+            // wait (bounded) for a free mailbox entry, then post
+            bool room = mb - ld_vol(&head_s[r]) < (uint32_t)kMbox;
+            if (!room) {
+              const uint64_t w0 = globaltimer();
+              while (!room) {
+                if (*abort_flag || globaltimer() - w0 > kWaitLimitNs) break;
+                room = mb - ld_vol(&head_s[r]) < (uint32_t)kMbox;
+              }
+            }
+            if (!room) {
+              *abort_flag = 1;
+              ok = false;
+              mask = 0;
+            } else {
+              __threadfence_block();
+              reinterpret_cast<volatile uint64_t *>(mbox)[(mb % kMbox) * kRows] = key;
+              ++mb;
+              __threadfence_block();
+              st_vol(&tail_s[r], mb);
             }
           }
         }
       }
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
     }
-    // ---------------------------------------------------------- epilogue
-    if (__all_sync(0xffffffffu, ok) && valid) {
-      const size_t row = (size_t)bh * L + t;
-      int32_t *srow = sel + row * K;
-      float *wrow = chunk_w + row * K;
-      // ascending chunk order (rows that kept every candidate are in order)
-      if (n_c <= K)
-        write_in_order(slots, cnt, K, srow, wrow);
-      else if (K <= 16)
-        write_sorted<16>(slots, K, srow, wrow);
-      else if (K <= 32)
-        write_sorted<32>(slots, K, srow, wrow);
-      else
-        write_sorted<64>(slots, K, srow, wrow);
-      if (want_lse) lse_lmk[row] = n_c > 0 ? (m2 + __log2f(l)) * kLn2 : -INFINITY;
+    if (h == 1) {
+      // hand over this half's log-sum-exp and close the mailbox
+      lsep_s[r] = make_float2(m2, l);
+      __threadfence_block();
+      st_vol(&tail_s[r], mb | kDone);
+    } else {
+      // drain what the other half still posts until it closes the mailbox
+      const uint64_t w0 = globaltimer();
+      bool closed = false;
+      for (uint32_t it = 0;; ++it) {
+        const uint32_t tv = drain();
+        if ((tv & kDone) && mb == (tv & ~kDone)) { closed = true; break; }
+        if ((it & 63u) == 63u && (globaltimer() - w0 > kWaitLimitNs)) break;
+      }
+      if (!closed) {
+        *abort_flag = 1;
+        ok = false;
+      }
+      __threadfence_block();
+      // ---------------------------------------------------------- epilogue
+      if (__all_sync(0xffffffffu, ok) && valid) {
+        const size_t row = (size_t)bh * L + t;
+        int32_t *srow = sel + row * K;
+        float *wrow = chunk_w + row * K;
+        // ascending chunk order (rows that kept every candidate are in order)
+        if (n_c <= K)
+          write_in_order(slots, cnt, K, srow, wrow);
+        else if (K <= 16)
+          write_sorted<16>(slots, K, srow, wrow);
+        else if (K <= 32)
+          write_sorted<32>(slots, K, srow, wrow);
+        else
+          write_sorted<64>(slots, K, srow, wrow);
+        if (want_lse) {
+          const float2 o = lsep_s[r];
+          const float mm = fmaxf(m2, o.x);
+          const float ls = (m2 > -INFINITY ? l * ex2_approx(m2 - mm) : 0.0f) +
+                           (o.x > -INFINITY ? o.y * ex2_approx(o.x - mm) : 0.0f);
+          lse_lmk[row] = n_c > 0 ? (mm + __log2f(ls)) * kLn2 : -INFINITY;
+        }
+      }
     }
   }
   tc_fence_before();

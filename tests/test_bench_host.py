@@ -52,8 +52,10 @@ def test_select_executed_flop_counts_mma_tiles():
     for t0 in range(0, w.L, 128):
         t_last = min(t0 + 127, w.L - 1)
         n = min(t_last // w.C, w.L // w.C)
-        tiles = -(-n // 64) + (1 if n > 0 else 0)
-        want += tiles * 2 * 128 * 64 * w.d
+        if n > 0:
+            want += 2 * 128 * 64 * w.d                          # seed tile
+        if n > w.topk:
+            want += -(-n // 64) * 2 * 128 * 64 * (w.d + 16)     # scan with the masking step
     assert bench.select_executed_flop(w) == want * w.B * w.Hq
 
 

@@ -21,8 +21,9 @@ def problem(w):
 
 
 def gpu_prefill(dq, dk, dv, dl, w, with_wfin=False):
-    sel, cw, lse_lmk = hb.select(dq, dl, w.topk, w.M)
-    out, lse, wf = hb.attn_fwd(dq, dk, dv, sel, cw, w.M, with_w_final=with_wfin)
+    # debug mode: a device-side check or a bounded wait that gave up raises
+    sel, cw, lse_lmk = hb.select(dq, dl, w.topk, w.M, debug_checks=True)
+    out, lse, wf = hb.attn_fwd(dq, dk, dv, sel, cw, w.M, with_w_final=with_wfin, debug_checks=True)
     torch.cuda.synchronize()
     return dict(sel=sel, w=cw, lse_lmk=lse_lmk, out=out, lse=lse, wfin=wf)
 
