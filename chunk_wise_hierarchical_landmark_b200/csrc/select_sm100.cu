@@ -741,6 +741,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         drain();  // the other half's candidates since the last tile
       else
         thr_u = ld_volf(&thr_s[r]);
+      __syncwarp();  // tcgen05.wait is warp-collective
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&bars->s_empty[sb]);

@@ -244,15 +244,41 @@ def _widen32(x) -> np.ndarray:
     return np.ascontiguousarray(a, dtype=np.float32)
 
 
+def _bf16_round(x: np.ndarray) -> np.ndarray:
+    """fp32 values rounded to the nearest bf16 (ties to even), as fp32."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
+    return (r.astype(np.uint32) << 16).view(np.float32)
+
+
 def qcal_query(q, h, w_down, w_up) -> np.ndarray:
     """Q-Cal scoring query: q_t + W_up[hq] (W_down h_t) for every head and
-    position, formed in fp64 and rounded once to fp32.
-    q [B,Hq,L,d] (fp32 / bf16), h [B,L,D] hidden states, w_down [r,D] (shared
-    by the heads), w_up [Hq,d,r]."""
-    qa = _widen32(q).astype(np.float64)
-    z = np.einsum("rD,bLD->bLr", np.asarray(w_down, np.float64), np.asarray(h, np.float64))
-    dq = np.einsum("hdr,bLr->bhLd", np.asarray(w_up, np.float64), z)
-    return (qa + dq).astype(np.float32)
+    position (molayo1419.me, "Engineering details", Q-Cal: a low-rank learnable
+    offset of the query used for the chunk-mass estimate).
+
+    q [B,Hq,L,d], h [B,L,D] hidden states, w_down [r,D] (shared by the heads),
+    w_up [Hq,d,r]; each fp32 or bf16 (widened exactly), fp64 data is first
+    rounded to fp32.  The pages fix no precision; the reading taken here is
+    the query's own: everything in fp32, every product and every partial sum
+    rounded (no fused multiply-add), in a fixed order --
+      z_r  = sum over i = 0 .. D-1 of w_down[r, i] * h_t[i]
+      dq_e = sum over j = 0 .. r-1 of w_up[hq, e, j] * z_j
+      q_cal = q + dq, rounded to bf16 (nearest even) when q is bf16
+    -- so that a scoring pass fed this query sees exactly these values.
+    Returns fp32 [B,Hq,L,d] (bf16 values widened exactly)."""
+    qa, q_bf16 = _as_array(q)
+    q32 = _widen32(q)
+    h32, wd32, wu32 = (_widen32(a) for a in (h, w_down, w_up))
+    B, Hq, L, d = q32.shape
+    r, D = wd32.shape
+    z = np.zeros((B, L, r), np.float32)
+    for i in range(D):
+        z = (z + (h32[:, :, None, i] * wd32[None, None, :, i]).astype(np.float32)).astype(np.float32)
+    dq = np.zeros((B, Hq, L, d), np.float32)
+    for j in range(r):
+        dq = (dq + (wu32[None, :, None, :, j] * z[:, None, :, j, None]).astype(np.float32)).astype(np.float32)
+    qc = (q32 + dq).astype(np.float32)
+    return _bf16_round(qc) if q_bf16 else qc
 
 
 def gather_pages(pages, page_table, L: int) -> np.ndarray:

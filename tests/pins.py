@@ -479,9 +479,28 @@ def pin_qcal_scoring_query(orc):
     landmark makes k = 1 pick that chunk on every row that can."""
     from oracle import qcal_query
     # hand value: D = 2, r = 1, d = 2, h_t = (1, 1): z = 1 + 2 = 3, dq = (3*3, 4*3)
-    qs = qcal_query(np.zeros((1, 1, 1, 2), np.float32), np.ones((1, 1, 2)), [[1.0, 2.0]],
-                    [[[3.0], [4.0]]])
+    qs = qcal_query(np.zeros((1, 1, 1, 2), np.float32), np.ones((1, 1, 2)),
+                    np.array([[1.0, 2.0]]), np.array([[[3.0], [4.0]]]))
     assert np.array_equal(qs.reshape(-1), np.array([9.0, 12.0], np.float32))
+    # the fixed fp32 order: 1 + 2^-24 + 2^-24 is 1 summed left to right (each
+    # partial sum rounds back to 1), but 1 + 2^-23 summed the other way round
+    one = np.float32(1.0)
+    eps = np.float32(2.0 ** -24)
+    qs = qcal_query(np.zeros((1, 1, 1, 1), np.float32), np.array([[[1.0, 1.0, 1.0]]]),
+                    np.array([[one, eps, eps]]), np.array([[[1.0]]]))
+    assert qs.reshape(-1)[0] == one
+    qs = qcal_query(np.zeros((1, 1, 1, 1), np.float32), np.array([[[1.0, 1.0, 1.0]]]),
+                    np.array([[eps, eps, one]]), np.array([[[1.0]]]))
+    assert qs.reshape(-1)[0] == np.float32(1.0 + 2.0 ** -23)
+    # a bf16 query gets a bf16 scoring query (spacing 2^-7 above 1): 1 + 2^-9
+    # is below the halfway point 1 + 2^-8 and rounds to 1, 1 + 3*2^-9 rounds up
+    import torch
+    qb = torch.zeros((1, 1, 2, 1), dtype=torch.bfloat16) + 1.0
+    qs = qcal_query(qb, np.ones((1, 2, 1)), np.array([[1.0]]),
+                    np.array([[[2.0 ** -9]]]))
+    assert np.array_equal(qs.reshape(-1), np.array([1.0, 1.0], np.float32))
+    qs = qcal_query(qb, np.ones((1, 2, 1)), np.array([[3.0]]), np.array([[[2.0 ** -9]]]))
+    assert np.array_equal(qs.reshape(-1), np.array([1.0 + 2.0 ** -7] * 2, np.float32))
     rng = _rng(43)
     B, Hq, Hkv, L, d, C, D, r = 1, 4, 2, 45, 8, 4, 12, 3
     q = _f32(B, Hq, L, d, rng=rng)
