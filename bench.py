@@ -483,6 +483,54 @@ def tile_union_sizes(hb, sel):
     return (u_off[1:] - u_off[:-1]).cpu().numpy()
 
 
+def bench_qcal(hb, synth, w, steps, warmup, r=32):
+    """The Q-Cal prefill of workload w: the calibrated scoring query
+    (hils_qcal_query: z = W_down h per position, q + W_up z per head) timed
+    alone and as part of hils_prefill_qcal.  h [B, L, Hq*d] and the weights
+    are seeded random data of the model's shapes (no trained weights)."""
+    dev = torch.device("cuda")
+    q, k, v, lmk = synth.make_inputs(w, "cuda", seed=w.seed)
+    D = w.Hq * w.d
+    g = torch.Generator(device=dev).manual_seed(w.seed + 31)
+    h = torch.randn((w.B, w.L, D), generator=g, device=dev).to(q.dtype)
+    wd = (torch.randn((r, D), generator=g, device=dev) / D ** 0.5).to(q.dtype)
+    # a calibration: the offset is about a tenth of the query (|z| ~ 1 per rank)
+    wu = (torch.randn((w.Hq, w.d, r), generator=g, device=dev) * (0.1 / r ** 0.5)).to(q.dtype)
+    p = hb.make_params(w.B, w.Hq, w.Hkv, w.L, w.d, w.topk, w.M, w.C, w.scale, q.dtype, False)
+    B, Hq, L, K = w.B, w.Hq, w.L, w.topk
+    sel = torch.empty((B, Hq, L, K), dtype=torch.int32, device=dev)
+    cw = torch.empty((B, Hq, L, K), dtype=torch.float32, device=dev)
+    lse_lmk = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+    q_cal = torch.empty_like(q)
+    ws = hb.qcal_workspace(p, r, dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    ms_q = timed(lambda: hb.hils_qcal_query(p, q, h, wd, wu, q_cal, ws, stream))
+    ms_all = timed(lambda: hb.hils_prefill_qcal(p, q, k, v, lmk, h, wd, wu, q_cal, sel, cw,
+                                                lse_lmk, out, lse, ws, stream))
+    esz = q.element_size()
+    nbytes = float(w.B * L * D * esz + 2 * q.numel() * esz + r * D * esz + Hq * w.d * r * esz)
+    return {"value": B * L / (ms_all * 1e-3), "unit": "query-tokens/s", "ms_per_step": ms_all,
+            "qcal_query_ms": ms_q, "rank": r, "hidden": D,
+            "qcal_query_bytes": nbytes, "qcal_query_gbs": nbytes / (ms_q * 1e-3) / 1e9,
+            "inputs": "seeded random h and weights of the model's shapes; offset about 0.1 x the query"}
+
+
 def union_stats(hb, sel, w):
     """Chunk-union size per group of M rows and adjacent-query overlap."""
     u_off, _ = hb.union(sel, M=w.M)
@@ -658,6 +706,12 @@ def run_ours(args):
             "pool": f"{r3['paged_pages']} pages of 64 tokens x {w3.Hkv} KV heads, random order",
             "equal_to_dense": r3["paged_equal"]}
         del r3
+        torch.cuda.empty_cache()
+        try:
+            extra["qcal_" + W.PREFILL_128K.name] = bench_qcal(hb, synth, W.PREFILL_128K,
+                                                              max(3, args.steps), 2)
+        except Exception as e:  # an extra entry must not cost the main line
+            extra["qcal_" + W.PREFILL_128K.name] = {"error": str(e)[:200]}
         torch.cuda.empty_cache()
         try:
             r4 = bench_hope(hb, w, max(5, args.steps), 3)

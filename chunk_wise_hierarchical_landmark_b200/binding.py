@@ -9,7 +9,6 @@ libhils.so is missing or fails to load, every call raises.
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 
 import torch
@@ -39,7 +38,8 @@ class Params(ctypes.Structure):
 _lib = None
 EXPORTS = ["hils_workspace_size", "hils_select", "hils_union_capacity", "hils_union",
            "hils_attn_fwd", "hils_prefill", "hils_decode_fwd", "hils_decode_fwd_paged",
-           "hils_decode_fwd_noalloc", "hils_hope",
+           "hils_decode_fwd_noalloc", "hils_hope", "hils_qcal_workspace_size", "hils_qcal_query",
+           "hils_prefill_qcal", "hils_hope_rope_pairs", "hils_test_set_wait_limit",
            "hils_status_string", "hils_last_error", "hils_launch_count"]
 
 
@@ -64,8 +64,17 @@ def lib():
         L.hils_decode_fwd_paged.argtypes = [PP, P, P, P, I64, P, I, P, P, P, P, P, P, P, SZ, P]
         L.hils_decode_fwd_noalloc.argtypes = [PP, P, P, P, P, P, P, P, P, P, P]
         L.hils_hope.argtypes = [P, I, I, I, I, I, I, I, ctypes.c_double, P]
+        L.hils_test_set_wait_limit.argtypes = [ctypes.c_uint64, I]
+        L.hils_test_set_wait_limit.restype = None
+        L.hils_hope_rope_pairs.argtypes = [I, ctypes.c_double, ctypes.c_double]
+        L.hils_hope_rope_pairs.restype = I
+        L.hils_qcal_workspace_size.argtypes = [PP, I]
+        L.hils_qcal_workspace_size.restype = SZ
+        L.hils_qcal_query.argtypes = [PP, P, P, P, P, I, I, P, P, SZ, P]
+        L.hils_prefill_qcal.argtypes = [PP, P, P, P, P, P, P, P, I, I, P, P, P, P, P, P, P, SZ, P]
         for f in ("hils_select", "hils_union", "hils_attn_fwd", "hils_prefill", "hils_decode_fwd",
-                  "hils_decode_fwd_paged", "hils_decode_fwd_noalloc", "hils_hope"):
+                  "hils_decode_fwd_paged", "hils_decode_fwd_noalloc", "hils_hope",
+                  "hils_qcal_query", "hils_prefill_qcal"):
             getattr(L, f).restype = I
         L.hils_status_string.argtypes = [I]
         L.hils_status_string.restype = ctypes.c_char_p
@@ -183,13 +192,52 @@ def hils_hope(x, n_rope_pairs: int, pos0: int = 0, base: float = 10000.0, stream
                            _stream(stream)))
 
 
+def qcal_workspace(p: Params, r: int, device=None) -> torch.Tensor:
+    n = lib().hils_qcal_workspace_size(ctypes.byref(p), int(r))
+    if n == 0:
+        raise HilsError(1, "hils_qcal_workspace_size rejected the parameters")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def hils_qcal_query(p: Params, q, h, w_down, w_up, q_cal, ws, stream=None):
+    r, D = w_down.shape
+    _check(lib().hils_qcal_query(ctypes.byref(p), _ptr(q), _ptr(h), _ptr(w_down), _ptr(w_up),
+                                 int(D), int(r), _ptr(q_cal), *_ws_args(ws), _stream(stream)))
+
+
+def hils_prefill_qcal(p: Params, q, k, v, lmk_k, h, w_down, w_up, q_cal, sel_idx, chunk_w,
+                      lse_lmk, out, lse, ws, stream=None):
+    r, D = w_down.shape
+    _check(lib().hils_prefill_qcal(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(lmk_k),
+                                   _ptr(h), _ptr(w_down), _ptr(w_up), int(D), int(r), _ptr(q_cal),
+                                   _ptr(sel_idx), _ptr(chunk_w), _ptr(lse_lmk), _ptr(out),
+                                   _ptr(lse), *_ws_args(ws), _stream(stream)))
+
+
+def prefill_qcal(q, k, v, lmk_k, h, w_down, w_up, topk, M=64, scale=None, debug_checks=False):
+    """Prefill with the Q-Cal scoring query (h [B,L,D], w_down [r,D], w_up
+    [Hq,d,r]): returns dict(out, lse, sel_idx, chunk_w, lse_lmk, q_cal)."""
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    p = make_params(B, Hq, Hkv, L, d, topk, M, 64, scale, q.dtype, debug_checks)
+    dev = q.device
+    sel = torch.empty((B, Hq, L, topk), dtype=torch.int32, device=dev)
+    w = torch.empty((B, Hq, L, topk), dtype=torch.float32, device=dev)
+    lse_lmk = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+    q_cal = torch.empty_like(q)
+    ws = qcal_workspace(p, w_down.shape[0], dev)
+    hils_prefill_qcal(p, q, k, v, lmk_k, h, w_down, w_up, q_cal, sel, w, lse_lmk, out, lse, ws)
+    return dict(out=out, lse=lse, sel_idx=sel, chunk_w=w, lse_lmk=lse_lmk, q_cal=q_cal)
+
+
 def rope_pairs_for(d: int, base: float, train_len: int) -> int:
-    """One split rule for HoPE: the pairs whose wavelength 2*pi*base^(2i/d)
-    fits in the pre-training length get RoPE (they are the first ones, as the
-    wavelength grows with i)."""
-    n = 0
-    while n < d // 2 and 2.0 * math.pi * base ** (2.0 * n / d) <= train_len:
-        n += 1
+    """The HoPE split of the library (hils_hope_rope_pairs): the pairs whose
+    wavelength fits in the pre-training length get RoPE."""
+    n = lib().hils_hope_rope_pairs(int(d), float(base), float(train_len))
+    if n < 0:
+        raise HilsError(1, "hils_hope_rope_pairs rejected its arguments")
     return n
 
 

@@ -147,6 +147,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
   const int b = bh / rs.Hq, hq = bh % rs.Hq, hkv = hq / (rs.Hq / rs.Hkv);
+  const uint64_t lim = rs.wait_ns;
   const int t0 = blockIdx.x * kRows;
   const int L = rs.L, K = rs.topk;
   const int nchunks = (L + kChunk - 1) / kChunk;
@@ -301,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       auto load_k = [&](int j) -> bool {
         const int c = itk.next();
         const int s = j % kStages;
-        if (j >= kStages && !mbar_wait(&bars->k_empty[s], ((j / kStages) - 1) & 1, abort_flag))
+        if (j >= kStages && !mbar_wait(&bars->k_empty[s], ((j / kStages) - 1) & 1, abort_flag, lim))
           return false;
         mbar_expect_tx(&bars->k_full[s], Lay::kKVBytes);
         unsigned char *ks = smem + Lay::k0 + s * Lay::kKVBytes;
@@ -313,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       auto load_v = [&](int j) -> bool {
         const int c = itv.next();
         const int s = j % kStages;
-        if (j >= kStages && !mbar_wait(&bars->v_empty[s], ((j / kStages) - 1) & 1, abort_flag))
+        if (j >= kStages && !mbar_wait(&bars->v_empty[s], ((j / kStages) - 1) & 1, abort_flag, lim))
           return false;
         mbar_expect_tx(&bars->v_full[s], Lay::kKVBytes);
         unsigned char *vs = smem + Lay::v0 + s * Lay::kKVBytes;
@@ -329,10 +330,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       // every load issued must land before the CTA may exit
       for (int i = (k_issued > kStages ? k_issued - kStages : 0); i < k_issued; ++i)
-        mbar_wait_bounded(&bars->k_full[i % kStages], (i / kStages) & 1);
+        mbar_wait_bounded(&bars->k_full[i % kStages], (i / kStages) & 1, lim);
       for (int i = (v_issued > kStages ? v_issued - kStages : 0); i < v_issued; ++i)
-        mbar_wait_bounded(&bars->v_full[i % kStages], (i / kStages) & 1);
-      mbar_wait_bounded(&bars->q, 0);
+        mbar_wait_bounded(&bars->v_full[i % kStages], (i / kStages) & 1, lim);
+      mbar_wait_bounded(&bars->q, 0, lim);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -344,8 +345,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       // has read P_{j-2} from that buffer
       auto qk = [&](int j) -> bool {
         const int s = j % kStages, b2 = j & 1;
-        if (!mbar_wait(&bars->k_full[s], (j / kStages) & 1, abort_flag)) return false;
-        if (j >= 2 && !mbar_wait(&bars->p_free[b2], ((j >> 1) - 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(&bars->k_full[s], (j / kStages) & 1, abort_flag, lim)) return false;
+        if (j >= 2 && !mbar_wait(&bars->p_free[b2], ((j >> 1) - 1) & 1, abort_flag, lim)) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(smem + Lay::k0 + s * Lay::kKVBytes);
 #pragma unroll
@@ -362,8 +363,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       // O += P_j V_j, P_j read from the first 32 columns of S buffer j & 1
       auto pv = [&](int j) -> bool {
         const int s = j % kStages, b2 = j & 1;
-        if (!mbar_wait(&bars->v_full[s], (j / kStages) & 1, abort_flag)) return false;
-        if (!mbar_wait(&bars->p_full[b2], (j >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(&bars->v_full[s], (j / kStages) & 1, abort_flag, lim)) return false;
+        if (!mbar_wait(&bars->p_full[b2], (j >> 1) & 1, abort_flag, lim)) return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(smem + Lay::v0 + s * Lay::kKVBytes);
 #pragma unroll
@@ -378,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         mma_commit(&bars->p_free[b2]);
         return true;
       };
-      bool ok = mbar_wait(&bars->q, 0, abort_flag);
+      bool ok = mbar_wait(&bars->q, 0, abort_flag, lim);
       if (ok) ok = qk(0);
       if (ok && n_steps > 1) ok = qk(1);
       for (int j = 0; ok && j < n_steps; ++j) {
@@ -388,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (ok) mma_commit(&bars->o_full);
       // all issued tensor-core work must finish before TMEM is released
       mma_commit(&bars->done);
-      mbar_wait_bounded(&bars->done, 0);
+      mbar_wait_bounded(&bars->done, 0, lim);
     }
   } else {
     // ------------------------------------------------------------ softmax rows
@@ -414,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int i = 0; i < n_steps; ++i) {
       const int c = it.next();
       const uint32_t sb = s_tmem + 64 * (i & 1) + lane_off;
-      ok = mbar_wait(&bars->s_full[i & 1], (i >> 1) & 1, abort_flag);
+      ok = mbar_wait(&bars->s_full[i & 1], (i >> 1) & 1, abort_flag, lim);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       float x[64];
@@ -507,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_arrive(&bars->p_full[i & 1]);
     }
     // ---------------------------------------------------------- epilogue
-    if (ok) ok = mbar_wait(&bars->o_full, 0, abort_flag);
+    if (ok) ok = mbar_wait(&bars->o_full, 0, abort_flag, lim);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const float lsum = ex2_approx(lse2_own - M2) + sumsel * ex2_approx(wmax2 - M2);

@@ -11,6 +11,7 @@
 #include "kernels.h"
 #include "hope.h"
 #include "paged.h"
+#include "qcal.h"
 
 #define HILS_API extern "C" __attribute__((visibility("default")))
 
@@ -72,8 +73,16 @@ hils_status check_params(const hils_params *p) {
     if ((ptr) && !aligned16(ptr)) return fail(HILS_ERR_INVALID_ARG, #ptr " is not 16-byte aligned"); \
   } while (0)
 
+// Failure-path test settings (hils_test_set_wait_limit); 0 = the default limit.
+std::atomic<unsigned long long> g_test_wait_ns{0};
+std::atomic<int> g_test_withhold{0};
+
 hils::RowSpec prefill_rows(const hils_params *p) {
-  return hils::RowSpec{p->B, p->Hq, p->Hkv, p->L, p->d, p->chunk, p->topk, p->scale, 0, p->L};
+  hils::RowSpec rs{p->B, p->Hq, p->Hkv, p->L, p->d, p->chunk, p->topk, p->scale, 0, p->L};
+  const unsigned long long ns = g_test_wait_ns.load();
+  if (ns) rs.wait_ns = ns;
+  rs.withhold = g_test_withhold.load();
+  return rs;
 }
 
 // Debug mode: clear the device error word before the launches ...
@@ -303,6 +312,53 @@ HILS_API hils_status hils_decode_fwd_paged(const hils_params *p, const void *q,
                      sel_idx, chunk_w, lse_lmk, out, lse, ws, ws_bytes, stream);
 }
 
+HILS_API size_t hils_qcal_workspace_size(const hils_params *p, int r) {
+  if (check_params(p) != HILS_OK || r < 1 || r > hils::kMaxQcalRank) return 0;
+  return kDebugWs + (((size_t)p->B * p->L * r * sizeof(float) + 255) & ~size_t(255));
+}
+
+HILS_API hils_status hils_qcal_query(const hils_params *p, const void *q, const void *h,
+                                     const void *w_down, const void *w_up, int D, int r,
+                                     void *q_cal, void *ws, size_t ws_bytes, void *stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  NEED(q);
+  NEED(h);
+  NEED(w_down);
+  NEED(w_up);
+  NEED(q_cal);
+  if (D < 1) return fail(HILS_ERR_INVALID_ARG, "D=%d must be >= 1", D);
+  if (r < 1 || r > hils::kMaxQcalRank)
+    return fail(HILS_ERR_UNSUPPORTED, "r=%d (supported: 1..%d)", r, hils::kMaxQcalRank);
+  if ((int64_t)p->B * p->L * D >= (int64_t)1 << 40)
+    return fail(HILS_ERR_UNSUPPORTED, "B*L*D too large");
+  const size_t need = hils_qcal_workspace_size(p, r);
+  if (!ws || ws_bytes < need)
+    return fail(HILS_ERR_WORKSPACE, "Q-Cal needs %zu bytes of workspace, got %zu", need, ws_bytes);
+  NEED(ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float *z = reinterpret_cast<float *>(static_cast<unsigned char *>(ws) + kDebugWs);
+  int n = 0;
+  cudaError_t e = hils::qcal_query(p->dtype == HILS_BF16, p->B, p->Hq, p->L, p->d, D, r, q, h,
+                                   w_down, w_up, q_cal, z, st, &n);
+  g_launches += n;
+  if (e != cudaSuccess) return cuda_fail(e, "Q-Cal launch");
+  return HILS_OK;
+}
+
+HILS_API hils_status hils_prefill_qcal(const hils_params *p, const void *q, const void *k,
+                                       const void *v, const void *lmk_k, const void *h,
+                                       const void *w_down, const void *w_up, int D, int r,
+                                       void *q_cal, int32_t *sel_idx, float *chunk_w,
+                                       float *lse_lmk, void *out, float *lse, void *ws,
+                                       size_t ws_bytes, void *stream) {
+  hils_status s = hils_qcal_query(p, q, h, w_down, w_up, D, r, q_cal, ws, ws_bytes, stream);
+  if (s != HILS_OK) return s;
+  s = hils_select(p, q_cal, lmk_k, sel_idx, chunk_w, lse_lmk, ws, ws_bytes, stream);
+  if (s != HILS_OK) return s;
+  return hils_attn_fwd(p, q, k, v, sel_idx, chunk_w, out, lse, nullptr, ws, ws_bytes, stream);
+}
+
 HILS_API hils_status hils_hope(void *x, int dtype, int B, int H, int L, int d, int pos0,
                                int n_rope_pairs, double base, void *stream) {
   NEED(x);
@@ -321,6 +377,21 @@ HILS_API hils_status hils_hope(void *x, int dtype, int B, int H, int L, int d, i
   g_launches += n;
   if (e != cudaSuccess) return cuda_fail(e, "hope launch");
   return HILS_OK;
+}
+
+HILS_API void hils_test_set_wait_limit(uint64_t ns, int withhold) {
+  g_test_wait_ns.store(ns);
+  g_test_withhold.store(withhold ? 1 : 0);
+}
+
+HILS_API int hils_hope_rope_pairs(int d, double base, double train_len) {
+  // pairs i (rotate-half) whose wavelength 2 pi base^(2i/d) fits the window;
+  // the wavelength grows with i, so they are the first ones
+  if (d < 2 || !(base > 1.0) || !std::isfinite(base) || std::isnan(train_len)) return -1;
+  const double two_pi = 6.283185307179586;
+  int n = 0;
+  while (n < d / 2 && two_pi * std::pow(base, 2.0 * n / d) <= train_len) ++n;
+  return n;
 }
 
 HILS_API const char *hils_status_string(hils_status s) {

@@ -15,6 +15,10 @@ struct RowSpec {
   int B, Hq, Hkv, L, d, C, topk;
   float scale;
   int t_first, t_count;
+  // bounded device waits give up after wait_ns; withhold = 1 (tests of the
+  // failure path only) keeps back one producer arrival of the scoring kernel
+  unsigned long long wait_ns = 2000000000ull;
+  int withhold = 0;
 };
 
 // SIMT kernels (hils_simt.cu)

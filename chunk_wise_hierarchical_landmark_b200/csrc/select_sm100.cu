@@ -379,6 +379,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
   const int b = bh / rs.Hq, hq = bh % rs.Hq, hkv = hq / (rs.Hq / rs.Hkv);
+  const uint64_t lim = rs.wait_ns;
   // this launch's level: tiles offset + i * period, heaviest first
   const int ntiles_rows = (rs.L + kRows - 1) / kRows;
   const int tile = level_offset(level) +
@@ -476,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           tma_load_2d(smem + Lay::l0 + kb * kRows * 128, &tm_q, &bars->q_smem, kb * 64, bh * L + t0);
       }
       // the ring holds the Q tile until the row threads have moved it to TMEM
-      bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->q_tmem, 0, abort_flag));
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->q_tmem, 0, abort_flag, lim));
       const __nv_bfloat16 negb = __float2bfloat16_rn(-1.0e30f);
       const uint32_t neg = (uint32_t)__bfloat16_as_ushort(negb);
       int issued = 0;
@@ -484,9 +485,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int i = 0; ok && i < n_scan; ++i) {
         const int s = i % kStages;
         bool w = true;
-        if (i >= kStages) w = mbar_wait(&bars->l_empty[s], ((i / kStages) - 1) & 1, abort_flag);
+        if (i >= kStages) w = mbar_wait(&bars->l_empty[s], ((i / kStages) - 1) & 1, abort_flag, lim);
         // the seed tile sits in the last ring stage until the seed MMA is done
-        if (w && i == kStages - 1) w = mbar_wait(&bars->seed_done, 0, abort_flag);
+        if (w && i == kStages - 1) w = mbar_wait(&bars->seed_done, 0, abort_flag, lim);
         if (!__all_sync(0xffffffffu, w)) break;
         // the landmark tile first (arrival 1 of 2, with its bytes) ...
         if (lane == 0) {
@@ -533,22 +534,24 @@ __global__ void __launch_bounds__(kThreads, 2)
         __syncwarp();
         if (lane == 0) {
           bias_flag[s] = need ? 1 : 0;
-          mbar_arrive(&bars->l_full[s]);  // arrival 2 of 2
+          // arrival 2 of 2 (a failure-path test keeps back tile 0's: the MMA
+          // issuer's bounded wait then runs out and every role unwinds)
+          if (!(rs.withhold && i == 0)) mbar_arrive(&bars->l_full[s]);
         }
       }
       if (lane == 0) {
         for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-          mbar_wait_bounded(&bars->l_full[i % kStages], (i / kStages) & 1);
-        mbar_wait_bounded(&bars->q_smem, 0);
+          mbar_wait_bounded(&bars->l_full[i % kStages], (i / kStages) & 1, lim);
+        mbar_wait_bounded(&bars->q_smem, 0, lim);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_ltiles > 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kRows, kTile, false, false);
-      bool ok = mbar_wait(&bars->q_tmem, 0, abort_flag);
+      bool ok = mbar_wait(&bars->q_tmem, 0, abort_flag, lim);
       // seed scores: Q * seeds^T (the seed landmark rows, staged by the rows)
-      ok = ok && mbar_wait(&bars->seed_ready, 0, abort_flag);
+      ok = ok && mbar_wait(&bars->seed_ready, 0, abort_flag, lim);
       tc_fence_after();
       if (ok) {
         const uint32_t sd_addr = smem_u32(seed_stage);
@@ -564,9 +567,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t bias_addr = smem_u32(smem + Lay::bias);
       for (int i = 0; ok && i < n_scan; ++i) {
         const int s = i % kStages, sb = i % kSBufs;
-        if (!mbar_wait(&bars->l_full[s], (i / kStages) & 1, abort_flag)) break;
-        if (i >= kSBufs && !mbar_wait(&bars->s_empty[sb], ((i / kSBufs) - 1) & 1, abort_flag)) break;
-        if (i == kSBufs - 1 && !mbar_wait(&bars->seed_read, 0, abort_flag)) break;
+        if (!mbar_wait(&bars->l_full[s], (i / kStages) & 1, abort_flag, lim)) break;
+        if (i >= kSBufs && !mbar_wait(&bars->s_empty[sb], ((i / kSBufs) - 1) & 1, abort_flag, lim)) break;
+        if (i == kSBufs - 1 && !mbar_wait(&bars->seed_read, 0, abort_flag, lim)) break;
         tc_fence_after();
         const uint32_t l_addr = smem_u32(smem + Lay::l0 + s * Lay::kLBytes);
         const uint32_t d_tmem = s_tmem0 + sb * kTile;
@@ -583,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         mma_commit(&bars->l_empty[s]);
       }
       mma_commit(&bars->done);
-      mbar_wait_bounded(&bars->done, 0);
+      mbar_wait_bounded(&bars->done, 0, lim);
     }
   } else {
     // ---------------------------------------------------------- row threads
@@ -618,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       // q row -> tensor memory (A operand of the scoring MMA): the row's
       // 128-byte lines of the swizzled staging tile, two bf16 per column;
       // the owner also writes the masking operand [1, row < 64, 0, ...]
-      ok = mbar_wait(&bars->q_smem, 0, abort_flag);
+      ok = mbar_wait(&bars->q_smem, 0, abort_flag, lim);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         if (h < D / 64) {
@@ -663,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       fence_async_smem();
       mbar_arrive(&bars->seed_ready);
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->seed_full, 0, abort_flag));
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->seed_full, 0, abort_flag, lim));
       if (ok) {
         tc_fence_after();
         float sa[32];
@@ -725,13 +728,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (mbar_try_wait(&bars->s_full[sb], par)) { got = true; break; }
             if ((it & 63u) == 0) {
               if (*abort_flag) break;
-              if (globaltimer() - w0 > kWaitLimitNs) { *abort_flag = 1; break; }
+              if (globaltimer() - w0 > lim) { *abort_flag = 1; break; }
             }
           }
         }
         ok = got;
       } else {
-        ok = mbar_wait(&bars->s_full[sb], par, abort_flag);
+        ok = mbar_wait(&bars->s_full[sb], par, abort_flag, lim);
       }
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
@@ -772,7 +775,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (!room) {
               const uint64_t w0 = globaltimer();
               while (!room) {
-                if (*abort_flag || globaltimer() - w0 > kWaitLimitNs) break;
+                if (*abort_flag || globaltimer() - w0 > lim) break;
                 room = mb - ld_vol(&head_s[r]) < (uint32_t)kMbox;
               }
             }
@@ -804,7 +807,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (uint32_t it = 0;; ++it) {
         const uint32_t tv = drain();
         if ((tv & kDone) && mb == (tv & ~kDone)) { closed = true; break; }
-        if ((it & 63u) == 63u && (globaltimer() - w0 > kWaitLimitNs)) break;
+        if ((it & 63u) == 63u && (globaltimer() - w0 > lim)) break;
       }
       if (!closed) {
         *abort_flag = 1;

@@ -214,6 +214,38 @@ hils_status hils_decode_fwd_noalloc(const hils_params *p, const void *q, const v
                                     void *stream);
 
 /*
+ * Q-Cal scoring query (molayo1419.me, "Engineering details", Q-Cal): a
+ * low-rank learnable offset of the query, used only for the chunk scores.
+ *   q_cal[b,hq,t,:] = q[b,hq,t,:] + W_up[hq] (W_down h[b,t,:])
+ *   q       [B,Hq,L,d] in (params dtype)
+ *   h       [B,L,D] in (params dtype): the token's hidden state
+ *   w_down  [r,D] in (params dtype), shared by the heads
+ *   w_up    [Hq,d,r] in (params dtype)
+ *   q_cal   [B,Hq,L,d] out (params dtype), may not alias q
+ *   1 <= r <= 64, D >= 1; ws >= hils_qcal_workspace_size(p, r) bytes
+ *   (device scratch, B*L*r fp32 plus 256 bytes).
+ * Arithmetic: fp32, each product and partial sum rounded separately (no
+ * fused multiply-add), sums over D then over r in ascending order, and a bf16
+ * query rounded to nearest even at the end -- the pages fix no precision, so
+ * the query's own is used and the scoring pass sees exactly this query.
+ * hils_select on q_cal gives the selection, the chunk logits and lse_lmk of
+ * the calibrated scores; attention (hils_attn_fwd) keeps q.
+ */
+size_t hils_qcal_workspace_size(const hils_params *p, int r);
+hils_status hils_qcal_query(const hils_params *p, const void *q, const void *h,
+                            const void *w_down, const void *w_up, int D, int r, void *q_cal,
+                            void *ws, size_t ws_bytes, void *stream);
+
+/* hils_qcal_query, then hils_select on q_cal, then hils_attn_fwd on q, on
+ * one stream.  q_cal [B,Hq,L,d] is the caller's scratch (the calibrated
+ * query, left there). */
+hils_status hils_prefill_qcal(const hils_params *p, const void *q, const void *k, const void *v,
+                              const void *lmk_k, const void *h, const void *w_down,
+                              const void *w_up, int D, int r, void *q_cal, int32_t *sel_idx,
+                              float *chunk_w, float *lse_lmk, void *out, float *lse, void *ws,
+                              size_t ws_bytes, void *stream);
+
+/*
  * HoPE, the positional encoding of the pages (molayo1419.me, "Engineering
  * details", HoPE): rotary position embedding on the dimensions inside the
  * pre-training window, none (NoPE) on the rest.  Applied in place to q or k
@@ -231,6 +263,30 @@ hils_status hils_decode_fwd_noalloc(const hils_params *p, const void *q, const v
  */
 hils_status hils_hope(void *x, int dtype, int B, int H, int L, int d, int pos0,
                       int n_rope_pairs, double base, void *stream);
+
+/*
+ * The HoPE split (molayo1419.me, "Engineering details", HoPE: rotary
+ * embedding on the dimensions inside the pre-training window, none beyond):
+ * the number of rotate-half pairs i whose wavelength 2*pi*base^(2i/d) is at
+ * most train_len, the pre-training length in tokens.  These are the pairs
+ * 0 .. n-1 (the wavelength grows with i); pass n as n_rope_pairs.  Host
+ * function, no GPU work; returns -1 for d < 2, base <= 1 or NaN arguments.
+ */
+int hils_hope_rope_pairs(int d, double base, double train_len);
+
+/*
+ * Failure-path testing only (not for production use).  Every device wait of
+ * the prefill kernels (hils_select, hils_attn_fwd and the calls built on
+ * them) is bounded: after ns nanoseconds (default 2 s; ns = 0 restores it)
+ * the waiting role raises the kernel's abort flag, every role unwinds through
+ * the common teardown (in-flight copies and tensor-core work are waited for,
+ * tensor memory is freed) and, with params.debug_checks = 1, the call
+ * returns HILS_ERR_TIMEOUT.  withhold = 1 makes the scoring kernel keep back
+ * one arrival on its first landmark tile, so that such a wait runs out on
+ * purpose; nothing faults, traps or waits without a bound.  Process-wide;
+ * set it only while no other thread calls the library.
+ */
+void hils_test_set_wait_limit(uint64_t ns, int withhold);
 
 /* Static description of a status code. */
 const char *hils_status_string(hils_status s);

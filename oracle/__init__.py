@@ -44,6 +44,7 @@ This module compiles the C source with gcc on first use (``build()``).
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 from dataclasses import dataclass
@@ -336,6 +337,22 @@ def hope(x, positions, n_rope_pairs: int, base: float = 10000.0) -> np.ndarray:
         out[..., :, i:i + 1] = xi * c - xj * s
         out[..., :, i + half:i + half + 1] = xi * s + xj * c
     return out
+
+
+def rope_pairs(d: int, base: float, train_len: float) -> int:
+    """The HoPE split (molayo1419.me, "Engineering details", HoPE: rotary
+    embedding on the dimensions that fall inside the pre-training window,
+    none on the others): the number of rotate-half pairs i whose wavelength
+    2 pi base^(2i/d) -- the positions one full turn of pair i takes -- is at
+    most the pre-training length.  The wavelength grows with i, so these are
+    the pairs 0 .. n-1."""
+    n = 0
+    for i in range(d // 2):
+        if 2.0 * math.pi * float(base) ** (2.0 * i / d) <= float(train_len):
+            n = i + 1
+        else:
+            break
+    return n
 
 
 _default = None

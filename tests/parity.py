@@ -49,11 +49,12 @@ def admissible_sets(scores: np.ndarray, k: int):
 
 
 def compare_rows(p: oracle.Problem, inputs, rows, gpu: dict, ref: dict, dtype: str,
-                 decode: bool = False, orc=None) -> dict:
+                 decode: bool = False, orc=None, score_q=None) -> dict:
     """Compare GPU outputs of `rows` (numbered as in oracle rows(); decode
     heads when decode=True) with the oracle's result `ref` for the same rows.
     gpu/ref: dicts of numpy arrays sel [n,k], w [n,k], out [n,d], lse [n],
-    optional lse_lmk [n] and wfin [n,k+1].  Raises AssertionError on a
+    optional lse_lmk [n] and wfin [n,k+1].  score_q: the query of the
+    landmark scores when it is not q (Q-Cal).  Raises AssertionError on a
     mismatch; returns statistics."""
     orc = orc or oracle.default()
     tol = tolerances(dtype)
@@ -68,7 +69,8 @@ def compare_rows(p: oracle.Problem, inputs, rows, gpu: dict, ref: dict, dtype: s
     near_ties = 0
     for i in np.nonzero(~same)[0]:
         t = p.L - 1 if decode else int(rows[i] % p.L)
-        sc = orc.scores(p, q, lmk, [rows[i]], decode=decode)[0][: t // p.C]
+        sc = orc.scores(p, q if score_q is None else score_q, lmk, [rows[i]],
+                        decode=decode)[0][: t // p.C]
         alts = admissible_sets(sc, K)
         got = tuple(int(c) for c in gpu["sel"][i] if c >= 0)
         if got not in alts:

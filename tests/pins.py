@@ -538,6 +538,24 @@ def pin_qcal_scoring_query(orc):
     assert (got["sel"][can, 0] == star).all()
 
 
+def pin_hope_split_rule(orc):
+    """The HoPE split [KR "Engineering details", HoPE]: pairs whose wavelength
+    fits the pre-training length are rotated.  Hand values: d = 128, base
+    10^4, window 4096 -- the wavelength 2 pi 10^4^(i/64) is about 4080 at
+    i = 45 and 4710 at i = 46, so 46 pairs; base 5*10^5, window 65536 --
+    about 63 900 at i = 45 and 78 400 at i = 46, so 46 again; a window below
+    2 pi rotates nothing, exactly 2 pi rotates pair 0; a window beyond the
+    longest wavelength rotates every pair."""
+    from oracle import rope_pairs
+    assert 4000 < 2 * math.pi * 1e4 ** (45 / 64) < 4096 < 2 * math.pi * 1e4 ** (46 / 64) < 4800
+    assert rope_pairs(128, 1e4, 4096) == 46
+    assert 63000 < 2 * math.pi * 5e5 ** (45 / 64) < 65536 < 2 * math.pi * 5e5 ** (46 / 64)
+    assert rope_pairs(128, 5e5, 65536) == 46
+    assert rope_pairs(64, 1e4, 6.0) == 0
+    assert rope_pairs(64, 1e4, 2 * math.pi) == 1
+    assert rope_pairs(64, 1e4, 1e12) == 32
+
+
 ALL_PINS = [
     pin_landmark_logit_and_normaliser,
     pin_topk_planted_ties,
@@ -554,4 +572,5 @@ ALL_PINS = [
     pin_paged_decode_is_dense_decode,
     pin_hope_rotation_properties,
     pin_qcal_scoring_query,
+    pin_hope_split_rule,
 ]

@@ -130,11 +130,31 @@ def test_hope_rejects_bad_arguments(lib, kw):
     assert lib.hils_hope(None, hb.HILS_BF16, 1, 1, 1, 64, 0, 1, 10000.0, None) == 1
 
 
-def test_rope_pairs_for_matches_its_definition():
-    """The split helper counts exactly the pairs whose wavelength fits."""
-    import math
-    for d in (64, 128):
-        for base in (10000.0, 500000.0):
-            for train in (1, 6, 4096, 65536, 10 ** 12):
-                want = sum(1 for i in range(d // 2) if 2 * math.pi * base ** (2 * i / d) <= train)
-                assert hb.rope_pairs_for(d, base, train) == want
+def test_hope_split_rule_matches_the_oracle(lib):
+    """hils_hope_rope_pairs (the library's HoPE split) equals the pinned
+    oracle split on a grid of head sizes, bases and windows, and refuses
+    arguments outside its domain."""
+    import oracle
+    for d in (2, 16, 64, 128):
+        for base in (1.5, 10000.0, 500000.0):
+            for train in (1, 6, 2 * 3.141592653589793, 4096, 65536, 1e12):
+                assert lib.hils_hope_rope_pairs(d, base, float(train)) == oracle.rope_pairs(d, base, train)
+                assert hb.rope_pairs_for(d, base, train) == oracle.rope_pairs(d, base, train)
+    assert lib.hils_hope_rope_pairs(1, 1e4, 100.0) == -1
+    assert lib.hils_hope_rope_pairs(64, 1.0, 100.0) == -1
+    assert lib.hils_hope_rope_pairs(64, 1e4, float("nan")) == -1
+
+
+def test_qcal_rejects_bad_arguments(lib):
+    p = _params()
+    assert lib.hils_qcal_workspace_size(ctypes.byref(p), 0) == 0
+    assert lib.hils_qcal_workspace_size(ctypes.byref(p), 65) == 0
+    assert lib.hils_qcal_workspace_size(ctypes.byref(p), 16) == 256 + 1 * 1024 * 16 * 4
+    ws = lib.hils_qcal_workspace_size(ctypes.byref(p), 16)
+    args = lambda D, r, wsb: (ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, D, r, FAKE, FAKE, wsb, None)
+    assert lib.hils_qcal_query(*args(512, 0, ws)) == 2      # rank outside 1..64
+    assert lib.hils_qcal_query(*args(512, 65, ws)) == 2
+    assert lib.hils_qcal_query(*args(0, 16, ws)) == 1       # D < 1
+    assert lib.hils_qcal_query(*args(512, 16, ws - 1)) == 3  # workspace too small
+    assert lib.hils_qcal_query(ctypes.byref(p), FAKE, MISALIGNED, FAKE, FAKE, 512, 16, FAKE, FAKE,
+                               ws, None) == 1

@@ -116,6 +116,18 @@ def _qcal_ignored(self, p, q, k, v, lmk, qs, rows, nthreads=0):
     return self.rows(p, q, k, v, lmk, rows)
 
 
+def _split_on_frequency(d, base, train_len):
+    # compares the angular frequency instead of the wavelength
+    return sum(1 for i in range(d // 2) if base ** (-2.0 * i / d) <= train_len)
+
+
+def _split_without_two_pi(d, base, train_len):
+    n = 0
+    while n < d // 2 and base ** (2.0 * n / d) <= train_len:
+        n += 1
+    return n
+
+
 PY_MUTANTS = [
     ("gather_ignores_table", oracle, "gather_pages", _gather_ignores_table,
      pins.pin_paged_decode_is_dense_decode),
@@ -131,6 +143,8 @@ PY_MUTANTS = [
     ("qcal_query_used_for_attention", oracle.Oracle, "rows_qcal", _qcal_everywhere,
      pins.pin_qcal_scoring_query),
     ("qcal_query_ignored", oracle.Oracle, "rows_qcal", _qcal_ignored, pins.pin_qcal_scoring_query),
+    ("split_on_frequency", oracle, "rope_pairs", _split_on_frequency, pins.pin_hope_split_rule),
+    ("split_without_two_pi", oracle, "rope_pairs", _split_without_two_pi, pins.pin_hope_split_rule),
 ]
 
 
