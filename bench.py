@@ -28,6 +28,7 @@ bounded sample of rows per step, scaled to query-tokens/s.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -483,6 +484,57 @@ def tile_union_sizes(hb, sel):
     return (u_off[1:] - u_off[:-1]).cpu().numpy()
 
 
+def backward_work(w: W.Workload) -> float:
+    """Algorithmic FLOPs of one backward pass over all heads: per (row,
+    attended key) the logit recomputed (2d), dP = <dO, v> (2d), and the dq,
+    dk and dv updates (2d each) -- 10d, the attention-backward count -- plus
+    4d per (row, selected chunk) for the landmark gradients (ds lmk into dq,
+    ds q into dlmk)."""
+    t = np.arange(w.L, dtype=np.int64)
+    n_c = t // w.C
+    keys = np.minimum(w.topk, n_c) * w.C + (t % w.C) + 1
+    heads = w.B * w.Hq
+    return float((10 * w.d * keys.sum() + 4 * w.d * np.minimum(w.topk, n_c).sum()) * heads)
+
+
+def bench_backward(hb, synth, w, steps, warmup):
+    """hils_attn_bwd for the forward's selection on workload w (seeded dout
+    and dlse); fp32 arithmetic on the CUDA cores."""
+    dev = torch.device("cuda")
+    q, k, v, lmk = synth.make_inputs(w, "cuda", seed=w.seed)
+    g = torch.Generator(device=dev).manual_seed(w.seed + 41)
+    dout = torch.randn(q.shape, generator=g, device=dev).to(q.dtype)
+    dlse = torch.randn(q.shape[:3], generator=g, device=dev)
+    sel, cw, _ = hb.select(q, lmk, w.topk, w.M)
+    _, lse, _ = hb.attn_fwd(q, k, v, sel, cw, w.M)
+    p = hb.make_params(w.B, w.Hq, w.Hkv, w.L, w.d, w.topk, w.M, w.C, w.scale, q.dtype, False)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    dl = torch.empty(lmk.shape, dtype=torch.float32, device=dev)
+    ws = torch.empty(hb.lib().hils_attn_bwd_workspace_size(ctypes.byref(p)), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hb.hils_attn_bwd(p, q, k, v, lmk, sel, cw, lse, dout, dlse, dq, dk, dv, dl, ws, stream)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    flop = backward_work(w)
+    return {"value": w.B * w.L / (ms * 1e-3), "unit": "query-tokens/s", "ms_per_step": ms,
+            "algorithmic_tflops": flop / (ms * 1e-3) / 1e12, "bound": "alu",
+            "workspace_bytes": ws.numel()}
+
+
 def bench_qcal(hb, synth, w, steps, warmup, r=32):
     """The Q-Cal prefill of workload w: the calibrated scoring query
     (hils_qcal_query: z = W_down h per position, q + W_up z per head) timed
@@ -548,6 +600,16 @@ def union_stats(hb, sel, w):
             "union_p99": float(torch.quantile(sizes, 0.99).item()),
             "adjacent_overlap": round(float(np.mean(ov)) if ov else float("nan"), 4),
             "pages_adjacent_overlap": 0.928}
+
+
+def alu_peak_tflops(clocks) -> float:
+    """fp32 CUDA-core peak: 148 SMs x 128 FMA lanes x 2 FLOP per clock, at the
+    median SM clock sampled during the main timed region (the maximum clock
+    when none was sampled)."""
+    mhz = None
+    if clocks:
+        mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz")
+    return 148 * 128 * 2 * (mhz or 1965.0) * 1e6 / 1e12
 
 
 def cpu_baseline(w, host_inputs, budget_s=15.0):
@@ -706,6 +768,14 @@ def run_ours(args):
             "pool": f"{r3['paged_pages']} pages of 64 tokens x {w3.Hkv} KV heads, random order",
             "equal_to_dense": r3["paged_equal"]}
         del r3
+        torch.cuda.empty_cache()
+        try:
+            rb = bench_backward(hb, synth, W.SMALL_32K, max(3, args.steps), 2)
+            rb["frac"] = rb["algorithmic_tflops"] / alu_peak_tflops(res["clocks"])
+            rb["peak_source"] = "fp32 FMA issue rate of the CUDA cores (148 SMs x 128 lanes x 2 FLOP x SM clock)"
+            extra["backward_" + W.SMALL_32K.name] = rb
+        except Exception as e:  # an extra entry must not cost the main line
+            extra["backward_" + W.SMALL_32K.name] = {"error": str(e)[:200]}
         torch.cuda.empty_cache()
         try:
             extra["qcal_" + W.PREFILL_128K.name] = bench_qcal(hb, synth, W.PREFILL_128K,

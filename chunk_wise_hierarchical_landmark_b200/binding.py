@@ -40,6 +40,7 @@ EXPORTS = ["hils_workspace_size", "hils_select", "hils_union_capacity", "hils_un
            "hils_attn_fwd", "hils_prefill", "hils_decode_fwd", "hils_decode_fwd_paged",
            "hils_decode_fwd_noalloc", "hils_hope", "hils_qcal_workspace_size", "hils_qcal_query",
            "hils_prefill_qcal", "hils_hope_rope_pairs", "hils_test_set_wait_limit",
+           "hils_attn_bwd_workspace_size", "hils_attn_bwd",
            "hils_status_string", "hils_last_error", "hils_launch_count"]
 
 
@@ -64,6 +65,10 @@ def lib():
         L.hils_decode_fwd_paged.argtypes = [PP, P, P, P, I64, P, I, P, P, P, P, P, P, P, SZ, P]
         L.hils_decode_fwd_noalloc.argtypes = [PP, P, P, P, P, P, P, P, P, P, P]
         L.hils_hope.argtypes = [P, I, I, I, I, I, I, I, ctypes.c_double, P]
+        L.hils_attn_bwd_workspace_size.argtypes = [PP]
+        L.hils_attn_bwd_workspace_size.restype = SZ
+        L.hils_attn_bwd.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.hils_attn_bwd.restype = I
         L.hils_test_set_wait_limit.argtypes = [ctypes.c_uint64, I]
         L.hils_test_set_wait_limit.restype = None
         L.hils_hope_rope_pairs.argtypes = [I, ctypes.c_double, ctypes.c_double]
@@ -230,6 +235,32 @@ def prefill_qcal(q, k, v, lmk_k, h, w_down, w_up, topk, M=64, scale=None, debug_
     ws = qcal_workspace(p, w_down.shape[0], dev)
     hils_prefill_qcal(p, q, k, v, lmk_k, h, w_down, w_up, q_cal, sel, w, lse_lmk, out, lse, ws)
     return dict(out=out, lse=lse, sel_idx=sel, chunk_w=w, lse_lmk=lse_lmk, q_cal=q_cal)
+
+
+def hils_attn_bwd(p: Params, q, k, v, lmk_k, sel_idx, chunk_w, lse, dout, dlse, dq, dk, dv,
+                  dlmk, ws, stream=None):
+    _check(lib().hils_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(lmk_k),
+                               _ptr(sel_idx), _ptr(chunk_w), _ptr(lse), _ptr(dout), _ptr(dlse),
+                               _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlmk), *_ws_args(ws),
+                               _stream(stream)))
+
+
+def attn_bwd(q, k, v, lmk_k, sel_idx, chunk_w, lse, dout, dlse=None, scale=None,
+             debug_checks=False):
+    """Backward pass for a forward's selection: returns fp32 (dq, dk, dv, dlmk)."""
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    topk = sel_idx.shape[-1]
+    p = make_params(B, Hq, Hkv, L, d, topk, 64, 64, scale, q.dtype, debug_checks)
+    dev = q.device
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    dl = torch.empty(lmk_k.shape, dtype=torch.float32, device=dev)
+    n = lib().hils_attn_bwd_workspace_size(ctypes.byref(p))
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    hils_attn_bwd(p, q, k, v, lmk_k, sel_idx, chunk_w, lse, dout, dlse, dq, dk, dv, dl, ws)
+    return dq, dk, dv, dl
 
 
 def rope_pairs_for(d: int, base: float, train_len: int) -> int:

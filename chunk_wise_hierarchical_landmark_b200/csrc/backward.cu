@@ -1,0 +1,509 @@
+// Backward pass of the HiLS forward (aiweekly.co, the paragraph on the
+// mechanism: the chunk outputs are fused by the chunk retrieval scores, so
+// the loss reaches those scores; molayo1419.me, "Core idea": the landmark keys
+// take part in the forward pass and are trained by it).  The top-k choice is
+// a discrete decision and carries no gradient; the forward's selection
+// (sel_idx), its landmark logits (chunk_w) and its lse are inputs.
+//
+// Per row t and attended chunk c (its selected chunks, slots 0..k-1, and its
+// own chunk, slot k), with p the softmax inside the chunk and w the fusion
+// weights (out = sum_c w_c sum_j p_cj v_j):
+//   dP_j = <dO, v_j>,  g_c = sum_j p_cj dP_j = <dO, O_c>,  D = sum_c w_c g_c
+//   ds_c = w_c (g_c - D + dlse)                      (the chunk's fusion logit)
+//   dx_j = w_c p_cj (dP_j - g_c) [+ p_own,j ds_own]  (the own chunk's logit is
+//                                                     its log-sum-exp)
+//   dq_t  = scale (sum_cj dx_j k_j + sum_{c selected} ds_c lmk_c)
+//   dk_j += scale dx_j q_t,  dv_j += w_c p_cj dO_t,  dlmk_c += scale ds_c q_t
+// Three stages, all on the CUDA cores in fp32 (bf16 inputs widen exactly):
+//   bwd_rows_kernel   one warp per row: per-chunk softmax recomputed from q and
+//                     the chunk's keys, g_c, w_c, D, ds_c -> per-(row, slot)
+//                     records (lse_c, w_c, g_c, ds_c); then dq.
+//   transposed selection: per (b, kv head, chunk) the (row, slot) pairs that
+//                     select it (count, exclusive scan, fill; the order inside
+//                     a chunk's list follows the atomic fill).
+//   bwd_chunks_kernel one CTA per (b, kv head, chunk): the chunk's K and V in
+//                     shared memory, a thread per (key, quarter of the head
+//                     dimension) accumulating dk and dv over the rows that
+//                     attend the chunk (its own rows, causally, and the rows
+//                     that selected it), dlmk over the selecting rows.
+#include <cuda_bf16.h>
+
+#include "backward.h"
+#include "common.cuh"
+
+namespace hils {
+namespace {
+
+constexpr int kC = 64;
+constexpr int kRowWarps = 8;       // rows per CTA of the row pass
+constexpr int kChunkThreads = 256; // 64 keys x 4 quarters
+constexpr int kRowBatch = 8;       // rows staged together in the chunk pass
+
+template <typename T>
+__device__ __forceinline__ float ldf(const T *p);
+template <>
+__device__ __forceinline__ float ldf<float>(const float *p) { return *p; }
+template <>
+__device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16 *p) {
+  return __bfloat162float(*p);
+}
+
+// the lane's D/32 consecutive elements of a row, widened
+template <typename T, int P>
+__device__ __forceinline__ void ld_slice(const T *row, int lane, float (&f)[P]) {
+#pragma unroll
+  for (int u = 0; u < P; ++u) f[u] = ldf(row + lane * P + u);
+}
+
+// Dot products of x (the lane's slice) with 32 consecutive rows (a reduce-
+// scatter butterfly: lane l ends with the full dot product of row l).
+template <typename T, int P>
+__device__ __forceinline__ float dot32(const T *rows, int D, int lane, const float (&x)[P]) {
+  float v[32];
+#pragma unroll
+  for (int jj = 0; jj < 32; ++jj) {
+    float f[P];
+    ld_slice<T, P>(rows + (size_t)jj * D, lane, f);
+    float a = 0.0f;
+#pragma unroll
+    for (int u = 0; u < P; ++u) a = fmaf(f[u], x[u], a);
+    v[jj] = a;
+  }
+#pragma unroll
+  for (int sft = 16; sft >= 1; sft >>= 1) {
+    const bool upper = (lane & sft) != 0;
+#pragma unroll
+    for (int i = 0; i < sft; ++i) {
+      const float send = upper ? v[i] : v[i + sft];
+      const float keep = upper ? v[i + sft] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
+    }
+  }
+  return v[0];
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// The chunk's logits x (keys lane and lane + 32 of the chunk) and dP.
+template <typename T, int D>
+__device__ __forceinline__ void chunk_logits(const T *kc, const T *vc, int nkeys, int lane,
+                                             const float (&qv)[D / 32], const float (&dov)[D / 32],
+                                             float scale, float (&x)[2], float (&dp)[2]) {
+  constexpr int P = D / 32;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    if (hh * 32 < nkeys) {
+      // rows past the chunk's keys are not read: clamp to its last key
+      const int base = hh * 32;
+      const int nblk = min(32, nkeys - base);
+      if (nblk == 32) {
+        x[hh] = dot32<T, P>(kc + (size_t)base * D, D, lane, qv) * scale;
+        dp[hh] = dot32<T, P>(vc + (size_t)base * D, D, lane, dov);
+      } else {
+        float vx[32], vd[32];
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int j = base + min(jj, nblk - 1);
+          float fk[P], fv[P];
+          ld_slice<T, P>(kc + (size_t)j * D, lane, fk);
+          ld_slice<T, P>(vc + (size_t)j * D, lane, fv);
+          float a = 0.0f, b = 0.0f;
+#pragma unroll
+          for (int u = 0; u < P; ++u) {
+            a = fmaf(fk[u], qv[u], a);
+            b = fmaf(fv[u], dov[u], b);
+          }
+          vx[jj] = a;
+          vd[jj] = b;
+        }
+#pragma unroll
+        for (int sft = 16; sft >= 1; sft >>= 1) {
+          const bool upper = (lane & sft) != 0;
+#pragma unroll
+          for (int i = 0; i < sft; ++i) {
+            const float sx = upper ? vx[i] : vx[i + sft], kx = upper ? vx[i + sft] : vx[i];
+            const float sd = upper ? vd[i] : vd[i + sft], kd = upper ? vd[i + sft] : vd[i];
+            vx[i] = kx + __shfl_xor_sync(0xffffffffu, sx, sft);
+            vd[i] = kd + __shfl_xor_sync(0xffffffffu, sd, sft);
+          }
+        }
+        x[hh] = vx[0] * scale;
+        dp[hh] = vd[0];
+      }
+    } else {
+      x[hh] = 0.0f;
+      dp[hh] = 0.0f;
+    }
+  }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kRowWarps * 32)
+    bwd_rows_kernel(BwdSpec bs, const T *__restrict__ q, const T *__restrict__ k,
+                    const T *__restrict__ v, const T *__restrict__ lmk,
+                    const int32_t *__restrict__ sel, const float *__restrict__ chunk_w,
+                    const float *__restrict__ lse, const T *__restrict__ dout,
+                    const float *__restrict__ dlse, float4 *__restrict__ rec,
+                    float *__restrict__ dq, uint32_t *__restrict__ err) {
+  constexpr int P = D / 32;
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  if (row >= (long long)bs.B * bs.Hq * bs.L) return;
+  const int L = bs.L, K = bs.topk;
+  const int bh = (int)(row / L), t = (int)(row % L);
+  const int b = bh / bs.Hq, hq = bh % bs.Hq, hkv = hq / (bs.Hq / bs.Hkv);
+  const int own = t / kC;
+  const size_t kv0 = ((size_t)b * bs.Hkv + hkv) * L;  // first key row of the KV head
+  float qv[P], dov[P];
+  ld_slice<T, P>(q + (size_t)row * D, lane, qv);
+  ld_slice<T, P>(dout + (size_t)row * D, lane, dov);
+  const float lse_t = lse[row];
+  const float dl = dlse ? dlse[row] : 0.0f;
+  const int32_t *srow = sel + (size_t)row * K;
+  const float *wrow = chunk_w + (size_t)row * K;
+  float4 *rrow = rec + (size_t)row * (K + 1);
+
+  // pass 1: per attended chunk lse_c, w_c, g_c; D = sum w_c g_c
+  float Dsum = 0.0f;
+  for (int slot = 0; slot <= K; ++slot) {
+    int c;
+    float s_sel = 0.0f;
+    if (slot < K) {
+      c = srow[slot];
+      if (c < 0) continue;
+      if (c >= own) {
+        report(err, DEV_BAD_INDEX);
+        continue;
+      }
+      s_sel = wrow[slot];
+    } else {
+      c = own;
+    }
+    const int nkeys = slot < K ? kC : t - own * kC + 1;
+    float x[2], dp[2];
+    chunk_logits<T, D>(k + (kv0 + (size_t)c * kC) * D, v + (kv0 + (size_t)c * kC) * D, nkeys, lane,
+                       qv, dov, bs.scale, x, dp);
+    const bool in0 = lane < nkeys, in1 = lane + 32 < nkeys;
+    const float m = warp_max(fmaxf(in0 ? x[0] : -INFINITY, in1 ? x[1] : -INFINITY));
+    const float e0 = in0 ? __expf(x[0] - m) : 0.0f, e1 = in1 ? __expf(x[1] - m) : 0.0f;
+    const float l = warp_sum(e0 + e1);
+    const float lc = m + __logf(l);
+    const float g = warp_sum(e0 * dp[0] + e1 * dp[1]) / l;
+    const float s = slot < K ? s_sel : lc;
+    const float w = __expf(s - lse_t);
+    Dsum += w * g;
+    if (lane == 0) rrow[slot] = make_float4(lc, w, g, 0.0f);
+  }
+  __syncwarp();
+  // pass 2: ds_c, and dq = scale (sum_cj dx_j k_j + sum_sel ds_c lmk_c)
+  float acc[P];
+#pragma unroll
+  for (int u = 0; u < P; ++u) acc[u] = 0.0f;
+  for (int slot = 0; slot <= K; ++slot) {
+    int c;
+    if (slot < K) {
+      c = srow[slot];
+      if (c < 0 || c >= own) continue;
+    } else {
+      c = own;
+    }
+    float4 r4 = rrow[slot];
+    const float lc = r4.x, w = r4.y, g = r4.z;
+    const float ds = w * (g - Dsum + dl);
+    if (lane == 0) rrow[slot] = make_float4(lc, w, g, ds);
+    const int nkeys = slot < K ? kC : t - own * kC + 1;
+    const T *kc = k + (kv0 + (size_t)c * kC) * D;
+    float x[2], dp[2];
+    chunk_logits<T, D>(kc, v + (kv0 + (size_t)c * kC) * D, nkeys, lane, qv, dov, bs.scale, x, dp);
+    float dx[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const bool in = lane + 32 * hh < nkeys;
+      const float pj = in ? __expf(x[hh] - lc) : 0.0f;
+      dx[hh] = w * pj * (dp[hh] - g) + (slot == K ? pj * ds : 0.0f);
+    }
+    // sum_j dx_j k_j over the lane's slice (dx_j broadcast from its lane)
+    for (int j = 0; j < nkeys; ++j) {
+      const float dxj = __shfl_sync(0xffffffffu, j < 32 ? dx[0] : dx[1], j & 31);
+      float f[P];
+      ld_slice<T, P>(kc + (size_t)j * D, lane, f);
+#pragma unroll
+      for (int u = 0; u < P; ++u) acc[u] = fmaf(dxj, f[u], acc[u]);
+    }
+    if (slot < K) {
+      float f[P];
+      ld_slice<T, P>(lmk + (((size_t)b * bs.Hkv + hkv) * bs.nlmk + c) * D, lane, f);
+#pragma unroll
+      for (int u = 0; u < P; ++u) acc[u] = fmaf(ds, f[u], acc[u]);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < P; ++u) dq[(size_t)row * D + lane * P + u] = acc[u] * bs.scale;
+}
+
+// the (row, slot) pairs that select each (b, kv head, chunk): count ...
+__global__ void bwd_count_kernel(BwdSpec bs, const int32_t *__restrict__ sel,
+                                 uint32_t *__restrict__ cnt) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long n = (long long)bs.B * bs.Hq * bs.L * bs.topk;
+  if (i >= n) return;
+  const int c = sel[i];
+  const long long row = i / bs.topk;
+  const int t = (int)(row % bs.L), bh = (int)(row / bs.L);
+  if (c < 0 || c >= t / kC) return;
+  const int b = bh / bs.Hq, hkv = (bh % bs.Hq) / (bs.Hq / bs.Hkv);
+  atomicAdd(&cnt[((size_t)b * bs.Hkv + hkv) * bs.nch + c], 1u);
+}
+
+// ... exclusive scan (one CTA; the counts become the fill cursors, zeroed) ...
+__global__ void __launch_bounds__(1024) bwd_scan_kernel(uint32_t *__restrict__ cnt,
+                                                        uint32_t *__restrict__ off, int n) {
+  __shared__ uint32_t wsum[32];
+  __shared__ uint32_t carry_s;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) carry_s = 0;
+  __syncthreads();
+  for (int base = 0; base < n; base += 1024) {
+    const int i = base + tid;
+    const uint32_t c = i < n ? cnt[i] : 0u;
+    uint32_t x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t s = wsum[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += y;
+      }
+      wsum[lane] = s;
+    }
+    __syncthreads();
+    const uint32_t carry = carry_s;
+    const uint32_t excl = carry + (warp > 0 ? wsum[warp - 1] : 0u) + x - c;
+    if (i < n) {
+      off[i] = excl;
+      cnt[i] = 0u;
+    }
+    __syncthreads();
+    if (tid == 1023) carry_s = excl + c;
+    __syncthreads();
+  }
+  if (tid == 0) off[n] = carry_s;
+}
+
+// ... and fill
+__global__ void bwd_fill_kernel(BwdSpec bs, const int32_t *__restrict__ sel,
+                                const uint32_t *__restrict__ off, uint32_t *__restrict__ cur,
+                                int32_t *__restrict__ ent_row, uint8_t *__restrict__ ent_slot) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long n = (long long)bs.B * bs.Hq * bs.L * bs.topk;
+  if (i >= n) return;
+  const int c = sel[i];
+  const long long row = i / bs.topk;
+  const int t = (int)(row % bs.L), bh = (int)(row / bs.L);
+  if (c < 0 || c >= t / kC) return;
+  const int b = bh / bs.Hq, hkv = (bh % bs.Hq) / (bs.Hq / bs.Hkv);
+  const size_t seg = ((size_t)b * bs.Hkv + hkv) * bs.nch + c;
+  const uint32_t pos = off[seg] + atomicAdd(&cur[seg], 1u);
+  ent_row[pos] = (int32_t)row;
+  ent_slot[pos] = (uint8_t)(i % bs.topk);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kChunkThreads)
+    bwd_chunks_kernel(BwdSpec bs, const T *__restrict__ q, const T *__restrict__ k,
+                      const T *__restrict__ v, const T *__restrict__ dout,
+                      const float4 *__restrict__ rec, const uint32_t *__restrict__ off,
+                      const int32_t *__restrict__ ent_row, const uint8_t *__restrict__ ent_slot,
+                      float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ dlmk) {
+  constexpr int DQ = D / 4;  // dimensions per thread
+  // K, V [key][quarter][DQ + 1] and the staged rows [row][quarter][DQ + 1]:
+  // the padding puts the 32 lanes of a warp (8 keys x 4 quarters) on
+  // distinct banks
+  extern __shared__ float csm[];
+  float *ks = csm;
+  float *vs = ks + kC * 4 * (DQ + 1);
+  float *qs = vs + kC * 4 * (DQ + 1);
+  float *os = qs + kRowBatch * 4 * (DQ + 1);
+  __shared__ float4 st[kRowBatch];
+  __shared__ int own_s[kRowBatch];  // 1: the row's own chunk (slot k), with its position offset
+  __shared__ int jmax_s[kRowBatch];
+  const int seg = blockIdx.x;  // (b * Hkv + hkv) * nch + c
+  const int c = seg % bs.nch, bk = seg / bs.nch;
+  const int b = bk / bs.Hkv, hkv = bk % bs.Hkv;
+  const int G = bs.Hq / bs.Hkv;
+  const int L = bs.L, K = bs.topk;
+  const int nkeys = min(kC, L - c * kC);
+  const size_t krow0 = (size_t)bk * L + (size_t)c * kC;
+  const int tid = threadIdx.x;
+  const int j = tid >> 2, qd = tid & 3;
+  auto at = [](int r, int e) { return (r * 4 + e / DQ) * (DQ + 1) + e % DQ; };
+  for (int i = tid; i < kC * D; i += kChunkThreads) {
+    const int jj = i / D, e = i % D;
+    ks[at(jj, e)] = jj < nkeys ? ldf(k + (krow0 + jj) * D + e) : 0.0f;
+    vs[at(jj, e)] = jj < nkeys ? ldf(v + (krow0 + jj) * D + e) : 0.0f;
+  }
+  float ak[DQ], av[DQ];
+#pragma unroll
+  for (int u = 0; u < DQ; ++u) ak[u] = av[u] = 0.0f;
+  float al = 0.0f;  // dlmk: thread tid < D owns dimension tid
+  // rows: own rows (every query head of the group, positions of this chunk),
+  // then the rows that selected the chunk
+  const int n_own = G * nkeys;
+  const uint32_t s0 = off[seg], s1 = off[seg + 1];
+  const int n_rows = n_own + (int)(s1 - s0);
+  for (int r0 = 0; r0 < n_rows; r0 += kRowBatch) {
+    const int nb = min(kRowBatch, n_rows - r0);
+    __syncthreads();
+    for (int i = tid; i < nb * D; i += kChunkThreads) {
+      const int rr = i / D, e = i % D;
+      const int ri = r0 + rr;
+      long long row;
+      if (ri < n_own) {
+        const int g = ri / nkeys, tt = ri % nkeys;
+        row = ((long long)b * bs.Hq + hkv * G + g) * L + (long long)c * kC + tt;
+      } else {
+        row = ent_row[s0 + (ri - n_own)];
+      }
+      qs[at(rr, e)] = ldf(q + (size_t)row * D + e);
+      os[at(rr, e)] = ldf(dout + (size_t)row * D + e);
+      if (e == 0) {
+        const int slot = ri < n_own ? K : (int)ent_slot[s0 + (ri - n_own)];
+        st[rr] = rec[(size_t)row * (K + 1) + slot];
+        own_s[rr] = ri < n_own ? 1 : 0;
+        jmax_s[rr] = ri < n_own ? (ri % nkeys) : kC - 1;
+      }
+    }
+    __syncthreads();
+    for (int rr = 0; rr < nb; ++rr) {
+      float a = 0.0f, d2 = 0.0f;
+      const float *qr = qs + (rr * 4 + qd) * (DQ + 1), *orow = os + (rr * 4 + qd) * (DQ + 1);
+      const float *kr = ks + (j * 4 + qd) * (DQ + 1), *vr = vs + (j * 4 + qd) * (DQ + 1);
+#pragma unroll
+      for (int u = 0; u < DQ; ++u) {
+        a = fmaf(qr[u], kr[u], a);
+        d2 = fmaf(orow[u], vr[u], d2);
+      }
+      a += __shfl_xor_sync(0xffffffffu, a, 1);
+      a += __shfl_xor_sync(0xffffffffu, a, 2);
+      d2 += __shfl_xor_sync(0xffffffffu, d2, 1);
+      d2 += __shfl_xor_sync(0xffffffffu, d2, 2);
+      const float4 s4 = st[rr];  // lse_c, w_c, g_c, ds_c
+      const bool in = j < nkeys && j <= jmax_s[rr];
+      const float pj = in ? __expf(a * bs.scale - s4.x) : 0.0f;
+      const float dx = s4.y * pj * (d2 - s4.z) + (own_s[rr] ? pj * s4.w : 0.0f);
+      const float pw = s4.y * pj;
+#pragma unroll
+      for (int u = 0; u < DQ; ++u) {
+        av[u] = fmaf(pw, orow[u], av[u]);
+        ak[u] = fmaf(dx, qr[u], ak[u]);
+      }
+      if (!own_s[rr] && tid < D) al = fmaf(s4.w, qs[at(rr, tid)], al);
+    }
+  }
+  if (j < nkeys) {
+#pragma unroll
+    for (int u = 0; u < DQ; ++u) {
+      const int e = qd * DQ + u;
+      dk[(krow0 + j) * D + e] = ak[u] * bs.scale;
+      dv[(krow0 + j) * D + e] = av[u];
+    }
+  }
+  if (c < bs.nlmk && tid < D) dlmk[((size_t)bk * bs.nlmk + c) * D + tid] = al * bs.scale;
+}
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+BwdSpec bwd_spec(int B, int Hq, int Hkv, int L, int d, int topk, float scale) {
+  BwdSpec bs{};
+  bs.B = B;
+  bs.Hq = Hq;
+  bs.Hkv = Hkv;
+  bs.L = L;
+  bs.d = d;
+  bs.topk = topk;
+  bs.scale = scale;
+  bs.nch = (L + kC - 1) / kC;
+  bs.nlmk = L / kC;
+  return bs;
+}
+
+size_t bwd_workspace_bytes(const BwdSpec &bs) {
+  const size_t rows = (size_t)bs.B * bs.Hq * bs.L;
+  const size_t nseg = (size_t)bs.B * bs.Hkv * bs.nch;
+  size_t n = 256;                                    // error word
+  n += al256(rows * (bs.topk + 1) * sizeof(float4)); // per-(row, slot) records
+  n += al256(nseg * sizeof(uint32_t));               // counts / fill cursors
+  n += al256((nseg + 1) * sizeof(uint32_t));         // segment offsets
+  n += al256(rows * bs.topk * sizeof(int32_t));      // entries: rows
+  n += al256(rows * bs.topk);                        // entries: slots
+  return n;
+}
+
+cudaError_t bwd_run(const BwdSpec &bs, bool bf16, const void *q, const void *k, const void *v,
+                    const void *lmk, const int32_t *sel, const float *chunk_w, const float *lse,
+                    const void *dout, const float *dlse, float *dq, float *dk, float *dv,
+                    float *dlmk, void *ws, uint32_t *err, cudaStream_t st, int *launches) {
+  const size_t rows = (size_t)bs.B * bs.Hq * bs.L;
+  const size_t nseg = (size_t)bs.B * bs.Hkv * bs.nch;
+  unsigned char *p = static_cast<unsigned char *>(ws) + 256;
+  auto take = [&](size_t bytes) {
+    unsigned char *r = p;
+    p += al256(bytes);
+    return r;
+  };
+  float4 *rec = reinterpret_cast<float4 *>(take(rows * (bs.topk + 1) * sizeof(float4)));
+  uint32_t *cnt = reinterpret_cast<uint32_t *>(take(nseg * sizeof(uint32_t)));
+  uint32_t *off = reinterpret_cast<uint32_t *>(take((nseg + 1) * sizeof(uint32_t)));
+  int32_t *ent_row = reinterpret_cast<int32_t *>(take(rows * bs.topk * sizeof(int32_t)));
+  uint8_t *ent_slot = reinterpret_cast<uint8_t *>(take(rows * bs.topk));
+  cudaError_t e;
+  const unsigned rgrid = (unsigned)((rows + kRowWarps - 1) / kRowWarps);
+#define HILS_BWD_ROWS(T, DD)                                                                     \
+  bwd_rows_kernel<T, DD><<<rgrid, kRowWarps * 32, 0, st>>>(                                     \
+      bs, (const T *)q, (const T *)k, (const T *)v, (const T *)lmk, sel, chunk_w, lse,           \
+      (const T *)dout, dlse, rec, dq, err)
+  if (bf16) { if (bs.d == 64) HILS_BWD_ROWS(__nv_bfloat16, 64); else HILS_BWD_ROWS(__nv_bfloat16, 128); }
+  else { if (bs.d == 64) HILS_BWD_ROWS(float, 64); else HILS_BWD_ROWS(float, 128); }
+#undef HILS_BWD_ROWS
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(cnt, 0, nseg * sizeof(uint32_t), st)) != cudaSuccess) return e;
+  const long long nsel = (long long)rows * bs.topk;
+  const unsigned sgrid = (unsigned)((nsel + 255) / 256);
+  bwd_count_kernel<<<sgrid, 256, 0, st>>>(bs, sel, cnt);
+  bwd_scan_kernel<<<1, 1024, 0, st>>>(cnt, off, (int)nseg);
+  bwd_fill_kernel<<<sgrid, 256, 0, st>>>(bs, sel, off, cnt, ent_row, ent_slot);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+#define HILS_BWD_CHUNKS(T, DD)                                                                   \
+  do {                                                                                           \
+    auto kern = bwd_chunks_kernel<T, DD>;                                                        \
+    const size_t smem = (size_t)(2 * kC + 2 * kRowBatch) * 4 * (DD / 4 + 1) * sizeof(float);     \
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e; \
+    kern<<<(unsigned)nseg, kChunkThreads, smem, st>>>(bs, (const T *)q, (const T *)k,            \
+        (const T *)v, (const T *)dout, rec, off, ent_row, ent_slot, dk, dv, dlmk);               \
+  } while (0)
+  if (bf16) { if (bs.d == 64) HILS_BWD_CHUNKS(__nv_bfloat16, 64); else HILS_BWD_CHUNKS(__nv_bfloat16, 128); }
+  else { if (bs.d == 64) HILS_BWD_CHUNKS(float, 64); else HILS_BWD_CHUNKS(float, 128); }
+#undef HILS_BWD_CHUNKS
+  *launches += 5;
+  return cudaGetLastError();
+}
+
+}  // namespace hils

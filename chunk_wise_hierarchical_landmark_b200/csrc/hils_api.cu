@@ -12,6 +12,7 @@
 #include "hope.h"
 #include "paged.h"
 #include "qcal.h"
+#include "backward.h"
 
 #define HILS_API extern "C" __attribute__((visibility("default")))
 
@@ -377,6 +378,52 @@ HILS_API hils_status hils_hope(void *x, int dtype, int B, int H, int L, int d, i
   g_launches += n;
   if (e != cudaSuccess) return cuda_fail(e, "hope launch");
   return HILS_OK;
+}
+
+HILS_API size_t hils_attn_bwd_workspace_size(const hils_params *p) {
+  if (check_params(p) != HILS_OK) return 0;
+  return hils::bwd_workspace_bytes(
+      hils::bwd_spec(p->B, p->Hq, p->Hkv, p->L, p->d, p->topk, p->scale));
+}
+
+HILS_API hils_status hils_attn_bwd(const hils_params *p, const void *q, const void *k,
+                                   const void *v, const void *lmk_k, const int32_t *sel_idx,
+                                   const float *chunk_w, const float *lse, const void *dout,
+                                   const float *dlse, float *dq, float *dk, float *dv,
+                                   float *dlmk, void *ws, size_t ws_bytes, void *stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  NEED(q);
+  NEED(k);
+  NEED(v);
+  NEED(sel_idx);
+  NEED(chunk_w);
+  NEED(lse);
+  NEED(dout);
+  MAYBE(dlse);
+  NEED(dq);
+  NEED(dk);
+  NEED(dv);
+  if (p->L >= p->chunk) {
+    NEED(lmk_k);
+    NEED(dlmk);
+  }
+  if ((int64_t)p->B * p->Hq * p->L * p->topk >= (int64_t)1 << 31)
+    return fail(HILS_ERR_UNSUPPORTED, "B*Hq*L*topk must be below 2^31 for the backward pass");
+  const hils::BwdSpec bs = hils::bwd_spec(p->B, p->Hq, p->Hkv, p->L, p->d, p->topk, p->scale);
+  const size_t need = hils::bwd_workspace_bytes(bs);
+  if (!ws || ws_bytes < need)
+    return fail(HILS_ERR_WORKSPACE, "backward needs %zu bytes of workspace, got %zu", need, ws_bytes);
+  NEED(ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t *err = nullptr;
+  if ((s = debug_begin(p, ws, ws_bytes, &err, st)) != HILS_OK) return s;
+  int n = 0;
+  cudaError_t e = hils::bwd_run(bs, p->dtype == HILS_BF16, q, k, v, lmk_k, sel_idx, chunk_w, lse,
+                                dout, dlse, dq, dk, dv, dlmk, ws, err, st, &n);
+  g_launches += n;
+  if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+  return debug_end(err, st);
 }
 
 HILS_API void hils_test_set_wait_limit(uint64_t ns, int withhold) {

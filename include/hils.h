@@ -214,6 +214,33 @@ hils_status hils_decode_fwd_noalloc(const hils_params *p, const void *q, const v
                                     void *stream);
 
 /*
+ * Backward pass of the forward above (aiweekly.co, mechanism paragraph: the
+ * chunk outputs are fused by the chunk scores, so the loss reaches them;
+ * molayo1419.me, "Core idea": the landmark keys take part in the forward
+ * pass).  The top-k choice carries no gradient: the forward's selection is an
+ * input.  Gradients of sum(out * dout) + sum(lse * dlse) with respect to q, k,
+ * v and the landmark keys:
+ *   q, k, v, lmk_k     in, as for the forward (params dtype)
+ *   sel_idx, chunk_w   in: the forward's selection and landmark logits
+ *   lse  [B,Hq,L] fp32 in: the forward's lse
+ *   dout [B,Hq,L,d]    in (params dtype); dlse [B,Hq,L] fp32 in, may be NULL (0)
+ *   dq [B,Hq,L,d], dk, dv [B,Hkv,L,d], dlmk [B,Hkv,L/C,d]  fp32 out (every
+ *   element written; dlmk may be NULL when L < C)
+ *   ws >= hils_attn_bwd_workspace_size(p) bytes: per-(row, attended chunk)
+ *   records of 16 bytes and the transposed selection (8 bytes per selected
+ *   chunk of every row), plus 2 KB.
+ * dk, dv and dlmk sum over the rows that attend a chunk in an order set by
+ * atomic operations, so their last bits may differ from run to run; dq is
+ * deterministic.  B*Hq*L*topk must be below 2^31.
+ */
+size_t hils_attn_bwd_workspace_size(const hils_params *p);
+hils_status hils_attn_bwd(const hils_params *p, const void *q, const void *k, const void *v,
+                          const void *lmk_k, const int32_t *sel_idx, const float *chunk_w,
+                          const float *lse, const void *dout, const float *dlse, float *dq,
+                          float *dk, float *dv, float *dlmk, void *ws, size_t ws_bytes,
+                          void *stream);
+
+/*
  * Q-Cal scoring query (molayo1419.me, "Engineering details", Q-Cal): a
  * low-rank learnable offset of the query, used only for the chunk scores.
  *   q_cal[b,hq,t,:] = q[b,hq,t,:] + W_up[hq] (W_down h[b,t,:])

@@ -86,3 +86,13 @@ def test_near_tie_sample_flags_a_wrong_selection():
             planted += 1
     st = bench.near_tie_sample(w, q, lmk, bad, n_rows=200, seed=3)
     assert planted > 0 and st["index_mismatches"] >= planted - st["near_ties"]
+
+
+def test_backward_work_counts_rows_one_by_one():
+    w = W.PREFILL_128K.with_(B=1, Hq=2, Hkv=1, L=200, d=8, topk=2)
+    want = 0
+    for t in range(w.L):
+        n_c = t // w.C
+        keys = min(w.topk, n_c) * w.C + t % w.C + 1
+        want += 10 * w.d * keys + 4 * w.d * min(w.topk, n_c)
+    assert bench.backward_work(w) == want * w.B * w.Hq

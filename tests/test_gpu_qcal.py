@@ -31,10 +31,12 @@ CASES = [
     (W.SMALL_32K.with_(B=2, Hq=2, Hkv=2, L=700, topk=16), 96, 8),
     # fp32 workload, odd D, rank 64 (the largest)
     (W.TINY_F32.with_(Hq=2, Hkv=1, L=650), 130, 64),
+    # an odd rank and an odd hidden size
+    (W.PREFILL_128K.with_(Hq=4, Hkv=2, L=333, topk=4), 37, 5),
 ]
 
 
-@pytest.mark.parametrize("w,D,r", CASES, ids=["bf16_gqa", "bf16_d64", "f32_r64"])
+@pytest.mark.parametrize("w,D,r", CASES, ids=["bf16_gqa", "bf16_d64", "f32_r64", "bf16_r5"])
 def test_qcal_prefill_matches_oracle(w, D, r):
     q, k, v, lmk = synth.make_inputs(w, "cpu")
     h, wd, wu = qcal_inputs(w, D, r, seed=w.seed + D)
