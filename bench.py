@@ -478,6 +478,61 @@ def bench_hope(hb, w, steps, warmup, train_len=65536, base=500000.0):
     return dict(ms=ms, bytes=nbytes, npairs=npairs)
 
 
+def bench_hope_fused(hb, synth, w, steps, warmup, train_len=65536, base=500000.0):
+    """Prefill with HoPE on the queries two ways: the query pre-pass
+    (hils_hope over q, into a copy) followed by hils_prefill, and
+    hils_prefill_hope, which rotates each query tile as the kernels stage
+    it.  The keys are rotated once beforehand in both (a cache holds them
+    rotated).  The two must agree bit for bit."""
+    dev = torch.device("cuda")
+    q, k, v, lmk = synth.make_inputs(w, dev)
+    npairs = hb.rope_pairs_for(w.d, base, train_len)
+    hb.hils_hope(k, npairs, 0, base)
+    p = hb.make_params(w.B, w.Hq, w.Hkv, w.L, w.d, w.topk, w.M, w.C, w.scale, q.dtype)
+    ws_t = hb.workspace(p, hb.HILS_OP_PREFILL, dev)
+    outs = []
+    for _ in range(2):
+        outs.append(dict(sel=torch.empty((w.B, w.Hq, w.L, w.topk), dtype=torch.int32, device=dev),
+                         cw=torch.empty((w.B, w.Hq, w.L, w.topk), dtype=torch.float32,
+                                        device=dev),
+                         ll=torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev),
+                         out=torch.empty_like(q),
+                         lse=torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)))
+    q_rot = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+
+    def two_step():
+        o = outs[0]
+        q_rot.copy_(q)
+        hb.hils_hope(q_rot, npairs, 0, base, stream)
+        hb.hils_prefill(p, q_rot, k, v, lmk, o["sel"], o["cw"], o["ll"], o["out"], o["lse"],
+                        ws_t, stream)
+
+    def fused():
+        o = outs[1]
+        hb.hils_prefill_hope(p, q, k, v, lmk, 0, npairs, base, o["sel"], o["cw"], o["ll"],
+                             o["out"], o["lse"], ws_t, stream)
+
+    res = dict(npairs=npairs)
+    for name, fn in (("prepass_ms", two_step), ("fused_ms", fused)):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        res[name] = a.elapsed_time(b) / steps
+    res["equal"] = all(torch.equal(outs[0][n].view(torch.int32) if outs[0][n].dtype ==
+                                   torch.float32 else outs[0][n],
+                                   outs[1][n].view(torch.int32) if outs[1][n].dtype ==
+                                   torch.float32 else outs[1][n]) for n in outs[0])
+    return res
+
+
 def tile_union_sizes(hb, sel):
     """Union size of every 128-row tile (the unit the attention kernel walks)."""
     u_off, _ = hb.union(sel, M=128)
@@ -793,6 +848,15 @@ def run_ours(args):
                 "hbm_frac": hgbs / peaks["hbm_gbs"]}
         except Exception as e:  # an extra entry must not cost the main line
             extra["hope_prepass_" + w.name] = {"error": str(e)[:200]}
+        torch.cuda.empty_cache()
+        try:
+            r5 = bench_hope_fused(hb, synth, W.PREFILL_128K, max(3, args.steps), 2)
+            r5["note"] = ("prefill with HoPE on q: hils_hope pre-pass over a copy of q then "
+                          "hils_prefill, against hils_prefill_hope (rotation in the kernels' "
+                          "query staging); keys pre-rotated in both")
+            extra["hope_fused_" + W.PREFILL_128K.name] = r5
+        except Exception as e:  # an extra entry must not cost the main line
+            extra["hope_fused_" + W.PREFILL_128K.name] = {"error": str(e)[:200]}
         line["workloads"] = extra
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, res["host_inputs"])

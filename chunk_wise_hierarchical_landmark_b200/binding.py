@@ -40,7 +40,7 @@ EXPORTS = ["hils_workspace_size", "hils_select", "hils_union_capacity", "hils_un
            "hils_attn_fwd", "hils_prefill", "hils_decode_fwd", "hils_decode_fwd_paged",
            "hils_decode_fwd_noalloc", "hils_hope", "hils_qcal_workspace_size", "hils_qcal_query",
            "hils_prefill_qcal", "hils_hope_rope_pairs", "hils_test_set_wait_limit",
-           "hils_attn_bwd_workspace_size", "hils_attn_bwd",
+           "hils_attn_bwd_workspace_size", "hils_attn_bwd", "hils_prefill_hope",
            "hils_status_string", "hils_last_error", "hils_launch_count"]
 
 
@@ -65,6 +65,9 @@ def lib():
         L.hils_decode_fwd_paged.argtypes = [PP, P, P, P, I64, P, I, P, P, P, P, P, P, P, SZ, P]
         L.hils_decode_fwd_noalloc.argtypes = [PP, P, P, P, P, P, P, P, P, P, P]
         L.hils_hope.argtypes = [P, I, I, I, I, I, I, I, ctypes.c_double, P]
+        L.hils_prefill_hope.argtypes = [PP, P, P, P, P, I, I, ctypes.c_double, P, P, P, P, P, P,
+                                        SZ, P]
+        L.hils_prefill_hope.restype = I
         L.hils_attn_bwd_workspace_size.argtypes = [PP]
         L.hils_attn_bwd_workspace_size.restype = SZ
         L.hils_attn_bwd.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
@@ -261,6 +264,32 @@ def attn_bwd(q, k, v, lmk_k, sel_idx, chunk_w, lse, dout, dlse=None, scale=None,
     ws = torch.empty(n, dtype=torch.uint8, device=dev)
     hils_attn_bwd(p, q, k, v, lmk_k, sel_idx, chunk_w, lse, dout, dlse, dq, dk, dv, dl, ws)
     return dq, dk, dv, dl
+
+
+def hils_prefill_hope(p: Params, q, k, v, lmk_k, pos0, n_rope_pairs, base, sel_idx, chunk_w,
+                      lse_lmk, out, lse, ws=None, stream=None):
+    _check(lib().hils_prefill_hope(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(lmk_k),
+                                   int(pos0), int(n_rope_pairs), float(base), _ptr(sel_idx),
+                                   _ptr(chunk_w), _ptr(lse_lmk), _ptr(out), _ptr(lse),
+                                   *_ws_args(ws), _stream(stream)))
+
+
+def prefill_hope(q, k, v, lmk_k, topk, n_rope_pairs, base, pos0=0, M=64, scale=None,
+                 debug_checks=False):
+    """Prefill with HoPE applied to the (unrotated) queries inside the kernels;
+    k holds rotated keys.  Returns dict(out, lse, sel_idx, chunk_w, lse_lmk)."""
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    p = make_params(B, Hq, Hkv, L, d, topk, M, 64, scale, q.dtype, debug_checks)
+    dev = q.device
+    sel = torch.empty((B, Hq, L, topk), dtype=torch.int32, device=dev)
+    w = torch.empty((B, Hq, L, topk), dtype=torch.float32, device=dev)
+    lse_lmk = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+    hils_prefill_hope(p, q, k, v, lmk_k, pos0, n_rope_pairs, base, sel, w, lse_lmk, out, lse,
+                      workspace(p, HILS_OP_PREFILL, dev))
+    return dict(out=out, lse=lse, sel_idx=sel, chunk_w=w, lse_lmk=lse_lmk)
 
 
 def rope_pairs_for(d: int, base: float, train_len: int) -> int:

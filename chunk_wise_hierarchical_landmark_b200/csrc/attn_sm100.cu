@@ -36,6 +36,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "hope.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -72,7 +73,7 @@ struct Layout {
 // s_full (QK^T done), p_full (the rows stored P), p_free (PV read P).
 struct Bars {
   uint64_t q, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages], s_full[2],
-      p_full[2], p_free[2], o_full, done;
+      p_full[2], p_free[2], o_full, done, q_rot;
 };
 static_assert(sizeof(Bars) <= 24 * 8, "barrier area");
 
@@ -122,6 +123,49 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// HoPE in place on row r of the swizzled bf16 Q tile (D/64 blocks of [128
+// rows][128 bytes]) at position pos: element e pairs with e + D/2, i.e. the
+// same 16-byte chunk of the other block (D = 128) or the chunk four chunks
+// away in the same block (D = 64).
+template <int D>
+__device__ __forceinline__ void hope_row_inplace(unsigned char *tile, int r, const HopeParams &hp,
+                                                 long long pos) {
+  constexpr int HALF = D / 2;
+#pragma unroll 1
+  for (int j = 0; j < (D == 128 ? 8 : 4); ++j) {
+    // first-half chunk (block 0, chunk j) and its partner
+    unsigned char *pa = tile + r * 128 + ((j ^ (r & 7)) << 4);
+    unsigned char *pb = D == 128 ? tile + kRows * 128 + r * 128 + ((j ^ (r & 7)) << 4)
+                                 : tile + r * 128 + (((j + 4) ^ (r & 7)) << 4);
+    uint4 a4 = *reinterpret_cast<const uint4 *>(pa);
+    uint4 b4 = *reinterpret_cast<const uint4 *>(pb);
+    uint32_t aw[4] = {a4.x, a4.y, a4.z, a4.w}, bw[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      float ya[2], yb[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int i = 8 * j + 2 * m + u;  // the pair (first element i < HALF)
+        const float xi = __uint_as_float(u ? (aw[m] & 0xFFFF0000u) : (aw[m] << 16));
+        const float xj = __uint_as_float(u ? (bw[m] & 0xFFFF0000u) : (bw[m] << 16));
+        ya[u] = xi;
+        yb[u] = xj;
+        if (i < hp.npairs && i < HALF) {
+          float sn, cs;
+          hope_sincos(hp.theta[i], pos, sn, cs);
+          hope_rotate(xi, xj, sn, cs, ya[u], yb[u]);
+        }
+      }
+      const __nv_bfloat162 a2 = __floats2bfloat162_rn(ya[0], ya[1]);
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(yb[0], yb[1]);
+      aw[m] = *reinterpret_cast<const uint32_t *>(&a2);
+      bw[m] = *reinterpret_cast<const uint32_t *>(&b2);
+    }
+    *reinterpret_cast<uint4 *>(pa) = make_uint4(aw[0], aw[1], aw[2], aw[3]);
+    *reinterpret_cast<uint4 *>(pb) = make_uint4(bw[0], bw[1], bw[2], bw[3]);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -129,7 +173,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                       const __grid_constant__ CUtensorMap tm_v, RowSpec rs,
                       const int32_t *__restrict__ sel, const float *__restrict__ chunk_w,
                       __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out,
-                      float *__restrict__ wfin, uint32_t *__restrict__ err) {
+                      float *__restrict__ wfin, uint32_t *__restrict__ err,
+                      const HopeParams hp) {
   using Lay = Layout<D>;
   // The 128-byte-swizzled tiles need a 1024-byte aligned base; the dynamic
   // shared window starts there (no static shared memory), checked here.
@@ -171,6 +216,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->done, 1);
+    mbar_init(&bars->q_rot, kRows);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -379,7 +425,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         mma_commit(&bars->p_free[b2]);
         return true;
       };
-      bool ok = mbar_wait(&bars->q, 0, abort_flag, lim);
+      // with HoPE the rows turn the Q tile before the first QK^T reads it
+      bool ok = hp.npairs > 0 ? mbar_wait(&bars->q_rot, 0, abort_flag, lim)
+                              : mbar_wait(&bars->q, 0, abort_flag, lim);
       if (ok) ok = qk(0);
       if (ok && n_steps > 1) ok = qk(1);
       for (int j = 0; ok && j < n_steps; ++j) {
@@ -397,6 +445,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float scale2 = rs.scale * kLog2e;
     float M2 = 0.0f, lse2_own = 0.0f;
     int ptr = 0;
+    bool ok = true;
     // the row's next four selected chunks (ids and logits), loaded ahead so
     // that a global load has several steps to land before it is used
     int qc[4];
@@ -407,12 +456,20 @@ __global__ void __launch_bounds__(kThreads, 2)
       qc[u] = have ? __ldg(mysel + u) : -1;
       qw[u] = have ? __ldg(myw + u) : 0.0f;
     }
+    if (hp.npairs > 0) {
+      // HoPE on the fly: each row turns its own line of the Q tile once the
+      // tile has landed; the generic-proxy writes are fenced for the tensor
+      // core before the arrival the MMA issuer waits on
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->q, 0, abort_flag, lim));
+      if (ok) hope_row_inplace<D>(q_s, r, hp, (long long)hp.pos0 + t);
+      fence_async_smem();
+      mbar_arrive(&bars->q_rot);
+    }
     ChunkIter it;
     it.init(bitmap, c0, n_own);
-    bool ok = true;
     // sum of the rounded probabilities this row stores (four partial sums)
     float rsum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    for (int i = 0; i < n_steps; ++i) {
+    for (int i = 0; ok && i < n_steps; ++i) {
       const int c = it.next();
       const uint32_t sb = s_tmem + 64 * (i & 1) + lane_off;
       ok = mbar_wait(&bars->s_full[i & 1], (i >> 1) & 1, abort_flag, lim);
@@ -592,7 +649,7 @@ size_t attn_sm100_smem(int d, int L) {
 
 cudaError_t attn_sm100(const RowSpec &rs, const void *q, const void *k, const void *v,
                        const int32_t *sel, const float *w, void *out, float *lse, float *wfin,
-                       uint32_t *err, cudaStream_t st) {
+                       uint32_t *err, cudaStream_t st, const HopeParams &hp) {
   CUtensorMap tq, tk, tv;
   cudaError_t e;
   const uint64_t qrows = (uint64_t)rs.B * rs.Hq * rs.L, kvrows = (uint64_t)rs.B * rs.Hkv * rs.L;
@@ -604,11 +661,11 @@ cudaError_t attn_sm100(const RowSpec &rs, const void *q, const void *k, const vo
   if (rs.d == 64) {
     auto kern = attn_sm100_kernel<64>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, rs, sel, w, (__nv_bfloat16 *)out, lse, wfin, err);
+    kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, rs, sel, w, (__nv_bfloat16 *)out, lse, wfin, err, hp);
   } else {
     auto kern = attn_sm100_kernel<128>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, rs, sel, w, (__nv_bfloat16 *)out, lse, wfin, err);
+    kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, rs, sel, w, (__nv_bfloat16 *)out, lse, wfin, err, hp);
   }
   return cudaGetLastError();
 }

@@ -317,6 +317,7 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
   const float *sc = scores + (size_t)h * n;
   if (staged) {
     // one pass over HBM/L2 with every load in flight; the rest reads shared memory
+#pragma unroll 8
     for (int i = tid; i < n; i += 256) sc_s[i] = sc[i];
     __syncthreads();
     sc = sc_s;
@@ -326,6 +327,7 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
 
   // log-sum-exp: block maximum, then the sum of exponentials against it
   float m = -INFINITY;
+#pragma unroll 8
   for (int i = tid; i < n; i += 256) m = fmaxf(m, sc[i]);
   for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane == 0) red[warp] = m;
@@ -335,8 +337,10 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
   for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
   __syncthreads();
   float l = 0.0f;
-  if (n > 0)
+  if (n > 0) {
+#pragma unroll 8
     for (int i = tid; i < n; i += 256) l += __expf(sc[i] - m);
+  }
   for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
   if (lane == 0) red[warp] = l;
   __syncthreads();
@@ -353,6 +357,102 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
       wrow[i] = i < n ? sc[i] : -INFINITY;
     }
     return;
+  }
+  // Threshold path (staged logits, at least k blocks of 32): the k-th largest
+  // block maximum tau bounds the k-th largest logit from below (the k best
+  // blocks hold k distinct logits >= tau), so every kept chunk is among the
+  // few logits >= tau; their exact top-k by (logit desc, chunk asc) is taken
+  // by counting, then written in chunk order through a bitmap.
+  const int nb = (n + 31) / 32;
+  constexpr int kCandCap = 8 * 256 / 2;  // 64-bit candidate keys in hist_w
+  if (staged && nb >= K && nb <= 256) {
+    uint32_t *bmax = hist;  // [256] block maxima (order-preserving bits)
+    uint64_t *cand = reinterpret_cast<uint64_t *>(hist_w);
+    __shared__ int n_cand_s;
+    __shared__ uint32_t tau_s;
+    __shared__ uint32_t keep[256];  // one bit per chunk (n <= 8192)
+    if (tid == 0) n_cand_s = 0;
+    keep[tid] = 0u;
+    if (tid < nb) {
+      // the block's 32 logits, visited in a lane-rotated order (no conflicts)
+      uint32_t m = 0u;
+#pragma unroll 8
+      for (int u = 0; u < 32; ++u) {
+        const int i = tid * 32 + ((u + tid) & 31);
+        if (i < n) m = max(m, score_bits(sc[i]));
+      }
+      bmax[tid] = m;
+    }
+    __syncthreads();
+    if (tid < nb) {
+      // rank of this block's maximum (ties: lower block first)
+      const uint32_t v = bmax[tid];
+      int rank = 0;
+#pragma unroll 8
+      for (int b2 = 0; b2 < nb; ++b2) {
+        const uint32_t x = bmax[b2];
+        rank += (x > v || (x == v && b2 < tid)) ? 1 : 0;
+      }
+      if (rank == K - 1) tau_s = v;
+    }
+    __syncthreads();
+    const uint32_t tau = tau_s;
+    for (int i0 = 0; i0 < n; i0 += 256) {
+      const int i = i0 + tid;
+      const uint32_t kb = i < n ? score_bits(sc[i]) : 0u;
+      const bool in = i < n && kb >= tau;
+      const uint32_t bal = __ballot_sync(0xffffffffu, in);
+      int base = 0;
+      if (lane == 0 && bal) base = atomicAdd(&n_cand_s, __popc(bal));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      const int pos = base + __popc(bal & ((1u << lane) - 1u));
+      if (in && pos < kCandCap) cand[pos] = ((uint64_t)kb << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)i);
+    }
+    __syncthreads();
+    const int m = n_cand_s;
+    if (m <= kCandCap) {
+      // exact rank of every candidate key; the k best are kept
+      for (int a = tid; a < m; a += 256) {
+        const uint64_t x = cand[a];
+        int rank = 0;
+#pragma unroll 8
+        for (int b2 = 0; b2 < m; ++b2) rank += cand[b2] > x ? 1 : 0;
+        if (rank < K) {
+          const int i = (int)(0xFFFFFFFFu - (uint32_t)x);
+          atomicOr(&keep[i >> 5], 1u << (i & 31));
+        }
+      }
+      __syncthreads();
+      // write in chunk order: word w's kept chunks go after those of words < w
+      if (warp == 0) {
+        int carry = 0;
+        for (int w0 = 0; w0 < 256; w0 += 32) {
+          const uint32_t word = keep[w0 + lane];
+          const int c1 = __popc(word);
+          int x = c1;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+          }
+          int pos = carry + x - c1;
+          uint32_t wd = word;
+          while (wd) {
+            const int i = (w0 + lane) * 32 + __ffs(wd) - 1;
+            wd &= wd - 1;
+            if (pos < K) {
+              srow[pos] = i;
+              wrow[pos] = sc[i];
+            }
+            ++pos;
+          }
+          carry += __shfl_sync(0xffffffffu, x, 31);
+        }
+      }
+      return;
+    }
+    // too many candidates (logits crowding at tau): the radix select below
+    __syncthreads();
   }
   // radix select of the K-th largest key: per pass a histogram of one 8-bit
   // digit of the keys that match the digits chosen so far (one histogram per
@@ -724,30 +824,29 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(DecodeSpec ds, const T
       const int pr = tid + s * 256;
       const int g = pr / e2n, e2 = pr % e2n;
       if (g < G && ((mask >> g) & 1u)) {
-        // two partial sums per output column keep the FMA chains short
-        float o0 = 0.0f, o1 = 0.0f, p0 = 0.0f, p1 = 0.0f;
-        for (int j = 0; j <= jmax; ++j) {
-          const float pj = xs[g * kC + j];
-          float v0, v1;
+        // even and odd keys in two packed (column pair) partial sums: short
+        // FMA chains, one fp32x2 FMA per key
+        auto vpair = [&](int j) {
           if constexpr (sizeof(T) == 2) {
             const uint32_t w = *reinterpret_cast<const uint32_t *>(vt + j * D + 2 * e2);
-            v0 = __uint_as_float(w << 16);
-            v1 = __uint_as_float(w & 0xFFFF0000u);
+            return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
           } else {
-            const float2 w = *reinterpret_cast<const float2 *>(vt + j * D + 2 * e2);
-            v0 = w.x;
-            v1 = w.y;
+            return *reinterpret_cast<const float2 *>(vt + j * D + 2 * e2);
           }
-          if (j & 1) {
-            p0 = fmaf(pj, v0, p0);
-            p1 = fmaf(pj, v1, p1);
-          } else {
-            o0 = fmaf(pj, v0, o0);
-            o1 = fmaf(pj, v1, o1);
-          }
+        };
+        float2 oe = make_float2(0.0f, 0.0f), oo = make_float2(0.0f, 0.0f);
+        int j = 0;
+#pragma unroll 4
+        for (; j + 1 <= jmax; j += 2) {
+          const float2 pp = *reinterpret_cast<const float2 *>(xs + g * kC + j);
+          oe = __ffma2_rn(make_float2(pp.x, pp.x), vpair(j), oe);
+          oo = __ffma2_rn(make_float2(pp.y, pp.y), vpair(j + 1), oo);
         }
-        o0 += p0;
-        o1 += p1;
+        if (j <= jmax) {
+          const float pj = xs[g * kC + j];
+          oe = __ffma2_rn(make_float2(pj, pj), vpair(j), oe);
+        }
+        const float o0 = oe.x + oo.x, o1 = oe.y + oo.y;
         const float lg = st[g * 4 + 2], l = st[g * 4 + 1];
         float mo = 0.0f, ln = 0.0f;
 #pragma unroll

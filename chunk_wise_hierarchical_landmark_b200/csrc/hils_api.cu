@@ -109,15 +109,17 @@ hils_status debug_end(uint32_t *err, cudaStream_t st) {
   return HILS_OK;
 }
 
+const hils::HopeParams kNoHope{};
+
 hils_status do_select(const hils_params *p, const hils::RowSpec &rs, const void *q,
                       const void *lmk, int32_t *sel, float *w, float *lse_lmk, uint32_t *err,
-                      cudaStream_t st) {
+                      cudaStream_t st, const hils::HopeParams &hp = kNoHope) {
   // bf16 prefill scores on the tensor cores; fp32 and the decode row on the CUDA cores
   const bool tc = p->dtype == HILS_BF16 && rs.t_first == 0 && rs.t_count == rs.L;
   int n = 0;
   cudaError_t e;
   if (tc) {
-    e = hils::select_sm100(rs, q, lmk, sel, w, lse_lmk, err, st, &n);
+    e = hils::select_sm100(rs, q, lmk, sel, w, lse_lmk, err, st, &n, hp);
   } else {
     e = hils::select_simt(rs, p->dtype == HILS_BF16, q, lmk, sel, w, lse_lmk, st);
     n = 1;
@@ -128,11 +130,12 @@ hils_status do_select(const hils_params *p, const hils::RowSpec &rs, const void 
 
 hils_status do_attn(const hils_params *p, const hils::RowSpec &rs, const void *q, const void *k,
                     const void *v, const int32_t *sel, const float *w, void *out, float *lse,
-                    float *wfin, uint32_t *err, cudaStream_t st) {
+                    float *wfin, uint32_t *err, cudaStream_t st,
+                    const hils::HopeParams &hp = kNoHope) {
   // bf16 prefill runs on the tensor cores; fp32 (no exact tensor-core path)
   // and the single decode row run on the CUDA cores
   const bool tc = p->dtype == HILS_BF16 && rs.t_first == 0 && rs.t_count == rs.L;
-  cudaError_t e = tc ? hils::attn_sm100(rs, q, k, v, sel, w, out, lse, wfin, err, st)
+  cudaError_t e = tc ? hils::attn_sm100(rs, q, k, v, sel, w, out, lse, wfin, err, st, hp)
                      : hils::attn_simt(rs, p->dtype == HILS_BF16, q, k, v, sel, w, out, lse,
                                        wfin, err, st);
   g_launches += 1;
@@ -378,6 +381,42 @@ HILS_API hils_status hils_hope(void *x, int dtype, int B, int H, int L, int d, i
   g_launches += n;
   if (e != cudaSuccess) return cuda_fail(e, "hope launch");
   return HILS_OK;
+}
+
+HILS_API hils_status hils_prefill_hope(const hils_params *p, const void *q, const void *k,
+                                       const void *v, const void *lmk_k, int pos0,
+                                       int n_rope_pairs, double base, int32_t *sel_idx,
+                                       float *chunk_w, float *lse_lmk, void *out, float *lse,
+                                       void *ws, size_t ws_bytes, void *stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  if (p->dtype != HILS_BF16)
+    return fail(HILS_ERR_UNSUPPORTED,
+                "the fused HoPE prefill runs on the bf16 tensor-core path; rotate fp32 queries "
+                "with hils_hope and call hils_prefill");
+  if (n_rope_pairs < 0 || n_rope_pairs > p->d / 2)
+    return fail(HILS_ERR_INVALID_ARG, "n_rope_pairs=%d outside [0, d/2]", n_rope_pairs);
+  if (pos0 < 0 || (int64_t)pos0 + p->L - 1 >= (int64_t)1 << 31)
+    return fail(HILS_ERR_INVALID_ARG, "positions pos0 .. pos0+L-1 must lie in [0, 2^31)");
+  if (!std::isfinite(base) || !(base > 1.0)) return fail(HILS_ERR_INVALID_ARG, "base must be finite and > 1");
+  NEED(q);
+  NEED(k);
+  NEED(v);
+  NEED(sel_idx);
+  NEED(chunk_w);
+  MAYBE(lse_lmk);
+  NEED(out);
+  NEED(lse);
+  if (p->L >= p->chunk) NEED(lmk_k);
+  const hils::HopeParams hp = hils::hope_params(p->d, n_rope_pairs, pos0, base);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t *err = nullptr;
+  if ((s = debug_begin(p, ws, ws_bytes, &err, st)) != HILS_OK) return s;
+  const hils::RowSpec rs = prefill_rows(p);
+  if ((s = do_select(p, rs, q, lmk_k, sel_idx, chunk_w, lse_lmk, err, st, hp)) != HILS_OK) return s;
+  if ((s = do_attn(p, rs, q, k, v, sel_idx, chunk_w, out, lse, nullptr, err, st, hp)) != HILS_OK)
+    return s;
+  return debug_end(err, st);
 }
 
 HILS_API size_t hils_attn_bwd_workspace_size(const hils_params *p) {

@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "hope.cuh"
+
 namespace hils {
 
 // Rows handled by a launch: positions [t_first, t_first + t_count) of every
@@ -30,15 +32,16 @@ cudaError_t attn_simt(const RowSpec &rs, bool bf16, const void *q, const void *k
 size_t simt_attn_smem(int d, int L, int C);
 
 // tcgen05 attention for bf16 prefill (attn_sm100.cu)
+// hp: HoPE applied to the query tile on the fly (hp.npairs = 0: none)
 cudaError_t attn_sm100(const RowSpec &rs, const void *q, const void *k, const void *v,
                        const int32_t *sel, const float *w, void *out, float *lse, float *wfin,
-                       uint32_t *err, cudaStream_t st);
+                       uint32_t *err, cudaStream_t st, const HopeParams &hp);
 size_t attn_sm100_smem(int d, int L);
 
 // tcgen05 landmark scoring + top-k for bf16 prefill (select_sm100.cu)
 cudaError_t select_sm100(const RowSpec &rs, const void *q, const void *lmk, int32_t *sel,
                          float *w, float *lse_lmk, uint32_t *err, cudaStream_t st,
-                         int *launches);
+                         int *launches, const HopeParams &hp);
 
 }  // namespace hils
 

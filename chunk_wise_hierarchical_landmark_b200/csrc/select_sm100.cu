@@ -41,6 +41,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "hope.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -349,13 +350,60 @@ __device__ __forceinline__ uint32_t ge_mask(const float (&a)[32], float u) {
   return (mq[0] | mq[1]) | (mq[2] | mq[3]);
 }
 
+// Row r of a swizzled bf16 Q tile (D/64 blocks of [128 rows][128 bytes])
+// with HoPE applied at position pos, into the row's tensor-memory columns
+// from taddr on (two bf16 per column, as the tile packs them).  Pair i joins
+// elements i and i + D/2; 16-byte chunk j of the first half (pairs 8j ..
+// 8j+7) has its partners in chunk j of block 1 (D = 128) or chunk j + 4 of
+// block 0 (D = 64).  The row's two threads split the chunks, h taking j = h,
+// h+2, ..., so each angle is formed once per row; every chunk pair goes out
+// as two 4-column stores (no register array is indexed by the rolled loop).
+template <int D>
+__device__ __forceinline__ void hope_row_split(const unsigned char *tile, int r, int h,
+                                               const HopeParams &hp, long long pos,
+                                               uint32_t taddr) {
+  constexpr int kChunks = D / 16;  // 16-byte chunks in the first half
+#pragma unroll 1
+  for (int j = h; j < kChunks; j += 2) {
+    const unsigned char *row = tile + r * 128;
+    const uint4 a4 = *reinterpret_cast<const uint4 *>(row + ((j ^ (r & 7)) << 4));
+    const uint4 b4 = D == 128
+        ? *reinterpret_cast<const uint4 *>(row + kRows * 128 + ((j ^ (r & 7)) << 4))
+        : *reinterpret_cast<const uint4 *>(row + (((j + 4) ^ (r & 7)) << 4));
+    uint32_t aw[4] = {a4.x, a4.y, a4.z, a4.w}, bw[4] = {b4.x, b4.y, b4.z, b4.w};
+    if (8 * j < hp.npairs) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        float ya[2], yb[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int i = 8 * j + 2 * m + u;
+          ya[u] = __uint_as_float(u ? (aw[m] & 0xFFFF0000u) : (aw[m] << 16));
+          yb[u] = __uint_as_float(u ? (bw[m] & 0xFFFF0000u) : (bw[m] << 16));
+          if (i < hp.npairs) {
+            float sn, cs;
+            hope_sincos(hp.theta[i], pos, sn, cs);
+            hope_rotate(ya[u], yb[u], sn, cs, ya[u], yb[u]);
+          }
+        }
+        const __nv_bfloat162 a2 = __floats2bfloat162_rn(ya[0], ya[1]);
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(yb[0], yb[1]);
+        aw[m] = *reinterpret_cast<const uint32_t *>(&a2);
+        bw[m] = *reinterpret_cast<const uint32_t *>(&b2);
+      }
+    }
+    tmem_st4(taddr + 4 * j, aw);
+    tmem_st4(taddr + D / 4 + 4 * j, bw);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
     select_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_l, RowSpec rs,
                         int32_t *__restrict__ sel, float *__restrict__ chunk_w,
                         float *__restrict__ lse_lmk, uint32_t *__restrict__ err, int level,
-                        const __nv_bfloat16 *__restrict__ lmk_raw) {
+                        const __nv_bfloat16 *__restrict__ lmk_raw, const HopeParams hp) {
   using Lay = SelLayout<D>;
   // The 128-byte-swizzled tiles need a 1024-byte aligned base; the dynamic
   // shared window starts there (there is no static shared memory), which the
@@ -624,7 +672,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       ok = mbar_wait(&bars->q_smem, 0, abort_flag, lim);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
-        if (h < D / 64) {
+        if (hp.npairs > 0) {
+          // HoPE on the fly: the query rotated as the pre-pass would
+          hope_row_split<D>(smem + Lay::l0, r, h, hp, (long long)hp.pos0 + t, q_tmem + lane_off);
+        } else if (h < D / 64) {
           uint32_t w[32];
           const unsigned char *line = smem + Lay::l0 + h * kRows * 128 + r * 128;
 #pragma unroll
@@ -851,7 +902,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 cudaError_t select_sm100(const RowSpec &rs, const void *q, const void *lmk, int32_t *sel,
                          float *w, float *lse_lmk, uint32_t *err, cudaStream_t st,
-                         int *launches) {
+                         int *launches, const HopeParams &hp) {
   CUtensorMap tq, tl;
   cudaError_t e;
   const int nlmk = rs.L / rs.C;
@@ -868,7 +919,7 @@ cudaError_t select_sm100(const RowSpec &rs, const void *q, const void *lmk, int3
     for (int lv = 0; lv < kLevels; ++lv) {
       const int n = level_count(lv, ntiles);
       if (n == 0) continue;
-      kern<<<dim3(n, rs.B * rs.Hq), kThreads, smem, st>>>(tq, tl, rs, sel, w, lse_lmk, err, lv, lraw);
+      kern<<<dim3(n, rs.B * rs.Hq), kThreads, smem, st>>>(tq, tl, rs, sel, w, lse_lmk, err, lv, lraw, hp);
       ++*launches;
       if ((e2 = cudaGetLastError()) != cudaSuccess) return e2;
     }

@@ -292,6 +292,22 @@ hils_status hils_hope(void *x, int dtype, int B, int H, int L, int d, int pos0,
                       int n_rope_pairs, double base, void *stream);
 
 /*
+ * Prefill with HoPE applied to the queries inside the kernels (bf16 only):
+ * q is taken as it comes, unrotated, and each query tile is rotated as it is
+ * staged -- in the scoring kernel on its way to tensor memory, in the
+ * attention kernel in shared memory -- exactly as hils_hope(q, pos0,
+ * n_rope_pairs, base) would rotate it (same arithmetic, same bits), so the
+ * query pre-pass over HBM disappears.  k must hold keys already rotated, as
+ * a cache does (hils_hope on the keys once, when they enter it); the
+ * landmark keys are used as given.  Everything else is hils_prefill's.
+ * fp32 parameters return HILS_ERR_UNSUPPORTED (rotate with hils_hope).
+ */
+hils_status hils_prefill_hope(const hils_params *p, const void *q, const void *k, const void *v,
+                              const void *lmk_k, int pos0, int n_rope_pairs, double base,
+                              int32_t *sel_idx, float *chunk_w, float *lse_lmk, void *out,
+                              float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * The HoPE split (molayo1419.me, "Engineering details", HoPE: rotary
  * embedding on the dimensions inside the pre-training window, none beyond):
  * the number of rotate-half pairs i whose wavelength 2*pi*base^(2i/d) is at
