@@ -152,7 +152,7 @@ __device__ __forceinline__ void hope_row_inplace(unsigned char *tile, int r, con
         yb[u] = xj;
         if (i < hp.npairs && i < HALF) {
           float sn, cs;
-          hope_sincos(hp.theta[i], pos, sn, cs);
+          hope_sincos(hp.turns[i], pos, sn, cs);
           hope_rotate(xi, xj, sn, cs, ya[u], yb[u]);
         }
       }

@@ -31,7 +31,7 @@ __global__ void __launch_bounds__(kHopeThreads) hope_kernel(T *__restrict__ x, i
   const int i = threadIdx.x;
   if (i >= hp.npairs) return;
   const int half = d / 2;
-  const double th = hp.theta[i];
+  const unsigned long long th = hp.turns[i];
   T *seq = x + (size_t)blockIdx.y * L * d;
   for (int t = blockIdx.x * blockDim.y + threadIdx.y; t < L; t += gridDim.x * blockDim.y) {
     float sn, cs;

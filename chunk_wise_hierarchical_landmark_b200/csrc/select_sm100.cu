@@ -382,7 +382,7 @@ __device__ __forceinline__ void hope_row_split(const unsigned char *tile, int r,
           yb[u] = __uint_as_float(u ? (bw[m] & 0xFFFF0000u) : (bw[m] << 16));
           if (i < hp.npairs) {
             float sn, cs;
-            hope_sincos(hp.theta[i], pos, sn, cs);
+            hope_sincos(hp.turns[i], pos, sn, cs);
             hope_rotate(ya[u], yb[u], sn, cs, ya[u], yb[u]);
           }
         }
