@@ -616,12 +616,10 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-}  // namespace
-
-// 2-D bf16 tensor map over a row-major [rows, cols] array with a
-// [box_rows, 64]-element box and 128-byte swizzle.
-cudaError_t make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
-                           uint32_t box_rows) {
+// 2-D tensor map over a row-major [rows, cols] array of 2- or 4-byte
+// elements with a [box_rows, 128 bytes] box and 128-byte swizzle.
+static cudaError_t make_tmap_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                                uint32_t box_rows, bool f32) {
   static EncodeTiledFn encode = nullptr;
   if (!encode) {
     void *fn = nullptr;
@@ -630,15 +628,28 @@ cudaError_t make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t rows, ui
     if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
     encode = reinterpret_cast<EncodeTiledFn>(fn);
   }
+  const uint32_t esz = f32 ? 4 : 2;
   const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint64_t strides[1] = {cols * esz};
+  const cuuint32_t box[2] = {128 / esz, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
-                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = encode(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                      2, const_cast<void *>(base), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                           uint32_t box_rows) {
+  return make_tmap_2d(map, base, rows, cols, box_rows, false);
+}
+
+cudaError_t make_tmap_f32(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                          uint32_t box_rows) {
+  return make_tmap_2d(map, base, rows, cols, box_rows, true);
 }
 
 size_t attn_sm100_smem(int d, int L) {

@@ -16,14 +16,19 @@
 //                  N = 16 padded heads) -> the logits of the G heads, into a
 //                  workspace array (decode_gemv: the same on the CUDA cores,
 //                  one thread per landmark, for fp32 or G > 16)
-//   decode_topk    grid (B*Hq): the head's log-sum-exp and exact top-k
-//                  (radix select on the logit bits) -> sel_idx / chunk_w,
-//                  ascending chunk ids, lse_lmk
+//   decode_topk    grid (B*Hq): the head's log-sum-exp and exact top-k ->
+//                  sel_idx / chunk_w, ascending chunk ids, lse_lmk.  The k-th
+//                  largest of the 32-logit block maxima bounds the k-th
+//                  largest logit from below; the logits at or above it are
+//                  ranked exactly by (logit, chunk) keys (radix select on the
+//                  logit bits when there are too many of them)
 //   decode_union   grid (B*Hkv): the KV head's chunk union with a per-entry
 //                  head mask and per-head logits
-//   decode_attn    grid (Q, B*Hkv): up to 16 union chunks per CTA, each chunk's
-//                  K and V staged once; per head an online (max, sum, acc)
-//                  partial over its chunks.  With a page table the chunk's
+//   decode_attn    grid (Q, B*Hkv), 128 threads: up to 16 union chunks per
+//                  CTA, each chunk's K and V staged once for all G heads (a
+//                  thread per key for the logits, a thread per column pair
+//                  for P V); per head an online (max, sum, acc) partial over
+//                  its chunks.  With a page table the chunk's
 //                  [64][d] slab of KV head hkv is read from its page
 //                  ([num_pages][Hkv][64][d] pools) instead of the dense cache
 //   decode_combine grid (B*Hq): partials -> out, lse
@@ -654,25 +659,88 @@ __global__ void __launch_bounds__(256) decode_union_kernel(DecodeSpec ds,
 }
 
 // ---------------------------------------------------------------------------
-template <typename T, int D>
-__global__ void __launch_bounds__(256) decode_attn_kernel(DecodeSpec ds, const T *__restrict__ q,
-                                                          const T *__restrict__ kc,
-                                                          const T *__restrict__ vc,
-                                                          const PagedKV pg,
-                                                          const int32_t *__restrict__ u_c,
-                                                          const uint32_t *__restrict__ u_mask,
-                                                          const float *__restrict__ u_logit,
-                                                          const int32_t *__restrict__ u_count,
-                                                          float *__restrict__ part,
-                                                          uint32_t *__restrict__ err) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  T *ks = reinterpret_cast<T *>(smem);             // [2][64][D]
-  T *vs = ks + 2 * kC * D;                         // [2][64][D]
-  float *qs = reinterpret_cast<float *>(vs + 2 * kC * D);  // [G][D] (scaled)
-  float *xs = qs + kMaxG * D;                      // [G][64] logits / probabilities
-  float *st = xs + kMaxG * kC;                     // [G][4]: per-chunk m, l, weight logit
-  __shared__ uint64_t bars[2];
-  __shared__ int abort_flag;
+// Chunk attention of the union.  CTA (qi, bk) takes union entries
+// [16 qi, 16 qi + 16) of (b, kv-head) bk; each chunk's K and V are copied
+// into shared memory once (double-buffered bulk copies: the next chunk in
+// flight while this one is used) and serve all G query heads of the KV head.
+//   logits   thread t: key j = t mod 64 and part t / 64 of the head
+//            dimension; K arrives as 128-byte-swizzled tiles of a 2-D tensor
+//            copy, so the 8 lanes of a shared-memory wavefront, reading the
+//            same 16-byte column chunk of 8 consecutive rows, find it at 8
+//            different bank groups; the scaled queries are broadcast, all
+//            heads accumulate in fp32 pairs, and the parts meet in shared
+//            memory
+//   softmax  warp w takes heads w, w + 4: the chunk's maximum and sum per
+//            head, the probabilities stored key-major [64][GB]
+//   P V      thread t: columns (2p, 2p+1), p = t mod (D/2), over key slice
+//            t / (D/2), every head at once (pairs of heads per fp32x2 FMA)
+// A running (max, sum, acc) per head merges the chunks under their fusion
+// logits; the key slices are summed at the end into one partial record
+// [M, L, acc[D]] per (bk, qi, g).
+#ifndef HILS_DECODE_THREADS
+#define HILS_DECODE_THREADS 256
+#endif
+constexpr int kAttnThreads = HILS_DECODE_THREADS;
+#ifndef HILS_DECODE_MINB
+#define HILS_DECODE_MINB 3
+#endif
+constexpr int kDimParts = kAttnThreads / 64;  // a key's dot product split over this many threads
+#ifndef HILS_DECODE_STAGES
+#define HILS_DECODE_STAGES 2
+#endif
+constexpr int kStages = HILS_DECODE_STAGES;  // chunk buffers per CTA (kStages - 1 copies ahead)
+
+template <typename T, int D, int GB>
+struct DecAttnLayout {
+  static constexpr int kRow = D * (int)sizeof(T);        // bytes of one K or V row
+  static constexpr int kBoxes = kRow / 128;              // 128-byte column boxes of K
+  static constexpr int kKBuf = kC * kRow;                // one chunk's K tiles [kBoxes][64][128]
+  // buffers: kStages, or as many as fit (fp32 rows are twice as long)
+  static constexpr int kFit = (227 * 1024 - 16 * 1024) / (2 * kKBuf);
+  static constexpr int kNS = kStages < kFit ? kStages : (kFit < 2 ? 2 : kFit);
+  static constexpr int ks = 0;                           // K tiles [kNS][kKBuf]
+  static constexpr int vs = ks + kNS * kKBuf;            // V slabs [kNS][64][kRow]
+  static constexpr int qs = vs + kNS * kC * kRow;        // queries [GB][D] fp32, scaled
+  static constexpr int xs = qs + GB * D * 4;             // partial logits [kDimParts][GB][64]
+  static constexpr int ps = xs + kDimParts * GB * kC * 4;  // probabilities [64][GB]
+  static constexpr int st = ps + kC * GB * 4;            // per head m, l, fusion logit, -
+  static constexpr int bars = st + GB * 16;              // kNS mbarriers
+  static constexpr int misc = bars + kNS * 8;            // abort flag
+  // the CTA's union entries, read once: chunk, head mask, first K row (-1:
+  // page outside the pool), element offset of the K / V slab, logits [GB]
+  static constexpr int ent_c = misc + 16;
+  static constexpr int ent_m = ent_c + kChunksPerCta * 4;
+  static constexpr int ent_y = ent_m + kChunksPerCta * 4;
+  static constexpr int ent_off = ent_y + kChunksPerCta * 4;
+  static constexpr int ent_l = ent_off + kChunksPerCta * 8;
+  static constexpr int total = ent_l + kChunksPerCta * GB * 4;
+  static_assert(kKBuf % 1024 == 0, "swizzled tiles are 1024-byte aligned");
+  static_assert(total <= 227 * 1024, "shared memory");
+  // the key-slice sums at the end reuse the K tiles
+  static_assert((kAttnThreads / (D / 2)) * GB * D * 4 <= kNS * kKBuf, "reduction area");
+};
+
+template <typename T, int D, int GB>
+__global__ void __launch_bounds__(kAttnThreads, HILS_DECODE_MINB) decode_attn_kernel(
+    const __grid_constant__ CUtensorMap tm_k, DecodeSpec ds, const T *__restrict__ q,
+    const T *__restrict__ kc, const T *__restrict__ vc, const PagedKV pg, const int32_t *__restrict__ u_c,
+    const uint32_t *__restrict__ u_mask, const float *__restrict__ u_logit,
+    const int32_t *__restrict__ u_count, float *__restrict__ part, uint32_t *__restrict__ err) {
+  using Lay = DecAttnLayout<T, D, GB>;
+  constexpr int NS = Lay::kNS;  // chunk buffers: NS - 1 copies in flight ahead
+  // a name of its own: this kernel asks the dynamic window for 1024-byte alignment
+  extern __shared__ __align__(1024) unsigned char smem_at[];
+  unsigned char *smem = smem_at;
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) report(err, DEV_BAD_INDEX);
+    return;
+  }
+  float *qs = reinterpret_cast<float *>(smem + Lay::qs);
+  float *xs = reinterpret_cast<float *>(smem + Lay::xs);
+  float *ps = reinterpret_cast<float *>(smem + Lay::ps);
+  float *st = reinterpret_cast<float *>(smem + Lay::st);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::bars);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::misc);
 
   const int G = ds.Hq / ds.Hkv;
   const int qi = blockIdx.x, bk = blockIdx.y;
@@ -685,212 +753,267 @@ __global__ void __launch_bounds__(256) decode_attn_kernel(DecodeSpec ds, const T
   const int t = ds.N - 1, own = ds.own;
 
   if (tid == 0) {
-    abort_flag = 0;
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    *abort_flag = 0;
+    for (int st2 = 0; st2 < NS; ++st2) mbar_init(&bars[st2], 1);
     fence_mbar_init();
+    prefetch_tmap(&tm_k);
   }
-  for (int i = tid; i < G * D; i += blockDim.x) {
+  for (int i = tid; i < GB * D; i += kAttnThreads) {
     const int g = i / D, e = i % D;
-    qs[i] = to_f(q[((size_t)b * ds.Hq + hkv * G + g) * D + e]) * ds.scale;
+    qs[i] = g < G ? to_f(q[((size_t)b * ds.Hq + hkv * G + g) * D + e]) * ds.scale : 0.0f;
   }
-  __syncthreads();
-  auto issue = [&](int i, int buf) {
-    const int c = u_c[(size_t)bk * cap + i];
-    const int rows = min(kC, ds.N - c * kC);
-    const uint32_t bytes = (uint32_t)rows * D * sizeof(T);
+  for (int i = tid; i < kC * GB; i += kAttnThreads) ps[i] = 0.0f;  // heads >= G stay 0
+  int *ent_c = reinterpret_cast<int *>(smem + Lay::ent_c);
+  uint32_t *ent_m = reinterpret_cast<uint32_t *>(smem + Lay::ent_m);
+  int *ent_y = reinterpret_cast<int *>(smem + Lay::ent_y);
+  size_t *ent_off = reinterpret_cast<size_t *>(smem + Lay::ent_off);
+  float *ent_l = reinterpret_cast<float *>(smem + Lay::ent_l);
+  if (tid < i1 - i0) {
+    const size_t ue = (size_t)bk * cap + i0 + tid;
+    const int c = u_c[ue];
     size_t off = (kvbase + (size_t)c * kC) * D;  // element offset of the chunk's [rows][D] slab
+    int y = (int)(kvbase + (size_t)c * kC);       // its first row in the K tensor map
     if (pg.table) {
       // paged: the chunk is page table[b][c], its KV head hkv at [page][hkv][C][D]
       const long long page = pg.table[(size_t)b * pg.max_pages + c];
-      if (page < 0 || page >= pg.num_pages) {
-        // no copy for an entry outside the pool: complete the phase without
-        // bytes (the chunk's logits are then unspecified) and report it
-        report(err, DEV_BAD_INDEX);
-        mbar_expect_tx(&bars[buf], 0);
-        return;
-      }
-      off = ((size_t)page * ds.Hkv + hkv) * kC * D;
+      const bool in_pool = page >= 0 && page < pg.num_pages;
+      off = in_pool ? ((size_t)page * ds.Hkv + hkv) * kC * D : 0;
+      y = in_pool ? (int)(((size_t)page * ds.Hkv + hkv) * kC) : -1;
     }
-    mbar_expect_tx(&bars[buf], 2 * bytes);
-    bulk_g2s(ks + buf * kC * D, kc + off, bytes, &bars[buf]);
-    bulk_g2s(vs + buf * kC * D, vc + off, bytes, &bars[buf]);
+    ent_c[tid] = c;
+    ent_m[tid] = u_mask[ue];
+    ent_y[tid] = y;
+    ent_off[tid] = off;
+    for (int g = 0; g < G; ++g) ent_l[tid * GB + g] = u_logit[ue * G + g];
+  }
+  __syncthreads();
+  // the copies of union entry i into buffer buf (thread 0): K as kBoxes
+  // swizzled [64 rows][128 bytes] tiles (a partial last chunk reads rows
+  // past the cache's end, never used), V as one slab of its valid rows
+  auto issue = [&](int i, int buf) {
+    const int li = i - i0;
+    const int rows = min(kC, ds.N - ent_c[li] * kC);
+    const int y = ent_y[li];
+    if (y < 0) {
+      // no copy for a page outside the pool: complete the phase without
+      // bytes (the chunk's logits are then unspecified) and report it
+      report(err, DEV_BAD_INDEX);
+      mbar_expect_tx(&bars[buf], 0);
+      return;
+    }
+    const size_t off = ent_off[li];
+    mbar_expect_tx(&bars[buf], (uint32_t)(kC + rows) * Lay::kRow);
+    unsigned char *kd = smem + Lay::ks + buf * Lay::kKBuf;
+#pragma unroll
+    for (int bx = 0; bx < Lay::kBoxes; ++bx)
+      tma_load_2d(kd + bx * kC * 128, &tm_k, &bars[buf], bx * (128 / (int)sizeof(T)), y);
+    bulk_g2s(smem + Lay::vs + buf * kC * Lay::kRow, vc + off, (uint32_t)rows * Lay::kRow,
+             &bars[buf]);
   };
-  if (tid == 0 && i0 < i1) issue(i0, 0);
+  // the first NS - 1 entries in flight before the loop
+  if (tid == 0)
+    for (int i = i0; i < min(i1, i0 + NS - 1); ++i) issue(i, (i - i0) % NS);
 
-  // running (max M, sum L, acc) per head: thread (g, e-pair) owns 2 columns of acc
-  const int e2n = D / 2;
-  float acc[2 * ((kMaxG * (D / 2) + 255) / 256)];
-  constexpr int kAccSlots = (kMaxG * (D / 2) + 255) / 256;
+  constexpr int NP = D / 2;                  // column pairs
+  constexpr int KS = kAttnThreads / NP;      // key slices of the P V pass
+  constexpr int KPS = kC / KS;               // keys per slice
+  constexpr int GP = GB >= 2 ? GB / 2 : 1;   // head pairs
+  const int pcol = tid % NP, ksl = tid / NP;
+  // acc for columns 2 pcol (a) and 2 pcol + 1 (b), heads (2 gp, 2 gp + 1) per pair
+  float2 acc_a[GP], acc_b[GP];
 #pragma unroll
-  for (int s = 0; s < 2 * kAccSlots; ++s) acc[s] = 0.0f;
-  float Mr[kMaxG], Lr[kMaxG];
+  for (int gp = 0; gp < GP; ++gp) acc_a[gp] = acc_b[gp] = make_float2(0.0f, 0.0f);
+  float Mr[GB], Lr[GB];
 #pragma unroll
-  for (int g = 0; g < kMaxG; ++g) { Mr[g] = -INFINITY; Lr[g] = 0.0f; }
+  for (int g = 0; g < GB; ++g) { Mr[g] = -INFINITY; Lr[g] = 0.0f; }
 
   bool ok = true;
   for (int i = i0; i < i1; ++i) {
-    const int buf = (i - i0) & 1;
-    if (tid == 0 && i + 1 < i1) issue(i + 1, buf ^ 1);
-    ok = __syncthreads_and(wait_bar(&bars[buf], ((i - i0) >> 1) & 1, &abort_flag));
+    const int buf = (i - i0) % NS;
+    // entry i + NS - 1 into the buffer entry i - 1 used (released by
+    // the end-of-iteration barrier)
+    if (tid == 0 && i + NS - 1 < i1) issue(i + NS - 1, (i + NS - 1 - i0) % NS);
+    ok = __syncthreads_and(wait_bar(&bars[buf], ((i - i0) / NS) & 1, abort_flag));
     if (!ok) {
-      // drain: a copy issued for the next chunk must land before the CTA exits
-      if (tid == 0 && i + 1 < i1) mbar_wait_bounded(&bars[buf ^ 1], ((i + 1 - i0) >> 1) & 1);
+      // drain: every copy issued must land before the CTA exits
+      if (tid == 0)
+        for (int k2 = i; k2 < min(i1, i + NS); ++k2)
+          mbar_wait_bounded(&bars[(k2 - i0) % NS], ((k2 - i0) / NS) & 1);
       break;
     }
-    const int c = u_c[(size_t)bk * cap + i];
-    const uint32_t mask = u_mask[(size_t)bk * cap + i];
+    const int c = ent_c[i - i0];
+    const uint32_t mask = ent_m[i - i0];
     const int jmax = (c == own) ? (t - c * kC) : (kC - 1);
-    const T *kt = ks + buf * kC * D;
-    const T *vt = vs + buf * kC * D;
-    // logits x[g][j] = scale * <q_g, k_j>.  A warp takes one head and 32
-    // keys; each lane holds a D/32 slice of the head's query in registers and
-    // reads the same slice of each key row (a warp reads whole rows, no bank
-    // conflicts), and a reduce-scatter butterfly (31 shuffles) leaves lane l
-    // with the full logit of key l.
-    for (int job = warp; job < 2 * G; job += blockDim.x / 32) {
-      const int g = job >> 1, j0 = (job & 1) * 32;
-      if (!((mask >> g) & 1u)) {
-        xs[g * kC + j0 + lane] = -INFINITY;
-        continue;
-      }
-      constexpr int kPer = D / 32;  // query / key elements per lane
-      float qv[kPer];
+    // ---- logits: partial dot products of key j with every head over part h of the dimension
+    {
+      const int j = tid & (kC - 1), h = tid >> 6;      // key, part of the head dimension
+      constexpr int kDP = D / kDimParts;                 // dimensions per part
+      const unsigned char *kr = smem + Lay::ks + buf * Lay::kKBuf + j * 128;
+      const float *qh = qs + h * kDP;
+      constexpr int kE = 16 / (int)sizeof(T);            // elements per 16-byte read
+      constexpr int kSteps = kDP / kE;
+      float2 a2[GB];
 #pragma unroll
-      for (int u = 0; u < kPer; ++u) qv[u] = qs[g * D + lane * kPer + u];
-      float v[32];
+      for (int g = 0; g < GB; ++g) a2[g] = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
-        const T *kr = kt + (j0 + jj) * D + lane * kPer;
-        float f[kPer];
+      for (int s2 = 0; s2 < kSteps; ++s2) {
+        const int cabs = h * kSteps + s2;  // 16-byte chunk of the row: box cabs / 8, column cabs % 8
+        const uint4 w = *reinterpret_cast<const uint4 *>(
+            kr + (cabs >> 3) * (kC * 128) + (((cabs & 7) ^ (j & 7)) << 4));
+        float f[kE];
         if constexpr (sizeof(T) == 2) {
-          if constexpr (kPer == 4) {
-            const uint2 w = *reinterpret_cast<const uint2 *>(kr);
-            f[0] = __uint_as_float(w.x << 16);
-            f[1] = __uint_as_float(w.x & 0xFFFF0000u);
-            f[2] = __uint_as_float(w.y << 16);
-            f[3] = __uint_as_float(w.y & 0xFFFF0000u);
-          } else {
-            const uint32_t w = *reinterpret_cast<const uint32_t *>(kr);
-            f[0] = __uint_as_float(w << 16);
-            f[1] = __uint_as_float(w & 0xFFFF0000u);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            f[2 * u] = __uint_as_float(ww[u] << 16);
+            f[2 * u + 1] = __uint_as_float(ww[u] & 0xFFFF0000u);
           }
         } else {
-#pragma unroll
-          for (int u = 0; u < kPer; ++u) f[u] = to_f(kr[u]);
+          f[0] = __uint_as_float(w.x);
+          f[1] = __uint_as_float(w.y);
+          f[2] = __uint_as_float(w.z);
+          f[3] = __uint_as_float(w.w);
         }
-        float a = 0.0f;
 #pragma unroll
-        for (int u = 0; u < kPer; ++u) a = fmaf(f[u], qv[u], a);
-        v[jj] = a;
-      }
+        for (int g = 0; g < GB; ++g) {
 #pragma unroll
-      for (int sft = 16; sft >= 1; sft >>= 1) {
-        const bool upper = (lane & sft) != 0;
-#pragma unroll
-        for (int i = 0; i < sft; ++i) {
-          const float send = upper ? v[i] : v[i + sft];
-          const float keep = upper ? v[i + sft] : v[i];
-          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
+          for (int u4 = 0; u4 < kE / 4; ++u4) {
+            const float4 qq = *reinterpret_cast<const float4 *>(qh + g * D + s2 * kE + 4 * u4);
+            a2[g] = __ffma2_rn(make_float2(f[4 * u4], f[4 * u4 + 1]), make_float2(qq.x, qq.y), a2[g]);
+            a2[g] = __ffma2_rn(make_float2(f[4 * u4 + 2], f[4 * u4 + 3]), make_float2(qq.z, qq.w), a2[g]);
+          }
         }
       }
-      const int j = j0 + lane;
-      xs[g * kC + j] = j <= jmax ? v[0] : -INFINITY;
+      float *xh = xs + h * GB * kC;
+#pragma unroll
+      for (int g = 0; g < GB; ++g) xh[g * kC + j] = a2[g].x + a2[g].y;
     }
     __syncthreads();
-    // per head: m, l over the chunk; probabilities e_j = exp(x_j - m)
-    for (int g = warp; g < G; g += blockDim.x / 32) {
-      const float a0 = xs[g * kC + lane], a1 = xs[g * kC + lane + 32];
-      float m = fmaxf(a0, a1);
+    // ---- per head: chunk maximum and sum, probabilities e_j = exp(x_j - m)
+    for (int g = warp; g < G; g += kAttnThreads / 32) {
+      if (!((mask >> g) & 1u)) {
+        ps[lane * GB + g] = 0.0f;
+        ps[(lane + 32) * GB + g] = 0.0f;
+        continue;
+      }
+      float x0 = 0.0f, x1 = 0.0f;
+#pragma unroll
+      for (int h = 0; h < kDimParts; ++h) {
+        x0 += xs[(h * GB + g) * kC + lane];
+        x1 += xs[(h * GB + g) * kC + lane + 32];
+      }
+      x0 = lane <= jmax ? x0 : -INFINITY;
+      x1 = lane + 32 <= jmax ? x1 : -INFINITY;
+      float m = fmaxf(x0, x1);  // finite: key 0 is always in the chunk
       for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      const float e0 = (m > -INFINITY) ? __expf(a0 - m) : 0.0f;
-      const float e1 = (m > -INFINITY) ? __expf(a1 - m) : 0.0f;
+      const float e0 = __expf(x0 - m), e1 = __expf(x1 - m);
       float l = e0 + e1;
       for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-      xs[g * kC + lane] = e0;
-      xs[g * kC + lane + 32] = e1;
+      ps[lane * GB + g] = e0;
+      ps[(lane + 32) * GB + g] = e1;
       if (lane == 0) {
         st[g * 4 + 0] = m;
         st[g * 4 + 1] = l;
         // the chunk's fusion logit: its landmark logit, or for the own chunk
         // the log-sum-exp of its causal token logits
-        st[g * 4 + 2] = (c == own) ? m + __logf(l) : u_logit[((size_t)bk * cap + i) * G + g];
+        st[g * 4 + 2] = (c == own) ? m + __logf(l) : ent_l[(i - i0) * GB + g];
       }
     }
     __syncthreads();
-    // acc_g = acc_g * exp(M_old - M_new) + exp(logit - M_new) / l * sum_j e_j v_j
+    // ---- P V over this thread's key slice, every head
+    {
+      const unsigned char *vb = smem + Lay::vs + buf * kC * Lay::kRow + pcol * 2 * (int)sizeof(T);
+      float2 oa[GP], ob[GP];
 #pragma unroll
-    for (int s = 0; s < kAccSlots; ++s) {
-      const int pr = tid + s * 256;
-      const int g = pr / e2n, e2 = pr % e2n;
-      if (g < G && ((mask >> g) & 1u)) {
-        // even and odd keys in two packed (column pair) partial sums: short
-        // FMA chains, one fp32x2 FMA per key
-        auto vpair = [&](int j) {
-          if constexpr (sizeof(T) == 2) {
-            const uint32_t w = *reinterpret_cast<const uint32_t *>(vt + j * D + 2 * e2);
-            return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-          } else {
-            return *reinterpret_cast<const float2 *>(vt + j * D + 2 * e2);
-          }
-        };
-        float2 oe = make_float2(0.0f, 0.0f), oo = make_float2(0.0f, 0.0f);
-        int j = 0;
+      for (int gp = 0; gp < GP; ++gp) oa[gp] = ob[gp] = make_float2(0.0f, 0.0f);
+      const int jlo = ksl * KPS, jend = min(jlo + KPS, jmax + 1);
 #pragma unroll 4
-        for (; j + 1 <= jmax; j += 2) {
-          const float2 pp = *reinterpret_cast<const float2 *>(xs + g * kC + j);
-          oe = __ffma2_rn(make_float2(pp.x, pp.x), vpair(j), oe);
-          oo = __ffma2_rn(make_float2(pp.y, pp.y), vpair(j + 1), oo);
+      for (int j = jlo; j < jend; ++j) {
+        float v0, v1;
+        if constexpr (sizeof(T) == 2) {
+          const uint32_t w = *reinterpret_cast<const uint32_t *>(vb + j * Lay::kRow);
+          v0 = __uint_as_float(w << 16);
+          v1 = __uint_as_float(w & 0xFFFF0000u);
+        } else {
+          const float2 w = *reinterpret_cast<const float2 *>(vb + j * Lay::kRow);
+          v0 = w.x;
+          v1 = w.y;
         }
-        if (j <= jmax) {
-          const float pj = xs[g * kC + j];
-          oe = __ffma2_rn(make_float2(pj, pj), vpair(j), oe);
-        }
-        const float o0 = oe.x + oo.x, o1 = oe.y + oo.y;
-        const float lg = st[g * 4 + 2], l = st[g * 4 + 1];
-        float mo = 0.0f, ln = 0.0f;
+        const float *pj = ps + j * GB;
+        if constexpr (GB == 1) {
+          oa[0].x = fmaf(pj[0], v0, oa[0].x);
+          ob[0].x = fmaf(pj[0], v1, ob[0].x);
+        } else {
 #pragma unroll
-        for (int gg = 0; gg < kMaxG; ++gg)
-          if (gg == g) { mo = Mr[gg]; ln = Lr[gg]; }
-        const float mn = fmaxf(mo, lg);
-        const float so = __expf(mo - mn), sn = __expf(lg - mn);
-        acc[2 * s] = acc[2 * s] * so + sn * o0 / l;
-        acc[2 * s + 1] = acc[2 * s + 1] * so + sn * o1 / l;
+          for (int gp = 0; gp < GP; ++gp) {
+            const float2 pp = *reinterpret_cast<const float2 *>(pj + 2 * gp);
+            oa[gp] = __ffma2_rn(pp, make_float2(v0, v0), oa[gp]);
+            ob[gp] = __ffma2_rn(pp, make_float2(v1, v1), ob[gp]);
+          }
+        }
+      }
+      // acc_g = acc_g exp(M_old - M_new) + exp(logit - M_new) / l * o_g
+      float so[GB], sn[GB];
+#pragma unroll
+      for (int g = 0; g < GB; ++g) {
+        so[g] = 1.0f;
+        sn[g] = 0.0f;
+        if (g < G && ((mask >> g) & 1u)) {
+          const float lg = st[g * 4 + 2], l = st[g * 4 + 1];
+          const float mn = fmaxf(Mr[g], lg);
+          so[g] = __expf(Mr[g] - mn);
+          const float e = __expf(lg - mn);
+          sn[g] = e / l;
+          Lr[g] = Lr[g] * so[g] + e;
+          Mr[g] = mn;
+        }
+      }
+      if constexpr (GB == 1) {
+        acc_a[0].x = acc_a[0].x * so[0] + sn[0] * oa[0].x;
+        acc_b[0].x = acc_b[0].x * so[0] + sn[0] * ob[0].x;
+      } else {
+#pragma unroll
+        for (int gp = 0; gp < GP; ++gp) {
+          const float2 s_o = make_float2(so[2 * gp], so[2 * gp + 1]);
+          const float2 s_n = make_float2(sn[2 * gp], sn[2 * gp + 1]);
+          acc_a[gp] = __ffma2_rn(acc_a[gp], s_o, __fmul2_rn(s_n, oa[gp]));
+          acc_b[gp] = __ffma2_rn(acc_b[gp], s_o, __fmul2_rn(s_n, ob[gp]));
+        }
       }
     }
-    // running max / sum per head (every thread keeps all heads' copies)
-#pragma unroll
-    for (int g = 0; g < kMaxG; ++g) {
-      if (g < G && ((mask >> g) & 1u)) {
-        const float lg = st[g * 4 + 2];
-        const float mn = fmaxf(Mr[g], lg);
-        Lr[g] = Lr[g] * __expf(Mr[g] - mn) + __expf(lg - mn);
-        Mr[g] = mn;
-      }
-    }
-    __syncthreads();  // the buffer and xs are reused
+    __syncthreads();  // the buffer, xs, ps and st are reused
   }
-  // partial record per (bk, qi, g): [M, L, acc[D]]
+  __syncthreads();  // every copy has landed (also on the timeout path)
+  // ---- sum the key slices; partial record per (bk, qi, g): [M, L, acc[D]]
+  float *red = reinterpret_cast<float *>(smem + Lay::ks);  // [KS][GB][D]
+#pragma unroll
+  for (int gp = 0; gp < GP; ++gp) {
+#pragma unroll
+    for (int u = 0; u < (GB == 1 ? 1 : 2); ++u) {
+      const int g = 2 * gp + u;
+      const float a = u ? acc_a[gp].y : acc_a[gp].x, bb = u ? acc_b[gp].y : acc_b[gp].x;
+      *reinterpret_cast<float2 *>(red + (ksl * GB + g) * D + 2 * pcol) = make_float2(a, bb);
+    }
+  }
+  __syncthreads();
   const size_t rec = 2 + D;
+  for (int i = tid; i < G * D; i += kAttnThreads) {
+    const int g = i / D, e = i % D;
+    float sum = 0.0f;
 #pragma unroll
-  for (int s = 0; s < kAccSlots; ++s) {
-    const int pr = tid + s * 256;
-    const int g = pr / e2n, e2 = pr % e2n;
-    if (g < G) {
-      float *r = part + (((size_t)bk * ds.Q + qi) * G + g) * rec;
-      r[2 + 2 * e2] = acc[2 * s];
-      r[3 + 2 * e2] = acc[2 * s + 1];
-      if (e2 == 0) {
-        float mo = 0.0f, lo = 0.0f;
-#pragma unroll
-        for (int gg = 0; gg < kMaxG; ++gg)
-          if (gg == g) { mo = Mr[gg]; lo = Lr[gg]; }
-        r[0] = mo;
-        r[1] = lo;
-      }
-    }
+    for (int k2 = 0; k2 < KS; ++k2) sum += red[(k2 * GB + g) * D + e];
+    part[(((size_t)bk * ds.Q + qi) * G + g) * rec + 2 + e] = sum;
   }
-  if (tid == 0 && abort_flag) report(err, DEV_TIMEOUT);
+  if (tid < G) {
+    float mo = 0.0f, lo = 0.0f;
+#pragma unroll
+    for (int g = 0; g < GB; ++g)
+      if (g == tid) { mo = Mr[g]; lo = Lr[g]; }
+    float *r = part + (((size_t)bk * ds.Q + qi) * G + tid) * rec;
+    r[0] = mo;
+    r[1] = lo;
+  }
+  if (tid == 0 && *abort_flag) report(err, DEV_TIMEOUT);
 }
 
 // ---------------------------------------------------------------------------
@@ -978,7 +1101,6 @@ static cudaError_t decode_run(const DecodeSpec &ds, bool bf16, const void *q, co
   float *part = reinterpret_cast<float *>(
       take(std::max(BK * G * (size_t)ds.n_c, BK * ds.Q * G * (size_t)(2 + ds.d)) * 4));
   float *scores = part;  // landmark logits, consumed before the partials are written
-  const size_t esz = bf16 ? 2 : 4;
   cudaError_t e;
 
   if (ds.P > 0 && bf16 && G <= kTcN) {
@@ -1023,15 +1145,30 @@ static cudaError_t decode_run(const DecodeSpec &ds, bool bf16, const void *q, co
     ++*launches;
   }
   {
-    const size_t smem = 4 * (size_t)kC * ds.d * esz + kMaxG * ds.d * 4 + kMaxG * kC * 4 + kMaxG * 16;
-#define HILS_ATTN(T, DD)                                                                        \
+    // K through a 2-D tensor map: the dense cache [B*Hkv*N rows][d], or the
+    // page pool [num_pages*Hkv*64 rows][d]
+    const uint64_t krows = pages.table ? (uint64_t)pages.num_pages * ds.Hkv * kC : (uint64_t)BK * ds.N;
+    if (krows >= (1ull << 31)) return cudaErrorInvalidValue;  // tensor-map rows are int32
+    CUtensorMap tk;
+    if ((e = bf16 ? make_tmap_bf16(&tk, k, krows, ds.d, kC) : make_tmap_f32(&tk, k, krows, ds.d, kC)) != cudaSuccess)
+      return e;
+#define HILS_ATTN(T, DD, GG)                                                                    \
   do {                                                                                          \
-    auto kern = decode_attn_kernel<T, DD>;                                                      \
+    auto kern = decode_attn_kernel<T, DD, GG>;                                                  \
+    const size_t smem = DecAttnLayout<T, DD, GG>::total;                                        \
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e; \
-    kern<<<dim3(ds.Q, (unsigned)BK), 256, smem, st>>>(ds, (const T *)q, (const T *)k, (const T *)v, pages, u_c, u_mask, u_logit, u_count, part, err); \
+    kern<<<dim3(ds.Q, (unsigned)BK), kAttnThreads, smem, st>>>(tk, ds, (const T *)q, (const T *)k, (const T *)v, pages, u_c, u_mask, u_logit, u_count, part, err); \
   } while (0)
-    if (bf16) { if (ds.d == 64) HILS_ATTN(__nv_bfloat16, 64); else HILS_ATTN(__nv_bfloat16, 128); }
-    else { if (ds.d == 64) HILS_ATTN(float, 64); else HILS_ATTN(float, 128); }
+#define HILS_ATTN_G(T, DD)                                                                      \
+  do {                                                                                          \
+    if (G <= 1) HILS_ATTN(T, DD, 1);                                                            \
+    else if (G <= 2) HILS_ATTN(T, DD, 2);                                                       \
+    else if (G <= 4) HILS_ATTN(T, DD, 4);                                                       \
+    else HILS_ATTN(T, DD, 8);                                                                   \
+  } while (0)
+    if (bf16) { if (ds.d == 64) HILS_ATTN_G(__nv_bfloat16, 64); else HILS_ATTN_G(__nv_bfloat16, 128); }
+    else { if (ds.d == 64) HILS_ATTN_G(float, 64); else HILS_ATTN_G(float, 128); }
+#undef HILS_ATTN_G
 #undef HILS_ATTN
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++*launches;

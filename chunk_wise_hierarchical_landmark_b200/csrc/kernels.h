@@ -51,6 +51,9 @@ namespace hils {
 // [box_rows x 64 elements], 128-byte swizzle (attn_sm100.cu)
 cudaError_t make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
                            uint32_t box_rows);
+// the same over an fp32 array: box [box_rows x 32 elements] (128 bytes)
+cudaError_t make_tmap_f32(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                          uint32_t box_rows);
 
 // Decode step (decode.cu).  One query per head at position N-1.
 struct DecodeSpec {
