@@ -310,7 +310,8 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
                                                           float *__restrict__ lse_lmk,
                                                           int staged) {
   extern __shared__ __align__(16) float sc_s[];  // the head's logits when staged
-  __shared__ uint32_t hist_w[8 * 256];  // per-warp digit histograms
+  // per-warp digit histograms; also read as 64-bit candidate keys, hence the alignment
+  __shared__ __align__(16) uint32_t hist_w[8 * 256];
   __shared__ uint32_t hist[256];
   __shared__ int wsum[8];
   __shared__ float red[8];
