@@ -97,6 +97,10 @@ struct SelLayout {
   static constexpr int seeds = misc + 32;                     // [kMaxK] int seed chunk ids
   static constexpr int total = seeds + kMaxK * 4;
   static_assert(bias % 1024 == 0, "swizzled tiles are 1024-byte aligned");
+  // the epilogue's per-warp staging blocks [32][64 + 4] words (4 owner warps)
+  // in the landmark ring and the masking tile that follows it, where they fit
+  // (d = 128; at d = 64 the rows are written directly)
+  static constexpr bool kStagedOut = 4 * 32 * (kMaxK + 4) * 4 <= heap - l0;
   // TMEM columns: Q [0, D/2) as bf16 pairs, the masking A operand [64, 72),
   // score buffers [128, 192) and [192, 256)
   static constexpr uint32_t kQCol = 0, kBiasCol = 64, kSCol = 128, kTmemCols = 256;
@@ -240,6 +244,77 @@ __device__ __forceinline__ void write_in_order(const uint64_t *slots, int cnt, i
 // below 2^25 (L < 2^31, C = 64), so (id << 6 | slot) fits a 32-bit word; a
 // bitonic network of N/2 log N (log N + 1) / 2 min/max pairs sorts N words in
 // registers without branches (words past K sort last).
+// The warp's 32 rows (K = N = 32 or 64, every row searched) written through
+// a per-warp staging block [32][N + 4] words in shared memory: each lane
+// sorts its row's (chunk << 6 | slot) words as write_sorted does and stores
+// them as a row of the block (a row stride of 4 mod 32 words keeps the
+// 16-byte accesses free of bank conflicts); the warp copies the chunk ids out
+// with coalesced 16-byte stores (two 256-byte rows per instruction for
+// N = 64); each lane then replaces its row's words by their logits, read from
+// its slots, and the warp copies those out the same way.  rows_valid: the
+// warp's rows below L.
+template <int N, bool kIds>
+__device__ __forceinline__ void copy_block_out(const uint32_t *stage, int lane,
+                                               uint32_t *__restrict__ dst, int rows_valid) {
+  constexpr int S = N + 4, P = N / 4;  // staging stride (words), 16-byte pieces per row
+#pragma unroll
+  for (int u = 0; u < P; ++u) {
+    const int pc = u * 32 + lane, row = pc / P, c = pc % P;
+    if (row < rows_valid) {
+      uint4 x = *reinterpret_cast<const uint4 *>(stage + row * S + 4 * c);
+      if (kIds) x = make_uint4(x.x >> 6, x.y >> 6, x.z >> 6, x.w >> 6);
+      *reinterpret_cast<uint4 *>(dst + (size_t)row * N + 4 * c) = x;
+    }
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void write_sorted_staged(const uint64_t *slots, uint32_t *stage,
+                                                    int lane, int32_t *__restrict__ sel_w,
+                                                    float *__restrict__ w_w, int rows_valid) {
+  constexpr int S = N + 4;
+  uint32_t *mine = stage + lane * S;
+  {
+    uint32_t v[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      const uint32_t lo = reinterpret_cast<const uint32_t *>(slots + i * kRows)[0];
+      v[i] = ((0xFFFFFFFFu - lo) << 6) | (uint32_t)i;
+    }
+#pragma unroll
+    for (int size = 2; size <= N; size <<= 1)
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1)
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+          const int j = i ^ stride;
+          if (j > i) {
+            const uint32_t x = v[i], y = v[j];
+            const bool up = (i & size) == 0;
+            v[i] = up ? min(x, y) : max(x, y);
+            v[j] = up ? max(x, y) : min(x, y);
+          }
+        }
+#pragma unroll
+    for (int i = 0; i < N; i += 4)
+      *reinterpret_cast<uint4 *>(mine + i) = make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+  }
+  __syncwarp();
+  copy_block_out<N, true>(stage, lane, reinterpret_cast<uint32_t *>(sel_w), rows_valid);
+  __syncwarp();
+#pragma unroll 4
+  for (int i = 0; i < N; i += 4) {
+    const uint4 x = *reinterpret_cast<const uint4 *>(mine + i);
+    *reinterpret_cast<uint4 *>(mine + i) =
+        make_uint4(__float_as_uint(key_score(slots[(x.x & 63u) * kRows])),
+                   __float_as_uint(key_score(slots[(x.y & 63u) * kRows])),
+                   __float_as_uint(key_score(slots[(x.z & 63u) * kRows])),
+                   __float_as_uint(key_score(slots[(x.w & 63u) * kRows])));
+  }
+  __syncwarp();
+  copy_block_out<N, false>(stage, lane, reinterpret_cast<uint32_t *>(w_w), rows_valid);
+}
+
 template <int N>
 __device__ __forceinline__ void write_sorted(const uint64_t *slots, int K,
                                              int32_t *__restrict__ srow,
@@ -395,6 +470,28 @@ __device__ __forceinline__ void hope_row_split(const unsigned char *tile, int r,
     tmem_st4(taddr + 4 * j, aw);
     tmem_st4(taddr + D / 4 + 4 * j, bw);
   }
+}
+
+// One row's selection in ascending chunk order (rows that kept every
+// candidate are already in order).
+__device__ __forceinline__ void write_row(const uint64_t *slots, int n_c, int cnt, int K,
+                                          int32_t *__restrict__ srow, float *__restrict__ wrow) {
+  if (n_c <= K)
+    write_in_order(slots, cnt, K, srow, wrow);
+  else if (K <= 16)
+    write_sorted<16>(slots, K, srow, wrow);
+  else if (K <= 32)
+    write_sorted<32>(slots, K, srow, wrow);
+  else
+    write_sorted<64>(slots, K, srow, wrow);
+}
+
+// The row's log-sum-exp from its two halves' (max, sum) in base 2.
+__device__ __forceinline__ float row_lse(float2 o, float m2, float l, int n_c) {
+  const float mm = fmaxf(m2, o.x);
+  const float ls = (m2 > -INFINITY ? l * ex2_approx(m2 - mm) : 0.0f) +
+                   (o.x > -INFINITY ? o.y * ex2_approx(o.x - mm) : 0.0f);
+  return n_c > 0 ? (mm + __log2f(ls)) * kLn2 : -INFINITY;
 }
 
 template <int D>
@@ -866,25 +963,34 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       __threadfence_block();
       // ---------------------------------------------------------- epilogue
-      if (__all_sync(0xffffffffu, ok) && valid) {
+      if constexpr (Lay::kStagedOut) {
+        // The warp's rows are 32 consecutive positions inside one chunk, so
+        // every valid lane has the candidate count of the warp's first row
+        // and the choice of the staged path is uniform over the warp (lanes
+        // past L take part but write nothing).  The staging blocks (K = 32
+        // or 64) sit in the landmark ring and the masking tile, idle once
+        // this warp has read its last score tile.
         const size_t row = (size_t)bh * L + t;
-        int32_t *srow = sel + row * K;
-        float *wrow = chunk_w + row * K;
-        // ascending chunk order (rows that kept every candidate are in order)
-        if (n_c <= K)
-          write_in_order(slots, cnt, K, srow, wrow);
-        else if (K <= 16)
-          write_sorted<16>(slots, K, srow, wrow);
-        else if (K <= 32)
-          write_sorted<32>(slots, K, srow, wrow);
-        else
-          write_sorted<64>(slots, K, srow, wrow);
-        if (want_lse) {
-          const float2 o = lsep_s[r];
-          const float mm = fmaxf(m2, o.x);
-          const float ls = (m2 > -INFINITY ? l * ex2_approx(m2 - mm) : 0.0f) +
-                           (o.x > -INFINITY ? o.y * ex2_approx(o.x - mm) : 0.0f);
-          lse_lmk[row] = n_c > 0 ? (mm + __log2f(ls)) * kLn2 : -INFINITY;
+        const int wrow0 = t0 + 32 * (warp & 3);  // the warp's first position
+        const int rows_valid = min(32, L - wrow0);
+        const int n_c_warp = min(wrow0 / C, nlmk);
+        if (__all_sync(0xffffffffu, ok) && rows_valid > 0 && n_c_warp > K && (K == 64 || K == 32)) {
+          uint32_t *stage = reinterpret_cast<uint32_t *>(smem + Lay::l0) + (warp & 3) * 32 * (K + 4);
+          const size_t r0 = (size_t)bh * L + wrow0;
+          if (K == 64)
+            write_sorted_staged<64>(slots, stage, lane, sel + r0 * K, chunk_w + r0 * K, rows_valid);
+          else
+            write_sorted_staged<32>(slots, stage, lane, sel + r0 * K, chunk_w + r0 * K, rows_valid);
+        } else if (__all_sync(0xffffffffu, ok) && valid) {
+          write_row(slots, n_c, cnt, K, sel + row * K, chunk_w + row * K);
+        }
+        if (__all_sync(0xffffffffu, ok) && valid && want_lse)
+          lse_lmk[row] = row_lse(lsep_s[r], m2, l, n_c);
+      } else {
+        if (__all_sync(0xffffffffu, ok) && valid) {
+          const size_t row = (size_t)bh * L + t;
+          write_row(slots, n_c, cnt, K, sel + row * K, chunk_w + row * K);
+          if (want_lse) lse_lmk[row] = row_lse(lsep_s[r], m2, l, n_c);
         }
       }
     }
