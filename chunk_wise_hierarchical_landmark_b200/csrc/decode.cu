@@ -49,6 +49,8 @@ using namespace sm100;
 constexpr int kGemvThreads = 128; // landmarks per scoring CTA
 constexpr int kChunksPerCta = 16; // union chunks per attention CTA
 constexpr int kMaxG = 8;         // query heads per KV head handled per CTA
+constexpr int kTkThreads = 512;  // top-k CTA (one head)
+constexpr int kTkWarps = kTkThreads / 32;
 constexpr int kC = 64;
 
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
@@ -303,18 +305,19 @@ __device__ __forceinline__ uint32_t score_bits(float s) {
 // order-preserving bits (four 8-bit digits, per-warp histograms); the kept
 // chunks are then written in ascending chunk order, the lowest ids among
 // scores equal to the k-th.
-__global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
+__global__ void __launch_bounds__(kTkThreads) decode_topk_kernel(DecodeSpec ds,
                                                           const float *__restrict__ scores,
                                                           int32_t *__restrict__ sel,
                                                           float *__restrict__ chunk_w,
                                                           float *__restrict__ lse_lmk,
                                                           int staged) {
   extern __shared__ __align__(16) float sc_s[];  // the head's logits when staged
-  // per-warp digit histograms; also read as 64-bit candidate keys, hence the alignment
+  // digit histograms (one per pair of warps); also read as 64-bit candidate
+  // keys, hence the alignment
   __shared__ __align__(16) uint32_t hist_w[8 * 256];
   __shared__ uint32_t hist[256];
-  __shared__ int wsum[8];
-  __shared__ float red[8];
+  __shared__ int wsum[kTkWarps];
+  __shared__ float red[kTkWarps];
   __shared__ uint32_t s_prefix, s_bin;
   __shared__ int s_need;
   const int h = blockIdx.x;  // b*Hq + hq
@@ -324,7 +327,7 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
   if (staged) {
     // one pass over HBM/L2 with every load in flight; the rest reads shared memory
 #pragma unroll 8
-    for (int i = tid; i < n; i += 256) sc_s[i] = sc[i];
+    for (int i = tid; i < n; i += kTkThreads) sc_s[i] = sc[i];
     __syncthreads();
     sc = sc_s;
   }
@@ -334,31 +337,31 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
   // log-sum-exp: block maximum, then the sum of exponentials against it
   float m = -INFINITY;
 #pragma unroll 8
-  for (int i = tid; i < n; i += 256) m = fmaxf(m, sc[i]);
+  for (int i = tid; i < n; i += kTkThreads) m = fmaxf(m, sc[i]);
   for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane == 0) red[warp] = m;
   __syncthreads();
   m = red[0];
 #pragma unroll
-  for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
+  for (int w = 1; w < kTkWarps; ++w) m = fmaxf(m, red[w]);
   __syncthreads();
   float l = 0.0f;
   if (n > 0) {
 #pragma unroll 8
-    for (int i = tid; i < n; i += 256) l += __expf(sc[i] - m);
+    for (int i = tid; i < n; i += kTkThreads) l += __expf(sc[i] - m);
   }
   for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
   if (lane == 0) red[warp] = l;
   __syncthreads();
   if (tid == 0 && lse_lmk) {
     float lt = 0.0f;
-    for (int w = 0; w < 8; ++w) lt += red[w];
+    for (int w = 0; w < kTkWarps; ++w) lt += red[w];
     lse_lmk[h] = n > 0 ? m + __logf(lt) : -INFINITY;
   }
 
   if (n <= K) {
     // every completed chunk is selected
-    for (int i = tid; i < K; i += 256) {
+    for (int i = tid; i < K; i += kTkThreads) {
       srow[i] = i < n ? i : -1;
       wrow[i] = i < n ? sc[i] : -INFINITY;
     }
@@ -378,38 +381,53 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
     __shared__ uint32_t tau_s;
     __shared__ uint32_t keep[256];  // one bit per chunk (n <= 8192)
     if (tid == 0) n_cand_s = 0;
-    keep[tid] = 0u;
-    if (tid < nb) {
-      // the block's 32 logits, visited in a lane-rotated order (no conflicts)
+    if (tid < 256) keep[tid] = 0u;
+    // block maxima: two threads per block, 16 logits each in a lane-rotated
+    // order (no bank conflicts), combined across the pair
+    // (whole warps take part, for the pair shuffles; act: the pair's block exists)
+    const int pair_warps_end = (2 * nb + 31) & ~31;
+    if (tid < pair_warps_end) {
+      const int bk = tid >> 1, hf = tid & 1;
+      const bool act = bk < nb;
       uint32_t m = 0u;
 #pragma unroll 8
-      for (int u = 0; u < 32; ++u) {
-        const int i = tid * 32 + ((u + tid) & 31);
-        if (i < n) m = max(m, score_bits(sc[i]));
+      for (int u = 0; u < 16; ++u) {
+        const int i = bk * 32 + hf * 16 + ((u + bk) & 15);
+        if (act && i < n) m = max(m, score_bits(sc[i]));
       }
-      bmax[tid] = m;
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      if (act && hf == 0) bmax[bk] = m;
     }
     __syncthreads();
-    if (tid < nb) {
-      // rank of this block's maximum (ties: lower block first)
-      const uint32_t v = bmax[tid];
+    if (tid < pair_warps_end) {
+      // rank of this block's maximum (ties: lower block first), the pair
+      // splitting the other blocks between them
+      const int bk = tid >> 1, hf = tid & 1;
+      const bool act = bk < nb;
+      const uint32_t v = act ? bmax[bk] : 0u;
       int rank = 0;
+      if (act) {
 #pragma unroll 8
-      for (int b2 = 0; b2 < nb; ++b2) {
-        const uint32_t x = bmax[b2];
-        rank += (x > v || (x == v && b2 < tid)) ? 1 : 0;
+        for (int b2 = hf; b2 < nb; b2 += 2) {
+          const uint32_t x = bmax[b2];
+          rank += (x > v || (x == v && b2 < bk)) ? 1 : 0;
+        }
       }
-      if (rank == K - 1) tau_s = v;
+      rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+      if (act && hf == 0 && rank == K - 1) tau_s = v;
     }
     __syncthreads();
     const uint32_t tau = tau_s;
-    for (int i0 = 0; i0 < n; i0 += 256) {
-      const int i = i0 + tid;
+    // candidates: only a block whose maximum reaches tau holds any; a warp
+    // per such block, one lane per logit
+    for (int b2 = warp; b2 < nb; b2 += kTkWarps) {
+      if (bmax[b2] < tau) continue;
+      const int i = b2 * 32 + lane;
       const uint32_t kb = i < n ? score_bits(sc[i]) : 0u;
       const bool in = i < n && kb >= tau;
       const uint32_t bal = __ballot_sync(0xffffffffu, in);
       int base = 0;
-      if (lane == 0 && bal) base = atomicAdd(&n_cand_s, __popc(bal));
+      if (lane == 0) base = atomicAdd(&n_cand_s, __popc(bal));
       base = __shfl_sync(0xffffffffu, base, 0);
       const int pos = base + __popc(bal & ((1u << lane) - 1u));
       if (in && pos < kCandCap) cand[pos] = ((uint64_t)kb << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)i);
@@ -418,7 +436,7 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
     const int m = n_cand_s;
     if (m <= kCandCap) {
       // exact rank of every candidate key; the k best are kept
-      for (int a = tid; a < m; a += 256) {
+      for (int a = tid; a < m; a += kTkThreads) {
         const uint64_t x = cand[a];
         int rank = 0;
 #pragma unroll 8
@@ -468,14 +486,14 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
   uint32_t last_bin = 0;  // keys equal to the final prefix
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    for (int i = tid; i < 8 * 256; i += 256) hist_w[i] = 0;
+    for (int i = tid; i < 8 * 256; i += kTkThreads) hist_w[i] = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += 256) {
+    for (int i = tid; i < n; i += kTkThreads) {
       const uint32_t k = score_bits(sc[i]);
-      if (pass == 0 || (k >> (shift + 8)) == prefix) atomicAdd(&hist_w[warp * 256 + ((k >> shift) & 255u)], 1u);
+      if (pass == 0 || (k >> (shift + 8)) == prefix) atomicAdd(&hist_w[(warp & 7) * 256 + ((k >> shift) & 255u)], 1u);
     }
     __syncthreads();
-    {
+    if (tid < 256) {
       uint32_t sum = 0;
 #pragma unroll
       for (int w = 0; w < 8; ++w) sum += hist_w[w * 256 + tid];
@@ -522,7 +540,7 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
   // per segment give every warp its output offset, then it writes in order.
   const uint32_t T = prefix;
   const bool all_eq = last_bin == (uint32_t)need;
-  const int seg = (n + 7) / 8;
+  const int seg = (n + kTkWarps - 1) / kTkWarps;
   const int lo = warp * seg, hi = min(n, lo + seg);
   auto key_at = [&](int i) { return score_bits(sc[i]); };
   int my_eq = 0;
@@ -535,7 +553,7 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
   __syncthreads();
   int eq_before = 0;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) eq_before += w < warp ? wsum[w] : 0;
+  for (int w = 0; w < kTkWarps; ++w) eq_before += w < warp ? wsum[w] : 0;
   __syncthreads();
   // takes per segment
   int my_take = 0;
@@ -556,7 +574,7 @@ __global__ void __launch_bounds__(256) decode_topk_kernel(DecodeSpec ds,
   __syncthreads();
   int base = 0;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) base += w < warp ? wsum[w] : 0;
+  for (int w = 0; w < kTkWarps; ++w) base += w < warp ? wsum[w] : 0;
   {
     int eq_run = eq_before;
     for (int i0 = lo; i0 < hi; i0 += 32) {
@@ -1134,7 +1152,7 @@ static cudaError_t decode_run(const DecodeSpec &ds, bool bf16, const void *q, co
     const size_t tsmem = (size_t)ds.n_c * sizeof(float);
     const int staged = tsmem <= 160 * 1024 ? 1 : 0;
     if (staged && (e = cudaFuncSetAttribute(decode_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem)) != cudaSuccess) return e;
-    decode_topk_kernel<<<(unsigned)(ds.B * ds.Hq), 256, staged ? tsmem : 0, st>>>(ds, scores, sel, w, lse_lmk, staged);
+    decode_topk_kernel<<<(unsigned)(ds.B * ds.Hq), kTkThreads, staged ? tsmem : 0, st>>>(ds, scores, sel, w, lse_lmk, staged);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   ++*launches;
