@@ -15,9 +15,11 @@
 //   dq_t  = scale (sum_cj dx_j k_j + sum_{c selected} ds_c lmk_c)
 //   dk_j += scale dx_j q_t,  dv_j += w_c p_cj dO_t,  dlmk_c += scale ds_c q_t
 // Three stages, all on the CUDA cores in fp32 (bf16 inputs widen exactly):
-//   bwd_rows_kernel   one warp per row: per-chunk softmax recomputed from q and
-//                     the chunk's keys, g_c, w_c, D, ds_c -> per-(row, slot)
-//                     records (lse_c, w_c, g_c, ds_c); then dq.
+//   bwd_rows_kernel   one warp per row, one pass over its chunks: per-chunk
+//                     softmax recomputed from q and the chunk's keys, g_c,
+//                     w_c, and dq with the D-dependent part factored out;
+//                     then D and the per-(row, slot) records (lse_c, w_c,
+//                     g_c, ds_c).
 //   transposed selection: per (b, kv head, chunk) the (row, slot) pairs that
 //                     select it (count, exclusive scan, fill; the order inside
 //                     a chunk's list follows the atomic fill).
@@ -172,7 +174,18 @@ __global__ void __launch_bounds__(kRowWarps * 32)
   const float *wrow = chunk_w + (size_t)row * K;
   float4 *rrow = rec + (size_t)row * (K + 1);
 
-  // pass 1: per attended chunk lse_c, w_c, g_c; D = sum w_c g_c
+  // One pass over the attended chunks.  w_c = exp(s_c - lse) is known up
+  // front, so dq splits into terms that need no D = sum_c w_c g_c and one
+  // that is D times a vector:
+  //   dq / scale = sum_c w_c (A_c - g_c B_c)              A_c = sum_j p_cj dP_cj k_j
+  //              + sum_sel w_c (g_c + dlse) lmk_c          B_c = sum_j p_cj k_j
+  //              + w_own (g_own + dlse) B_own
+  //              - D (sum_sel w_c lmk_c + w_own B_own)
+  // (the ds_c = w_c (g_c - D + dlse) terms and the own chunk's p ds_own term
+  // regrouped); ds_c goes into the records afterwards.
+  float acc[P], accd[P];
+#pragma unroll
+  for (int u = 0; u < P; ++u) acc[u] = accd[u] = 0.0f;
   float Dsum = 0.0f;
   for (int slot = 0; slot <= K; ++slot) {
     int c;
@@ -189,9 +202,9 @@ __global__ void __launch_bounds__(kRowWarps * 32)
       c = own;
     }
     const int nkeys = slot < K ? kC : t - own * kC + 1;
+    const T *kc = k + (kv0 + (size_t)c * kC) * D;
     float x[2], dp[2];
-    chunk_logits<T, D>(k + (kv0 + (size_t)c * kC) * D, v + (kv0 + (size_t)c * kC) * D, nkeys, lane,
-                       qv, dov, bs.scale, x, dp);
+    chunk_logits<T, D>(kc, v + (kv0 + (size_t)c * kC) * D, nkeys, lane, qv, dov, bs.scale, x, dp);
     const bool in0 = lane < nkeys, in1 = lane + 32 < nkeys;
     const float m = warp_max(fmaxf(in0 ? x[0] : -INFINITY, in1 ? x[1] : -INFINITY));
     const float e0 = in0 ? __expf(x[0] - m) : 0.0f, e1 = in1 ? __expf(x[1] - m) : 0.0f;
@@ -202,52 +215,54 @@ __global__ void __launch_bounds__(kRowWarps * 32)
     const float w = __expf(s - lse_t);
     Dsum += w * g;
     if (lane == 0) rrow[slot] = make_float4(lc, w, g, 0.0f);
-  }
-  __syncwarp();
-  // pass 2: ds_c, and dq = scale (sum_cj dx_j k_j + sum_sel ds_c lmk_c)
-  float acc[P];
+    // A_c and B_c over the lane's slice (p_j and p_j dP_j broadcast from their lanes)
+    const float p0 = e0 / l, p1 = e1 / l;
+    const float pd0 = p0 * dp[0], pd1 = p1 * dp[1];
+    float av[P], bv[P];
 #pragma unroll
-  for (int u = 0; u < P; ++u) acc[u] = 0.0f;
-  for (int slot = 0; slot <= K; ++slot) {
-    int c;
-    if (slot < K) {
-      c = srow[slot];
-      if (c < 0 || c >= own) continue;
-    } else {
-      c = own;
-    }
-    float4 r4 = rrow[slot];
-    const float lc = r4.x, w = r4.y, g = r4.z;
-    const float ds = w * (g - Dsum + dl);
-    if (lane == 0) rrow[slot] = make_float4(lc, w, g, ds);
-    const int nkeys = slot < K ? kC : t - own * kC + 1;
-    const T *kc = k + (kv0 + (size_t)c * kC) * D;
-    float x[2], dp[2];
-    chunk_logits<T, D>(kc, v + (kv0 + (size_t)c * kC) * D, nkeys, lane, qv, dov, bs.scale, x, dp);
-    float dx[2];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const bool in = lane + 32 * hh < nkeys;
-      const float pj = in ? __expf(x[hh] - lc) : 0.0f;
-      dx[hh] = w * pj * (dp[hh] - g) + (slot == K ? pj * ds : 0.0f);
-    }
-    // sum_j dx_j k_j over the lane's slice (dx_j broadcast from its lane)
+    for (int u = 0; u < P; ++u) av[u] = bv[u] = 0.0f;
     for (int j = 0; j < nkeys; ++j) {
-      const float dxj = __shfl_sync(0xffffffffu, j < 32 ? dx[0] : dx[1], j & 31);
+      const float pj = __shfl_sync(0xffffffffu, j < 32 ? p0 : p1, j & 31);
+      const float pdj = __shfl_sync(0xffffffffu, j < 32 ? pd0 : pd1, j & 31);
       float f[P];
       ld_slice<T, P>(kc + (size_t)j * D, lane, f);
 #pragma unroll
-      for (int u = 0; u < P; ++u) acc[u] = fmaf(dxj, f[u], acc[u]);
+      for (int u = 0; u < P; ++u) {
+        av[u] = fmaf(pdj, f[u], av[u]);
+        bv[u] = fmaf(pj, f[u], bv[u]);
+      }
     }
+    const float wg = w * (g + dl);
     if (slot < K) {
       float f[P];
       ld_slice<T, P>(lmk + (((size_t)b * bs.Hkv + hkv) * bs.nlmk + c) * D, lane, f);
 #pragma unroll
-      for (int u = 0; u < P; ++u) acc[u] = fmaf(ds, f[u], acc[u]);
+      for (int u = 0; u < P; ++u) {
+        acc[u] += w * (av[u] - g * bv[u]) + wg * f[u];
+        accd[u] = fmaf(w, f[u], accd[u]);
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < P; ++u) {
+        acc[u] += w * (av[u] - g * bv[u]) + wg * bv[u];
+        accd[u] = fmaf(w, bv[u], accd[u]);
+      }
     }
   }
 #pragma unroll
-  for (int u = 0; u < P; ++u) dq[(size_t)row * D + lane * P + u] = acc[u] * bs.scale;
+  for (int u = 0; u < P; ++u)
+    dq[(size_t)row * D + lane * P + u] = (acc[u] - Dsum * accd[u]) * bs.scale;
+  // ds_c = w_c (g_c - D + dlse) into the records of the attended slots
+  __syncwarp();
+  for (int slot = lane; slot <= K; slot += 32) {
+    if (slot < K) {
+      const int c = srow[slot];
+      if (c < 0 || c >= own) continue;
+    }
+    float4 r4 = rrow[slot];
+    r4.w = r4.y * (r4.z - Dsum + dl);
+    rrow[slot] = r4;
+  }
 }
 
 // the (row, slot) pairs that select each (b, kv head, chunk): count ...

@@ -88,6 +88,15 @@ def test_topk_edges(topk):
     check_all_rows(w, with_wfin=True)
 
 
+def test_staged_epilogue_k32_all_rows():
+    """bf16, d=128, k=32 on rows with more than 32 completed chunks (the
+    selection's rows leave through the per-warp staging blocks for K = 32),
+    and a ragged last tile (29 rows) whose warps past L write nothing."""
+    w = W.PREFILL_128K.with_(Hq=4, Hkv=2, L=64 * 40 + 29)
+    st = check_all_rows(w)
+    assert st["near_ties"] <= 0.01 * w.B * w.Hq * w.L
+
+
 def test_deterministic():
     w = W.PREFILL_128K.with_(Hq=4, Hkv=1, L=2048)
     q, k, v, lmk = (x.cuda() for x in synth.make_inputs(w, "cpu"))
