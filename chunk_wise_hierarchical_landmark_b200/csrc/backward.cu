@@ -23,12 +23,15 @@
 //   transposed selection: per (b, kv head, chunk) the (row, slot) pairs that
 //                     select it (count, exclusive scan, fill; the order inside
 //                     a chunk's list follows the atomic fill).
-//   bwd_chunks_kernel one CTA per (b, kv head, chunk): the chunk's K and V in
-//                     shared memory, a thread per (key, quarter of the head
-//                     dimension) accumulating dk and dv over the rows that
-//                     attend the chunk (its own rows, causally, and the rows
-//                     that selected it), dlmk over the selecting rows.
+//   bwd_chunks_kernel one CTA per (b, kv head, chunk): a thread per (key,
+//                     quarter of the head dimension), that quarter of the
+//                     key's K and V rows in registers, accumulating dk and dv
+//                     over the rows that attend the chunk (its own rows,
+//                     causally, and the rows that selected it; staged in
+//                     shared memory in batches), dlmk over the selecting rows.
 #include <cuda_bf16.h>
+
+#include <type_traits>
 
 #include "backward.h"
 #include "common.cuh"
@@ -39,22 +42,52 @@ namespace {
 constexpr int kC = 64;
 constexpr int kRowWarps = 8;       // rows per CTA of the row pass
 constexpr int kChunkThreads = 256; // 64 keys x 4 quarters
-constexpr int kRowBatch = 8;       // rows staged together in the chunk pass
+constexpr int kRowBatch = 16;      // rows staged together in the chunk pass
 
-template <typename T>
-__device__ __forceinline__ float ldf(const T *p);
-template <>
-__device__ __forceinline__ float ldf<float>(const float *p) { return *p; }
-template <>
-__device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16 *p) {
-  return __bfloat162float(*p);
-}
-
-// the lane's D/32 consecutive elements of a row, widened
+// the lane's D/32 consecutive elements of a row, widened (one vector load
+// for the two- and four-element slices of d = 64 and 128)
 template <typename T, int P>
 __device__ __forceinline__ void ld_slice(const T *row, int lane, float (&f)[P]) {
+  const T *r = row + lane * P;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value && P == 4) {
+    const uint2 w = *reinterpret_cast<const uint2 *>(r);
+    f[0] = __uint_as_float(w.x << 16);
+    f[1] = __uint_as_float(w.x & 0xFFFF0000u);
+    f[2] = __uint_as_float(w.y << 16);
+    f[3] = __uint_as_float(w.y & 0xFFFF0000u);
+  } else if constexpr (std::is_same<T, __nv_bfloat16>::value && P == 2) {
+    const uint32_t w = *reinterpret_cast<const uint32_t *>(r);
+    f[0] = __uint_as_float(w << 16);
+    f[1] = __uint_as_float(w & 0xFFFF0000u);
+  } else if constexpr (std::is_same<T, float>::value && P == 4) {
+    const float4 a = *reinterpret_cast<const float4 *>(r);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  } else if constexpr (std::is_same<T, float>::value && P == 2) {
+    const float2 a = *reinterpret_cast<const float2 *>(r);
+    f[0] = a.x; f[1] = a.y;
+  } else {
+    static_assert(P == 2 || P == 4, "head dimension 64 or 128");
+  }
+}
+
+// Eight consecutive elements of a row (16-byte aligned) widened to fp32.
+template <typename T>
+__device__ __forceinline__ void ld8(const T *p, float (&f)[8]);
+template <>
+__device__ __forceinline__ void ld8<__nv_bfloat16>(const __nv_bfloat16 *p, float (&f)[8]) {
+  const uint4 w = *reinterpret_cast<const uint4 *>(p);
+  const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-  for (int u = 0; u < P; ++u) f[u] = ldf(row + lane * P + u);
+  for (int u = 0; u < 4; ++u) {
+    f[2 * u] = __uint_as_float(ww[u] << 16);
+    f[2 * u + 1] = __uint_as_float(ww[u] & 0xFFFF0000u);
+  }
+}
+template <>
+__device__ __forceinline__ void ld8<float>(const float *p, float (&f)[8]) {
+  const float4 a = *reinterpret_cast<const float4 *>(p), b = *reinterpret_cast<const float4 *>(p + 4);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
 // Dot products of x (the lane's slice) with 32 consecutive rows (a reduce-
@@ -165,6 +198,7 @@ __global__ void __launch_bounds__(kRowWarps * 32)
   const int b = bh / bs.Hq, hq = bh % bs.Hq, hkv = hq / (bs.Hq / bs.Hkv);
   const int own = t / kC;
   const size_t kv0 = ((size_t)b * bs.Hkv + hkv) * L;  // first key row of the KV head
+  __shared__ float2 pd_s[kRowWarps][2 * 32];
   float qv[P], dov[P];
   ld_slice<T, P>(q + (size_t)row * D, lane, qv);
   ld_slice<T, P>(dout + (size_t)row * D, lane, dov);
@@ -215,21 +249,26 @@ __global__ void __launch_bounds__(kRowWarps * 32)
     const float w = __expf(s - lse_t);
     Dsum += w * g;
     if (lane == 0) rrow[slot] = make_float4(lc, w, g, 0.0f);
-    // A_c and B_c over the lane's slice (p_j and p_j dP_j broadcast from their lanes)
+    // A_c and B_c over the lane's slice (p_j and p_j dP_j broadcast from the
+    // warp's shared memory)
     const float p0 = e0 / l, p1 = e1 / l;
-    const float pd0 = p0 * dp[0], pd1 = p1 * dp[1];
+    float2 *pp = pd_s[threadIdx.x >> 5];
+    __syncwarp();
+    pp[lane] = make_float2(p0, p0 * dp[0]);
+    pp[lane + 32] = make_float2(p1, p1 * dp[1]);
+    __syncwarp();
     float av[P], bv[P];
 #pragma unroll
     for (int u = 0; u < P; ++u) av[u] = bv[u] = 0.0f;
+#pragma unroll 4
     for (int j = 0; j < nkeys; ++j) {
-      const float pj = __shfl_sync(0xffffffffu, j < 32 ? p0 : p1, j & 31);
-      const float pdj = __shfl_sync(0xffffffffu, j < 32 ? pd0 : pd1, j & 31);
+      const float2 pj = pp[j];
       float f[P];
       ld_slice<T, P>(kc + (size_t)j * D, lane, f);
 #pragma unroll
       for (int u = 0; u < P; ++u) {
-        av[u] = fmaf(pdj, f[u], av[u]);
-        bv[u] = fmaf(pj, f[u], bv[u]);
+        av[u] = fmaf(pj.y, f[u], av[u]);
+        bv[u] = fmaf(pj.x, f[u], bv[u]);
       }
     }
     const float wg = w * (g + dl);
@@ -339,6 +378,18 @@ __global__ void bwd_fill_kernel(BwdSpec bs, const int32_t *__restrict__ sel,
   ent_slot[pos] = (uint8_t)(i % bs.topk);
 }
 
+// n consecutive elements (a multiple of 8, 16-byte aligned) widened to fp32
+template <typename T, int N>
+__device__ __forceinline__ void ld_vec(const T *p, float (&f)[N]) {
+#pragma unroll
+  for (int u = 0; u < N; u += 8) {
+    float g[8];
+    ld8<T>(p + u, g);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[u + i] = g[i];
+  }
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kChunkThreads)
     bwd_chunks_kernel(BwdSpec bs, const T *__restrict__ q, const T *__restrict__ k,
@@ -346,15 +397,11 @@ __global__ void __launch_bounds__(kChunkThreads)
                       const float4 *__restrict__ rec, const uint32_t *__restrict__ off,
                       const int32_t *__restrict__ ent_row, const uint8_t *__restrict__ ent_slot,
                       float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ dlmk) {
-  constexpr int DQ = D / 4;  // dimensions per thread
-  // K, V [key][quarter][DQ + 1] and the staged rows [row][quarter][DQ + 1]:
-  // the padding puts the 32 lanes of a warp (8 keys x 4 quarters) on
-  // distinct banks
-  extern __shared__ float csm[];
-  float *ks = csm;
-  float *vs = ks + kC * 4 * (DQ + 1);
-  float *qs = vs + kC * 4 * (DQ + 1);
-  float *os = qs + kRowBatch * 4 * (DQ + 1);
+  constexpr int DQ = D / 4;   // dimensions per thread
+  constexpr int DS = DQ + 4;  // stride of a staged quarter row: 16-byte aligned, and the
+                              // four quarters a warp reads fall in distinct bank groups
+  // the staged rows [row][quarter][DS] of q and dO
+  __shared__ __align__(16) float qs[kRowBatch * 4 * DS], os[kRowBatch * 4 * DS];
   __shared__ float4 st[kRowBatch];
   __shared__ int own_s[kRowBatch];  // 1: the row's own chunk (slot k), with its position offset
   __shared__ int jmax_s[kRowBatch];
@@ -367,11 +414,13 @@ __global__ void __launch_bounds__(kChunkThreads)
   const size_t krow0 = (size_t)bk * L + (size_t)c * kC;
   const int tid = threadIdx.x;
   const int j = tid >> 2, qd = tid & 3;
-  auto at = [](int r, int e) { return (r * 4 + e / DQ) * (DQ + 1) + e % DQ; };
-  for (int i = tid; i < kC * D; i += kChunkThreads) {
-    const int jj = i / D, e = i % D;
-    ks[at(jj, e)] = jj < nkeys ? ldf(k + (krow0 + jj) * D + e) : 0.0f;
-    vs[at(jj, e)] = jj < nkeys ? ldf(v + (krow0 + jj) * D + e) : 0.0f;
+  // the thread's quarter of its key's K and V row, kept in registers (keys
+  // past the chunk's end read its last key; their p is zero)
+  float kr[DQ], vr[DQ];
+  {
+    const size_t kj = (krow0 + min(j, nkeys - 1)) * D + qd * DQ;
+    ld_vec<T, DQ>(k + kj, kr);
+    ld_vec<T, DQ>(v + kj, vr);
   }
   float ak[DQ], av[DQ];
 #pragma unroll
@@ -385,8 +434,9 @@ __global__ void __launch_bounds__(kChunkThreads)
   for (int r0 = 0; r0 < n_rows; r0 += kRowBatch) {
     const int nb = min(kRowBatch, n_rows - r0);
     __syncthreads();
-    for (int i = tid; i < nb * D; i += kChunkThreads) {
-      const int rr = i / D, e = i % D;
+    // stage the batch: 8 elements of a row per thread and step
+    for (int i = tid; i < nb * (D / 8); i += kChunkThreads) {
+      const int rr = i / (D / 8), e = (i % (D / 8)) * 8;
       const int ri = r0 + rr;
       long long row;
       if (ri < n_own) {
@@ -395,8 +445,14 @@ __global__ void __launch_bounds__(kChunkThreads)
       } else {
         row = ent_row[s0 + (ri - n_own)];
       }
-      qs[at(rr, e)] = ldf(q + (size_t)row * D + e);
-      os[at(rr, e)] = ldf(dout + (size_t)row * D + e);
+      float f[8];
+      const int at = (rr * 4 + e / DQ) * DS + e % DQ;
+      ld8<T>(q + (size_t)row * D + e, f);
+      *reinterpret_cast<float4 *>(qs + at) = make_float4(f[0], f[1], f[2], f[3]);
+      *reinterpret_cast<float4 *>(qs + at + 4) = make_float4(f[4], f[5], f[6], f[7]);
+      ld8<T>(dout + (size_t)row * D + e, f);
+      *reinterpret_cast<float4 *>(os + at) = make_float4(f[0], f[1], f[2], f[3]);
+      *reinterpret_cast<float4 *>(os + at + 4) = make_float4(f[4], f[5], f[6], f[7]);
       if (e == 0) {
         const int slot = ri < n_own ? K : (int)ent_slot[s0 + (ri - n_own)];
         st[rr] = rec[(size_t)row * (K + 1) + slot];
@@ -406,37 +462,52 @@ __global__ void __launch_bounds__(kChunkThreads)
     }
     __syncthreads();
     for (int rr = 0; rr < nb; ++rr) {
-      float a = 0.0f, d2 = 0.0f;
-      const float *qr = qs + (rr * 4 + qd) * (DQ + 1), *orow = os + (rr * 4 + qd) * (DQ + 1);
-      const float *kr = ks + (j * 4 + qd) * (DQ + 1), *vr = vs + (j * 4 + qd) * (DQ + 1);
+      const float4 *qr = reinterpret_cast<const float4 *>(qs + (rr * 4 + qd) * DS);
+      const float4 *orow = reinterpret_cast<const float4 *>(os + (rr * 4 + qd) * DS);
+      float2 a2 = make_float2(0.0f, 0.0f), d22 = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int u = 0; u < DQ; ++u) {
-        a = fmaf(qr[u], kr[u], a);
-        d2 = fmaf(orow[u], vr[u], d2);
+      for (int u = 0; u < DQ / 4; ++u) {
+        const float4 q4 = qr[u], o4 = orow[u];
+        a2 = __ffma2_rn(make_float2(q4.x, q4.y), make_float2(kr[4 * u], kr[4 * u + 1]), a2);
+        a2 = __ffma2_rn(make_float2(q4.z, q4.w), make_float2(kr[4 * u + 2], kr[4 * u + 3]), a2);
+        d22 = __ffma2_rn(make_float2(o4.x, o4.y), make_float2(vr[4 * u], vr[4 * u + 1]), d22);
+        d22 = __ffma2_rn(make_float2(o4.z, o4.w), make_float2(vr[4 * u + 2], vr[4 * u + 3]), d22);
       }
+      float a = a2.x + a2.y, d2 = d22.x + d22.y;
       a += __shfl_xor_sync(0xffffffffu, a, 1);
       a += __shfl_xor_sync(0xffffffffu, a, 2);
       d2 += __shfl_xor_sync(0xffffffffu, d2, 1);
       d2 += __shfl_xor_sync(0xffffffffu, d2, 2);
       const float4 s4 = st[rr];  // lse_c, w_c, g_c, ds_c
+      const bool own_r = own_s[rr] != 0;
       const bool in = j < nkeys && j <= jmax_s[rr];
       const float pj = in ? __expf(a * bs.scale - s4.x) : 0.0f;
-      const float dx = s4.y * pj * (d2 - s4.z) + (own_s[rr] ? pj * s4.w : 0.0f);
+      const float dx = s4.y * pj * (d2 - s4.z) + (own_r ? pj * s4.w : 0.0f);
       const float pw = s4.y * pj;
+      const float2 dx2 = make_float2(dx, dx), pw2 = make_float2(pw, pw);
 #pragma unroll
-      for (int u = 0; u < DQ; ++u) {
-        av[u] = fmaf(pw, orow[u], av[u]);
-        ak[u] = fmaf(dx, qr[u], ak[u]);
+      for (int u = 0; u < DQ / 4; ++u) {
+        const float4 q4 = qr[u], o4 = orow[u];
+        float2 t;
+        t = __ffma2_rn(pw2, make_float2(o4.x, o4.y), make_float2(av[4 * u], av[4 * u + 1]));
+        av[4 * u] = t.x; av[4 * u + 1] = t.y;
+        t = __ffma2_rn(pw2, make_float2(o4.z, o4.w), make_float2(av[4 * u + 2], av[4 * u + 3]));
+        av[4 * u + 2] = t.x; av[4 * u + 3] = t.y;
+        t = __ffma2_rn(dx2, make_float2(q4.x, q4.y), make_float2(ak[4 * u], ak[4 * u + 1]));
+        ak[4 * u] = t.x; ak[4 * u + 1] = t.y;
+        t = __ffma2_rn(dx2, make_float2(q4.z, q4.w), make_float2(ak[4 * u + 2], ak[4 * u + 3]));
+        ak[4 * u + 2] = t.x; ak[4 * u + 3] = t.y;
       }
-      if (!own_s[rr] && tid < D) al = fmaf(s4.w, qs[at(rr, tid)], al);
+      if (!own_r && tid < D) al = fmaf(s4.w, qs[(rr * 4 + tid / DQ) * DS + tid % DQ], al);
     }
   }
   if (j < nkeys) {
+    float *dkr = dk + (krow0 + j) * D + qd * DQ, *dvr = dv + (krow0 + j) * D + qd * DQ;
 #pragma unroll
-    for (int u = 0; u < DQ; ++u) {
-      const int e = qd * DQ + u;
-      dk[(krow0 + j) * D + e] = ak[u] * bs.scale;
-      dv[(krow0 + j) * D + e] = av[u];
+    for (int u = 0; u < DQ; u += 4) {
+      *reinterpret_cast<float4 *>(dkr + u) =
+          make_float4(ak[u] * bs.scale, ak[u + 1] * bs.scale, ak[u + 2] * bs.scale, ak[u + 3] * bs.scale);
+      *reinterpret_cast<float4 *>(dvr + u) = make_float4(av[u], av[u + 1], av[u + 2], av[u + 3]);
     }
   }
   if (c < bs.nlmk && tid < D) dlmk[((size_t)bk * bs.nlmk + c) * D + tid] = al * bs.scale;
@@ -509,9 +580,7 @@ cudaError_t bwd_run(const BwdSpec &bs, bool bf16, const void *q, const void *k, 
 #define HILS_BWD_CHUNKS(T, DD)                                                                   \
   do {                                                                                           \
     auto kern = bwd_chunks_kernel<T, DD>;                                                        \
-    const size_t smem = (size_t)(2 * kC + 2 * kRowBatch) * 4 * (DD / 4 + 1) * sizeof(float);     \
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e; \
-    kern<<<(unsigned)nseg, kChunkThreads, smem, st>>>(bs, (const T *)q, (const T *)k,            \
+    kern<<<(unsigned)nseg, kChunkThreads, 0, st>>>(bs, (const T *)q, (const T *)k,               \
         (const T *)v, (const T *)dout, rec, off, ent_row, ent_slot, dk, dv, dlmk);               \
   } while (0)
   if (bf16) { if (bs.d == 64) HILS_BWD_CHUNKS(__nv_bfloat16, 64); else HILS_BWD_CHUNKS(__nv_bfloat16, 128); }
