@@ -15,11 +15,11 @@
 //   dq_t  = scale (sum_cj dx_j k_j + sum_{c selected} ds_c lmk_c)
 //   dk_j += scale dx_j q_t,  dv_j += w_c p_cj dO_t,  dlmk_c += scale ds_c q_t
 // Three stages, all on the CUDA cores in fp32 (bf16 inputs widen exactly):
-//   bwd_rows_kernel   one warp per row, one pass over its chunks: per-chunk
-//                     softmax recomputed from q and the chunk's keys, g_c,
-//                     w_c, and dq with the D-dependent part factored out;
-//                     then D and the per-(row, slot) records (lse_c, w_c,
-//                     g_c, ds_c).
+//   bwd_rows_kernel   one warp per row (eight lanes per key, four keys per
+//                     step), one pass over its chunks: per-chunk softmax
+//                     recomputed from q and the chunk's keys, g_c, w_c, and
+//                     dq with the D-dependent part factored out; then D and
+//                     the per-(row, slot) records (lse_c, w_c, g_c, ds_c).
 //   transposed selection: per (b, kv head, chunk) the (row, slot) pairs that
 //                     select it (count, exclusive scan, fill; the order inside
 //                     a chunk's list follows the atomic fill).
@@ -44,32 +44,6 @@ constexpr int kRowWarps = 8;       // rows per CTA of the row pass
 constexpr int kChunkThreads = 256; // 64 keys x 4 quarters
 constexpr int kRowBatch = 16;      // rows staged together in the chunk pass
 
-// the lane's D/32 consecutive elements of a row, widened (one vector load
-// for the two- and four-element slices of d = 64 and 128)
-template <typename T, int P>
-__device__ __forceinline__ void ld_slice(const T *row, int lane, float (&f)[P]) {
-  const T *r = row + lane * P;
-  if constexpr (std::is_same<T, __nv_bfloat16>::value && P == 4) {
-    const uint2 w = *reinterpret_cast<const uint2 *>(r);
-    f[0] = __uint_as_float(w.x << 16);
-    f[1] = __uint_as_float(w.x & 0xFFFF0000u);
-    f[2] = __uint_as_float(w.y << 16);
-    f[3] = __uint_as_float(w.y & 0xFFFF0000u);
-  } else if constexpr (std::is_same<T, __nv_bfloat16>::value && P == 2) {
-    const uint32_t w = *reinterpret_cast<const uint32_t *>(r);
-    f[0] = __uint_as_float(w << 16);
-    f[1] = __uint_as_float(w & 0xFFFF0000u);
-  } else if constexpr (std::is_same<T, float>::value && P == 4) {
-    const float4 a = *reinterpret_cast<const float4 *>(r);
-    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-  } else if constexpr (std::is_same<T, float>::value && P == 2) {
-    const float2 a = *reinterpret_cast<const float2 *>(r);
-    f[0] = a.x; f[1] = a.y;
-  } else {
-    static_assert(P == 2 || P == 4, "head dimension 64 or 128");
-  }
-}
-
 // Eight consecutive elements of a row (16-byte aligned) widened to fp32.
 template <typename T>
 __device__ __forceinline__ void ld8(const T *p, float (&f)[8]);
@@ -90,31 +64,16 @@ __device__ __forceinline__ void ld8<float>(const float *p, float (&f)[8]) {
   f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
-// Dot products of x (the lane's slice) with 32 consecutive rows (a reduce-
-// scatter butterfly: lane l ends with the full dot product of row l).
-template <typename T, int P>
-__device__ __forceinline__ float dot32(const T *rows, int D, int lane, const float (&x)[P]) {
-  float v[32];
+// n consecutive elements (a multiple of 8, 16-byte aligned) widened to fp32
+template <typename T, int N>
+__device__ __forceinline__ void ld_vec(const T *p, float (&f)[N]) {
 #pragma unroll
-  for (int jj = 0; jj < 32; ++jj) {
-    float f[P];
-    ld_slice<T, P>(rows + (size_t)jj * D, lane, f);
-    float a = 0.0f;
+  for (int u = 0; u < N; u += 8) {
+    float g[8];
+    ld8<T>(p + u, g);
 #pragma unroll
-    for (int u = 0; u < P; ++u) a = fmaf(f[u], x[u], a);
-    v[jj] = a;
+    for (int i = 0; i < 8; ++i) f[u + i] = g[i];
   }
-#pragma unroll
-  for (int sft = 16; sft >= 1; sft >>= 1) {
-    const bool upper = (lane & sft) != 0;
-#pragma unroll
-    for (int i = 0; i < sft; ++i) {
-      const float send = upper ? v[i] : v[i + sft];
-      const float keep = upper ? v[i + sft] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
-    }
-  }
-  return v[0];
 }
 
 __device__ __forceinline__ float warp_max(float x) {
@@ -128,59 +87,32 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-// The chunk's logits x (keys lane and lane + 32 of the chunk) and dP.
-template <typename T, int D>
-__device__ __forceinline__ void chunk_logits(const T *kc, const T *vc, int nkeys, int lane,
-                                             const float (&qv)[D / 32], const float (&dov)[D / 32],
-                                             float scale, float (&x)[2], float (&dp)[2]) {
-  constexpr int P = D / 32;
+// acc += a * x over a lane's dimensions, as fp32 pairs
+template <int N>
+__device__ __forceinline__ void axpy2(float a, const float (&x)[N], float (&acc)[N]) {
+  const float2 a2 = make_float2(a, a);
 #pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    if (hh * 32 < nkeys) {
-      // rows past the chunk's keys are not read: clamp to its last key
-      const int base = hh * 32;
-      const int nblk = min(32, nkeys - base);
-      if (nblk == 32) {
-        x[hh] = dot32<T, P>(kc + (size_t)base * D, D, lane, qv) * scale;
-        dp[hh] = dot32<T, P>(vc + (size_t)base * D, D, lane, dov);
-      } else {
-        float vx[32], vd[32];
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int j = base + min(jj, nblk - 1);
-          float fk[P], fv[P];
-          ld_slice<T, P>(kc + (size_t)j * D, lane, fk);
-          ld_slice<T, P>(vc + (size_t)j * D, lane, fv);
-          float a = 0.0f, b = 0.0f;
-#pragma unroll
-          for (int u = 0; u < P; ++u) {
-            a = fmaf(fk[u], qv[u], a);
-            b = fmaf(fv[u], dov[u], b);
-          }
-          vx[jj] = a;
-          vd[jj] = b;
-        }
-#pragma unroll
-        for (int sft = 16; sft >= 1; sft >>= 1) {
-          const bool upper = (lane & sft) != 0;
-#pragma unroll
-          for (int i = 0; i < sft; ++i) {
-            const float sx = upper ? vx[i] : vx[i + sft], kx = upper ? vx[i + sft] : vx[i];
-            const float sd = upper ? vd[i] : vd[i + sft], kd = upper ? vd[i + sft] : vd[i];
-            vx[i] = kx + __shfl_xor_sync(0xffffffffu, sx, sft);
-            vd[i] = kd + __shfl_xor_sync(0xffffffffu, sd, sft);
-          }
-        }
-        x[hh] = vx[0] * scale;
-        dp[hh] = vd[0];
-      }
-    } else {
-      x[hh] = 0.0f;
-      dp[hh] = 0.0f;
-    }
+  for (int u = 0; u < N; u += 2) {
+    const float2 t = __ffma2_rn(a2, make_float2(x[u], x[u + 1]), make_float2(acc[u], acc[u + 1]));
+    acc[u] = t.x;
+    acc[u + 1] = t.y;
   }
 }
 
+// <x, y> over a lane's dimensions, fp32 pairs
+template <int N>
+__device__ __forceinline__ float dot2(const float (&x)[N], const float (&y)[N]) {
+  float2 a = make_float2(0.0f, 0.0f);
+#pragma unroll
+  for (int u = 0; u < N; u += 2)
+    a = __ffma2_rn(make_float2(x[u], x[u + 1]), make_float2(y[u], y[u + 1]), a);
+  return a.x + a.y;
+}
+
+// A warp per row.  Lane layout: eight lanes per key (sub = lane & 7 holds the
+// head dimensions [sub * DL, sub * DL + DL)), four keys per step (grp =
+// lane >> 3 takes key 4 i + grp at step i), so a 16-byte load of the warp
+// covers four whole key rows and a dot product needs three shuffle levels.
 template <typename T, int D>
 __global__ void __launch_bounds__(kRowWarps * 32)
     bwd_rows_kernel(BwdSpec bs, const T *__restrict__ q, const T *__restrict__ k,
@@ -189,19 +121,22 @@ __global__ void __launch_bounds__(kRowWarps * 32)
                     const float *__restrict__ lse, const T *__restrict__ dout,
                     const float *__restrict__ dlse, float4 *__restrict__ rec,
                     float *__restrict__ dq, uint32_t *__restrict__ err) {
-  constexpr int P = D / 32;
-  const int lane = threadIdx.x & 31;
-  const long long row = (long long)blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  constexpr int DL = D / 8;  // dimensions per lane
+  const int lane = threadIdx.x & 31, sub = lane & 7, grp = lane >> 3;
+  const int wi = threadIdx.x >> 5;
+  const long long row = (long long)blockIdx.x * kRowWarps + wi;
   if (row >= (long long)bs.B * bs.Hq * bs.L) return;
   const int L = bs.L, K = bs.topk;
   const int bh = (int)(row / L), t = (int)(row % L);
   const int b = bh / bs.Hq, hq = bh % bs.Hq, hkv = hq / (bs.Hq / bs.Hkv);
   const int own = t / kC;
   const size_t kv0 = ((size_t)b * bs.Hkv + hkv) * L;  // first key row of the KV head
-  __shared__ float2 pd_s[kRowWarps][2 * 32];
-  float qv[P], dov[P];
-  ld_slice<T, P>(q + (size_t)row * D, lane, qv);
-  ld_slice<T, P>(dout + (size_t)row * D, lane, dov);
+  // per warp: (x, dP) and then (p, p dP) of the chunk's keys
+  __shared__ float2 xd_s[kRowWarps][kC], pd_s[kRowWarps][kC];
+  float2 *xd = xd_s[wi], *pp = pd_s[wi];
+  float qv[DL], dov[DL];
+  ld_vec<T, DL>(q + (size_t)row * D + sub * DL, qv);
+  ld_vec<T, DL>(dout + (size_t)row * D + sub * DL, dov);
   const float lse_t = lse[row];
   const float dl = dlse ? dlse[row] : 0.0f;
   const int32_t *srow = sel + (size_t)row * K;
@@ -216,11 +151,14 @@ __global__ void __launch_bounds__(kRowWarps * 32)
   //              + w_own (g_own + dlse) B_own
   //              - D (sum_sel w_c lmk_c + w_own B_own)
   // (the ds_c = w_c (g_c - D + dlse) terms and the own chunk's p ds_own term
-  // regrouped); ds_c goes into the records afterwards.
-  float acc[P], accd[P];
+  // regrouped); ds_c goes into the records afterwards.  Every term is linear
+  // in A_c and B_c, so each key group accumulates its own keys' share and the
+  // four groups are summed once, at the end.
+  float acc[DL], accd[DL];
 #pragma unroll
-  for (int u = 0; u < P; ++u) acc[u] = accd[u] = 0.0f;
+  for (int u = 0; u < DL; ++u) acc[u] = accd[u] = 0.0f;
   float Dsum = 0.0f;
+  const float g0 = grp == 0 ? 1.0f : 0.0f;  // the landmark terms enter once
   for (int slot = 0; slot <= K; ++slot) {
     int c;
     float s_sel = 0.0f;
@@ -236,61 +174,85 @@ __global__ void __launch_bounds__(kRowWarps * 32)
       c = own;
     }
     const int nkeys = slot < K ? kC : t - own * kC + 1;
-    const T *kc = k + (kv0 + (size_t)c * kC) * D;
-    float x[2], dp[2];
-    chunk_logits<T, D>(kc, v + (kv0 + (size_t)c * kC) * D, nkeys, lane, qv, dov, bs.scale, x, dp);
+    const int nsteps = (nkeys + 3) >> 2;
+    const T *kc = k + (kv0 + (size_t)c * kC) * D + sub * DL;
+    const T *vc = v + (kv0 + (size_t)c * kC) * D + sub * DL;
+    __syncwarp();  // the previous chunk's reads of xd and pp are done
+#pragma unroll 8
+    for (int i = 0; i < nsteps; ++i) {
+      const int jj = 4 * i + grp, j = min(jj, nkeys - 1);
+      float fk[DL], fv[DL];
+      ld_vec<T, DL>(kc + (size_t)j * D, fk);
+      ld_vec<T, DL>(vc + (size_t)j * D, fv);
+      float a = dot2<DL>(fk, qv), d = dot2<DL>(fv, dov);
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        d += __shfl_xor_sync(0xffffffffu, d, o);
+      }
+      if (sub == 0) xd[jj] = make_float2(a * bs.scale, d);
+    }
+    __syncwarp();
+    // softmax over keys lane and lane + 32
     const bool in0 = lane < nkeys, in1 = lane + 32 < nkeys;
-    const float m = warp_max(fmaxf(in0 ? x[0] : -INFINITY, in1 ? x[1] : -INFINITY));
-    const float e0 = in0 ? __expf(x[0] - m) : 0.0f, e1 = in1 ? __expf(x[1] - m) : 0.0f;
+    const float2 r0 = in0 ? xd[lane] : make_float2(0.0f, 0.0f);
+    const float2 r1 = in1 ? xd[lane + 32] : make_float2(0.0f, 0.0f);
+    const float m = warp_max(fmaxf(in0 ? r0.x : -INFINITY, in1 ? r1.x : -INFINITY));
+    const float e0 = in0 ? __expf(r0.x - m) : 0.0f, e1 = in1 ? __expf(r1.x - m) : 0.0f;
     const float l = warp_sum(e0 + e1);
     const float lc = m + __logf(l);
-    const float g = warp_sum(e0 * dp[0] + e1 * dp[1]) / l;
+    const float g = warp_sum(e0 * r0.y + e1 * r1.y) / l;
     const float s = slot < K ? s_sel : lc;
     const float w = __expf(s - lse_t);
     Dsum += w * g;
     if (lane == 0) rrow[slot] = make_float4(lc, w, g, 0.0f);
-    // A_c and B_c over the lane's slice (p_j and p_j dP_j broadcast from the
-    // warp's shared memory)
     const float p0 = e0 / l, p1 = e1 / l;
-    float2 *pp = pd_s[threadIdx.x >> 5];
+    pp[lane] = make_float2(p0, p0 * r0.y);
+    pp[lane + 32] = make_float2(p1, p1 * r1.y);
     __syncwarp();
-    pp[lane] = make_float2(p0, p0 * dp[0]);
-    pp[lane + 32] = make_float2(p1, p1 * dp[1]);
-    __syncwarp();
-    float av[P], bv[P];
+    // the group's share of A_c and B_c (keys past nkeys have p = 0)
+    float av[DL], bv[DL];
 #pragma unroll
-    for (int u = 0; u < P; ++u) av[u] = bv[u] = 0.0f;
-#pragma unroll 4
-    for (int j = 0; j < nkeys; ++j) {
-      const float2 pj = pp[j];
-      float f[P];
-      ld_slice<T, P>(kc + (size_t)j * D, lane, f);
-#pragma unroll
-      for (int u = 0; u < P; ++u) {
-        av[u] = fmaf(pj.y, f[u], av[u]);
-        bv[u] = fmaf(pj.x, f[u], bv[u]);
-      }
+    for (int u = 0; u < DL; ++u) av[u] = bv[u] = 0.0f;
+#pragma unroll 8
+    for (int i = 0; i < nsteps; ++i) {
+      const int jj = 4 * i + grp, j = min(jj, nkeys - 1);
+      const float2 pj = pp[jj];
+      float fk[DL];
+      ld_vec<T, DL>(kc + (size_t)j * D, fk);
+      axpy2<DL>(pj.y, fk, av);
+      axpy2<DL>(pj.x, fk, bv);
     }
     const float wg = w * (g + dl);
+#pragma unroll
+    for (int u = 0; u < DL; ++u) av[u] -= g * bv[u];
+    axpy2<DL>(w, av, acc);
     if (slot < K) {
-      float f[P];
-      ld_slice<T, P>(lmk + (((size_t)b * bs.Hkv + hkv) * bs.nlmk + c) * D, lane, f);
-#pragma unroll
-      for (int u = 0; u < P; ++u) {
-        acc[u] += w * (av[u] - g * bv[u]) + wg * f[u];
-        accd[u] = fmaf(w, f[u], accd[u]);
-      }
+      float f[DL];
+      ld_vec<T, DL>(lmk + (((size_t)b * bs.Hkv + hkv) * bs.nlmk + c) * D + sub * DL, f);
+      axpy2<DL>(wg * g0, f, acc);
+      axpy2<DL>(w * g0, f, accd);
     } else {
-#pragma unroll
-      for (int u = 0; u < P; ++u) {
-        acc[u] += w * (av[u] - g * bv[u]) + wg * bv[u];
-        accd[u] = fmaf(w, bv[u], accd[u]);
-      }
+      axpy2<DL>(wg, bv, acc);
+      axpy2<DL>(w, bv, accd);
     }
   }
+  // sum the four key groups; group 0 writes the lane's dimensions of dq
 #pragma unroll
-  for (int u = 0; u < P; ++u)
-    dq[(size_t)row * D + lane * P + u] = (acc[u] - Dsum * accd[u]) * bs.scale;
+  for (int u = 0; u < DL; ++u) {
+    acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], 8);
+    acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], 16);
+    accd[u] += __shfl_xor_sync(0xffffffffu, accd[u], 8);
+    accd[u] += __shfl_xor_sync(0xffffffffu, accd[u], 16);
+  }
+  if (grp == 0) {
+    float *dqr = dq + (size_t)row * D + sub * DL;
+#pragma unroll
+    for (int u = 0; u < DL; u += 4)
+      *reinterpret_cast<float4 *>(dqr + u) =
+          make_float4((acc[u] - Dsum * accd[u]) * bs.scale, (acc[u + 1] - Dsum * accd[u + 1]) * bs.scale,
+                      (acc[u + 2] - Dsum * accd[u + 2]) * bs.scale, (acc[u + 3] - Dsum * accd[u + 3]) * bs.scale);
+  }
   // ds_c = w_c (g_c - D + dlse) into the records of the attended slots
   __syncwarp();
   for (int slot = lane; slot <= K; slot += 32) {
@@ -376,18 +338,6 @@ __global__ void bwd_fill_kernel(BwdSpec bs, const int32_t *__restrict__ sel,
   const uint32_t pos = off[seg] + atomicAdd(&cur[seg], 1u);
   ent_row[pos] = (int32_t)row;
   ent_slot[pos] = (uint8_t)(i % bs.topk);
-}
-
-// n consecutive elements (a multiple of 8, 16-byte aligned) widened to fp32
-template <typename T, int N>
-__device__ __forceinline__ void ld_vec(const T *p, float (&f)[N]) {
-#pragma unroll
-  for (int u = 0; u < N; u += 8) {
-    float g[8];
-    ld8<T>(p + u, g);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) f[u + i] = g[i];
-  }
 }
 
 template <typename T, int D>
