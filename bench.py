@@ -578,16 +578,18 @@ def bench_backward(hb, synth, w, steps, warmup):
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
+    n0 = hb.launch_count()
     a.record(stream)
     for _ in range(steps):
         step()
     b.record(stream)
     torch.cuda.synchronize()
+    launches = hb.launch_count() - n0
     ms = a.elapsed_time(b) / steps
     flop = backward_work(w)
     return {"value": w.B * w.L / (ms * 1e-3), "unit": "query-tokens/s", "ms_per_step": ms,
             "algorithmic_tflops": flop / (ms * 1e-3) / 1e12, "bound": "alu",
-            "workspace_bytes": ws.numel()}
+            "workspace_bytes": ws.numel(), "launches": launches}
 
 
 def bench_qcal(hb, synth, w, steps, warmup, r=32):
@@ -706,6 +708,8 @@ def run_ours(args):
     w = W.BY_NAME[args.workload]
     if w.decode:
         return run_decode_line(hb, synth, w, args, ws, rank)
+    if args.backward:
+        return run_backward_line(hb, synth, w, args, ws, rank)
     res = bench_prefill(hb, synth, w, args.steps, args.warmup, ws, rank, seed_offset=rank)
     ms = max_over_ranks(res["ms"], ws)
     e2e_ms = max_over_ranks(res["e2e_ms"], ws)
@@ -891,6 +895,33 @@ def run_decode_line(hb, synth, w, args, ws, rank):
         torch.distributed.destroy_process_group()
 
 
+def run_backward_line(hb, synth, w, args, ws, rank):
+    """The backward pass of a prefill workload as the main line (used for
+    profiler captures of the backward kernels): step = one hils_attn_bwd call
+    on the forward's selection, with dO and dlse seeded."""
+    r = bench_backward(hb, synth, w, args.steps, args.warmup)
+    launches = r["launches"]
+    ms = max_over_ranks(r["ms_per_step"], ws)
+    peak = alu_peak_tflops(None)
+    tflops = backward_work(w) / (ms * 1e-3) / 1e12
+    line = {"metric": "HiLS backward query-tokens/s", "value": w.B * w.L * ws / (ms * 1e-3),
+            "unit": "query-tokens/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic (seeded; dO and dlse seeded)",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L,
+                       "d": w.d, "chunk": w.C, "topk": w.topk, "inputs": w.dtype},
+            "roofline": {"bound": "alu", "kernel": "hils_attn_bwd", "achieved": tflops,
+                         "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
+                         "peak_source": "fp32 FMA issue rate at the maximum SM clock "
+                                        "(148 SMs x 128 lanes x 2 FLOP x 1965 MHz)",
+                         "traffic": None},
+            "gpu_launches": launches}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
 def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
@@ -942,6 +973,8 @@ def main():
     ap.add_argument("--extra", dest="extra", action="store_true", default=True)
     ap.add_argument("--no-extra", dest="extra", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass of the (prefill) workload instead")
     ap.add_argument("--hq", type=int, default=None,
                     help="override the query-head count (smaller cases for profiler captures)")
     ap.add_argument("--hkv", type=int, default=None, help="override the KV-head count")

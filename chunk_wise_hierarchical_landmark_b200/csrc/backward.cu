@@ -42,7 +42,7 @@ namespace {
 constexpr int kC = 64;
 constexpr int kRowWarps = 8;       // rows per CTA of the row pass
 constexpr int kChunkThreads = 256; // 64 keys x 4 quarters
-constexpr int kRowBatch = 16;      // rows staged together in the chunk pass
+constexpr int kRowBatch = 32;      // rows staged together in the chunk pass
 
 // Eight consecutive elements of a row (16-byte aligned) widened to fp32.
 template <typename T>
@@ -114,7 +114,7 @@ __device__ __forceinline__ float dot2(const float (&x)[N], const float (&y)[N]) 
 // lane >> 3 takes key 4 i + grp at step i), so a 16-byte load of the warp
 // covers four whole key rows and a dot product needs three shuffle levels.
 template <typename T, int D>
-__global__ void __launch_bounds__(kRowWarps * 32)
+__global__ void __launch_bounds__(kRowWarps * 32, 3)  // three CTAs per SM: a latency-bound loop
     bwd_rows_kernel(BwdSpec bs, const T *__restrict__ q, const T *__restrict__ k,
                     const T *__restrict__ v, const T *__restrict__ lmk,
                     const int32_t *__restrict__ sel, const float *__restrict__ chunk_w,
