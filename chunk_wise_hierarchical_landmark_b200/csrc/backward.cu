@@ -41,7 +41,6 @@ namespace {
 
 constexpr int kC = 64;
 constexpr int kRowWarps = 8;       // rows per CTA of the row pass
-constexpr int kChunkThreads = 256; // 64 keys x 4 quarters
 constexpr int kRowBatch = 32;      // rows staged together in the chunk pass
 
 // Eight consecutive elements of a row (16-byte aligned) widened to fp32.
@@ -340,16 +339,27 @@ __global__ void bwd_fill_kernel(BwdSpec bs, const int32_t *__restrict__ sel,
   ent_slot[pos] = (uint8_t)(i % bs.topk);
 }
 
+// Keys per thread of the chunk pass: two at d = 64 (each staged q / dO value
+// read from shared memory then feeds two keys), one at d = 128 (registers).
+template <int D>
+struct ChunkCfg {
+  static constexpr int kKeys = D == 64 ? 2 : 1;
+  static constexpr int kThreads = kC * 4 / kKeys;
+  static constexpr int kMinBlocks = D == 64 ? 3 : 1;
+};
+
 template <typename T, int D>
-__global__ void __launch_bounds__(kChunkThreads)
+__global__ void __launch_bounds__(ChunkCfg<D>::kThreads, ChunkCfg<D>::kMinBlocks)
     bwd_chunks_kernel(BwdSpec bs, const T *__restrict__ q, const T *__restrict__ k,
                       const T *__restrict__ v, const T *__restrict__ dout,
                       const float4 *__restrict__ rec, const uint32_t *__restrict__ off,
                       const int32_t *__restrict__ ent_row, const uint8_t *__restrict__ ent_slot,
                       float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ dlmk) {
-  constexpr int DQ = D / 4;   // dimensions per thread
-  constexpr int DS = DQ + 4;  // stride of a staged quarter row: 16-byte aligned, and the
-                              // four quarters a warp reads fall in distinct bank groups
+  constexpr int KPT = ChunkCfg<D>::kKeys, NT = ChunkCfg<D>::kThreads;
+  constexpr int KS = kC / KPT;  // distance between a thread's keys
+  constexpr int DQ = D / 4;     // dimensions per thread
+  constexpr int DS = DQ + 4;    // stride of a staged quarter row: 16-byte aligned, and the
+                                // four quarters a warp reads fall in distinct bank groups
   // the staged rows [row][quarter][DS] of q and dO
   __shared__ __align__(16) float qs[kRowBatch * 4 * DS], os[kRowBatch * 4 * DS];
   __shared__ float4 st[kRowBatch];
@@ -363,18 +373,21 @@ __global__ void __launch_bounds__(kChunkThreads)
   const int nkeys = min(kC, L - c * kC);
   const size_t krow0 = (size_t)bk * L + (size_t)c * kC;
   const int tid = threadIdx.x;
-  const int j = tid >> 2, qd = tid & 3;
-  // the thread's quarter of its key's K and V row, kept in registers (keys
+  const int jp = tid >> 2, qd = tid & 3;  // keys jp + kk * KS, dimension quarter qd
+  // the thread's quarter of its keys' K and V rows, kept in registers (keys
   // past the chunk's end read its last key; their p is zero)
-  float kr[DQ], vr[DQ];
-  {
-    const size_t kj = (krow0 + min(j, nkeys - 1)) * D + qd * DQ;
-    ld_vec<T, DQ>(k + kj, kr);
-    ld_vec<T, DQ>(v + kj, vr);
-  }
-  float ak[DQ], av[DQ];
+  float kr[KPT][DQ], vr[KPT][DQ];
 #pragma unroll
-  for (int u = 0; u < DQ; ++u) ak[u] = av[u] = 0.0f;
+  for (int kk = 0; kk < KPT; ++kk) {
+    const size_t kj = (krow0 + min(jp + kk * KS, nkeys - 1)) * D + qd * DQ;
+    ld_vec<T, DQ>(k + kj, kr[kk]);
+    ld_vec<T, DQ>(v + kj, vr[kk]);
+  }
+  float ak[KPT][DQ], av[KPT][DQ];
+#pragma unroll
+  for (int kk = 0; kk < KPT; ++kk)
+#pragma unroll
+    for (int u = 0; u < DQ; ++u) ak[kk][u] = av[kk][u] = 0.0f;
   float al = 0.0f;  // dlmk: thread tid < D owns dimension tid
   // rows: own rows (every query head of the group, positions of this chunk),
   // then the rows that selected the chunk
@@ -385,7 +398,7 @@ __global__ void __launch_bounds__(kChunkThreads)
     const int nb = min(kRowBatch, n_rows - r0);
     __syncthreads();
     // stage the batch: 8 elements of a row per thread and step
-    for (int i = tid; i < nb * (D / 8); i += kChunkThreads) {
+    for (int i = tid; i < nb * (D / 8); i += NT) {
       const int rr = i / (D / 8), e = (i % (D / 8)) * 8;
       const int ri = r0 + rr;
       long long row;
@@ -414,50 +427,71 @@ __global__ void __launch_bounds__(kChunkThreads)
     for (int rr = 0; rr < nb; ++rr) {
       const float4 *qr = reinterpret_cast<const float4 *>(qs + (rr * 4 + qd) * DS);
       const float4 *orow = reinterpret_cast<const float4 *>(os + (rr * 4 + qd) * DS);
-      float2 a2 = make_float2(0.0f, 0.0f), d22 = make_float2(0.0f, 0.0f);
+      float2 a2[KPT], d22[KPT];
+#pragma unroll
+      for (int kk = 0; kk < KPT; ++kk) a2[kk] = d22[kk] = make_float2(0.0f, 0.0f);
 #pragma unroll
       for (int u = 0; u < DQ / 4; ++u) {
         const float4 q4 = qr[u], o4 = orow[u];
-        a2 = __ffma2_rn(make_float2(q4.x, q4.y), make_float2(kr[4 * u], kr[4 * u + 1]), a2);
-        a2 = __ffma2_rn(make_float2(q4.z, q4.w), make_float2(kr[4 * u + 2], kr[4 * u + 3]), a2);
-        d22 = __ffma2_rn(make_float2(o4.x, o4.y), make_float2(vr[4 * u], vr[4 * u + 1]), d22);
-        d22 = __ffma2_rn(make_float2(o4.z, o4.w), make_float2(vr[4 * u + 2], vr[4 * u + 3]), d22);
+#pragma unroll
+        for (int kk = 0; kk < KPT; ++kk) {
+          a2[kk] = __ffma2_rn(make_float2(q4.x, q4.y), make_float2(kr[kk][4 * u], kr[kk][4 * u + 1]), a2[kk]);
+          a2[kk] = __ffma2_rn(make_float2(q4.z, q4.w), make_float2(kr[kk][4 * u + 2], kr[kk][4 * u + 3]), a2[kk]);
+          d22[kk] = __ffma2_rn(make_float2(o4.x, o4.y), make_float2(vr[kk][4 * u], vr[kk][4 * u + 1]), d22[kk]);
+          d22[kk] = __ffma2_rn(make_float2(o4.z, o4.w), make_float2(vr[kk][4 * u + 2], vr[kk][4 * u + 3]), d22[kk]);
+        }
       }
-      float a = a2.x + a2.y, d2 = d22.x + d22.y;
-      a += __shfl_xor_sync(0xffffffffu, a, 1);
-      a += __shfl_xor_sync(0xffffffffu, a, 2);
-      d2 += __shfl_xor_sync(0xffffffffu, d2, 1);
-      d2 += __shfl_xor_sync(0xffffffffu, d2, 2);
       const float4 s4 = st[rr];  // lse_c, w_c, g_c, ds_c
       const bool own_r = own_s[rr] != 0;
-      const bool in = j < nkeys && j <= jmax_s[rr];
-      const float pj = in ? __expf(a * bs.scale - s4.x) : 0.0f;
-      const float dx = s4.y * pj * (d2 - s4.z) + (own_r ? pj * s4.w : 0.0f);
-      const float pw = s4.y * pj;
-      const float2 dx2 = make_float2(dx, dx), pw2 = make_float2(pw, pw);
+      const int jm = jmax_s[rr];
+      float2 dx2[KPT], pw2[KPT];
+#pragma unroll
+      for (int kk = 0; kk < KPT; ++kk) {
+        float a = a2[kk].x + a2[kk].y, d2 = d22[kk].x + d22[kk].y;
+        a += __shfl_xor_sync(0xffffffffu, a, 1);
+        a += __shfl_xor_sync(0xffffffffu, a, 2);
+        d2 += __shfl_xor_sync(0xffffffffu, d2, 1);
+        d2 += __shfl_xor_sync(0xffffffffu, d2, 2);
+        const int j = jp + kk * KS;
+        const bool in = j < nkeys && j <= jm;
+        const float pj = in ? __expf(a * bs.scale - s4.x) : 0.0f;
+        const float dx = s4.y * pj * (d2 - s4.z) + (own_r ? pj * s4.w : 0.0f);
+        const float pw = s4.y * pj;
+        dx2[kk] = make_float2(dx, dx);
+        pw2[kk] = make_float2(pw, pw);
+      }
 #pragma unroll
       for (int u = 0; u < DQ / 4; ++u) {
         const float4 q4 = qr[u], o4 = orow[u];
-        float2 t;
-        t = __ffma2_rn(pw2, make_float2(o4.x, o4.y), make_float2(av[4 * u], av[4 * u + 1]));
-        av[4 * u] = t.x; av[4 * u + 1] = t.y;
-        t = __ffma2_rn(pw2, make_float2(o4.z, o4.w), make_float2(av[4 * u + 2], av[4 * u + 3]));
-        av[4 * u + 2] = t.x; av[4 * u + 3] = t.y;
-        t = __ffma2_rn(dx2, make_float2(q4.x, q4.y), make_float2(ak[4 * u], ak[4 * u + 1]));
-        ak[4 * u] = t.x; ak[4 * u + 1] = t.y;
-        t = __ffma2_rn(dx2, make_float2(q4.z, q4.w), make_float2(ak[4 * u + 2], ak[4 * u + 3]));
-        ak[4 * u + 2] = t.x; ak[4 * u + 3] = t.y;
+#pragma unroll
+        for (int kk = 0; kk < KPT; ++kk) {
+          float2 t;
+          t = __ffma2_rn(pw2[kk], make_float2(o4.x, o4.y), make_float2(av[kk][4 * u], av[kk][4 * u + 1]));
+          av[kk][4 * u] = t.x; av[kk][4 * u + 1] = t.y;
+          t = __ffma2_rn(pw2[kk], make_float2(o4.z, o4.w), make_float2(av[kk][4 * u + 2], av[kk][4 * u + 3]));
+          av[kk][4 * u + 2] = t.x; av[kk][4 * u + 3] = t.y;
+          t = __ffma2_rn(dx2[kk], make_float2(q4.x, q4.y), make_float2(ak[kk][4 * u], ak[kk][4 * u + 1]));
+          ak[kk][4 * u] = t.x; ak[kk][4 * u + 1] = t.y;
+          t = __ffma2_rn(dx2[kk], make_float2(q4.z, q4.w), make_float2(ak[kk][4 * u + 2], ak[kk][4 * u + 3]));
+          ak[kk][4 * u + 2] = t.x; ak[kk][4 * u + 3] = t.y;
+        }
       }
       if (!own_r && tid < D) al = fmaf(s4.w, qs[(rr * 4 + tid / DQ) * DS + tid % DQ], al);
     }
   }
-  if (j < nkeys) {
-    float *dkr = dk + (krow0 + j) * D + qd * DQ, *dvr = dv + (krow0 + j) * D + qd * DQ;
 #pragma unroll
-    for (int u = 0; u < DQ; u += 4) {
-      *reinterpret_cast<float4 *>(dkr + u) =
-          make_float4(ak[u] * bs.scale, ak[u + 1] * bs.scale, ak[u + 2] * bs.scale, ak[u + 3] * bs.scale);
-      *reinterpret_cast<float4 *>(dvr + u) = make_float4(av[u], av[u + 1], av[u + 2], av[u + 3]);
+  for (int kk = 0; kk < KPT; ++kk) {
+    const int j = jp + kk * KS;
+    if (j < nkeys) {
+      float *dkr = dk + (krow0 + j) * D + qd * DQ, *dvr = dv + (krow0 + j) * D + qd * DQ;
+#pragma unroll
+      for (int u = 0; u < DQ; u += 4) {
+        *reinterpret_cast<float4 *>(dkr + u) =
+            make_float4(ak[kk][u] * bs.scale, ak[kk][u + 1] * bs.scale, ak[kk][u + 2] * bs.scale,
+                        ak[kk][u + 3] * bs.scale);
+        *reinterpret_cast<float4 *>(dvr + u) =
+            make_float4(av[kk][u], av[kk][u + 1], av[kk][u + 2], av[kk][u + 3]);
+      }
     }
   }
   if (c < bs.nlmk && tid < D) dlmk[((size_t)bk * bs.nlmk + c) * D + tid] = al * bs.scale;
@@ -530,7 +564,7 @@ cudaError_t bwd_run(const BwdSpec &bs, bool bf16, const void *q, const void *k, 
 #define HILS_BWD_CHUNKS(T, DD)                                                                   \
   do {                                                                                           \
     auto kern = bwd_chunks_kernel<T, DD>;                                                        \
-    kern<<<(unsigned)nseg, kChunkThreads, 0, st>>>(bs, (const T *)q, (const T *)k,               \
+    kern<<<(unsigned)nseg, ChunkCfg<DD>::kThreads, 0, st>>>(bs, (const T *)q, (const T *)k,      \
         (const T *)v, (const T *)dout, rec, off, ent_row, ent_slot, dk, dv, dlmk);               \
   } while (0)
   if (bf16) { if (bs.d == 64) HILS_BWD_CHUNKS(__nv_bfloat16, 64); else HILS_BWD_CHUNKS(__nv_bfloat16, 128); }
