@@ -35,6 +35,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <utility>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -174,6 +175,7 @@ __global__ void __launch_bounds__(192, 1)
                           const __nv_bfloat16 *__restrict__ q, float *__restrict__ scores,
                           uint32_t *__restrict__ err) {
   using Lay = GemvTcLayout<D>;
+  grid_dep_launch();  // the top-k may launch (it waits for this grid's scores)
   // a name of its own: this kernel asks the dynamic window for 1024-byte alignment
   extern __shared__ __align__(1024) unsigned char smem_tc[];
   unsigned char *smem = smem_tc;
@@ -324,6 +326,8 @@ __global__ void __launch_bounds__(kTkThreads) decode_topk_kernel(DecodeSpec ds,
   const int n = ds.n_c, K = ds.topk;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float *sc = scores + (size_t)h * n;
+  grid_dep_launch();
+  grid_dep_wait();  // the landmark pass's scores
   if (staged) {
     // one pass over HBM/L2 with every load in flight; the rest reads shared memory
 #pragma unroll 8
@@ -620,6 +624,8 @@ __global__ void __launch_bounds__(256) decode_union_kernel(DecodeSpec ds,
   const int own = ds.own;
 
   for (int i = tid; i < ds.nwords; i += blockDim.x) bitmap[i] = 0;
+  grid_dep_launch();
+  grid_dep_wait();  // the top-k's selections
   __syncthreads();
   for (int i = tid; i < G * K; i += blockDim.x) {
     const int g = i / K, j = i % K;
@@ -752,6 +758,7 @@ __global__ void __launch_bounds__(kAttnThreads, HILS_DECODE_MINB) decode_attn_ke
   unsigned char *smem = smem_at;
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) report(err, DEV_BAD_INDEX);
+    grid_dep_wait();  // complete only after the kernels before it (the next ones rely on that)
     return;
   }
   float *qs = reinterpret_cast<float *>(smem + Lay::qs);
@@ -765,8 +772,6 @@ __global__ void __launch_bounds__(kAttnThreads, HILS_DECODE_MINB) decode_attn_ke
   const int qi = blockIdx.x, bk = blockIdx.y;
   const int b = bk / ds.Hkv, hkv = bk % ds.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int count = u_count[bk];
-  const int i0 = qi * kChunksPerCta, i1 = min(count, i0 + kChunksPerCta);
   const int cap = ds.ucap;
   const size_t kvbase = (size_t)bk * ds.N;
   const int t = ds.N - 1, own = ds.own;
@@ -782,6 +787,10 @@ __global__ void __launch_bounds__(kAttnThreads, HILS_DECODE_MINB) decode_attn_ke
     qs[i] = g < G ? to_f(q[((size_t)b * ds.Hq + hkv * G + g) * D + e]) * ds.scale : 0.0f;
   }
   for (int i = tid; i < kC * GB; i += kAttnThreads) ps[i] = 0.0f;  // heads >= G stay 0
+  grid_dep_launch();
+  grid_dep_wait();  // the union (everything above reads inputs only)
+  const int count = u_count[bk];
+  const int i0 = qi * kChunksPerCta, i1 = min(count, i0 + kChunksPerCta);
   int *ent_c = reinterpret_cast<int *>(smem + Lay::ent_c);
   uint32_t *ent_m = reinterpret_cast<uint32_t *>(smem + Lay::ent_m);
   int *ent_y = reinterpret_cast<int *>(smem + Lay::ent_y);
@@ -1046,6 +1055,7 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeSpec ds,
   const int b = h / ds.Hq, hq = h % ds.Hq;
   const int bk = b * ds.Hkv + hq / G, g = hq % G;
   const size_t rec = 2 + D;
+  grid_dep_wait();  // the chunk attention's partials
   float M = -INFINITY;
   for (int s = 0; s < ds.Q; ++s) M = fmaxf(M, part[(((size_t)bk * ds.Q + s) * G + g) * rec]);
   float L = 0.0f, o = 0.0f;
@@ -1100,7 +1110,30 @@ size_t decode_workspace_bytes(const DecodeSpec &ds) {
 
 size_t decode_max_g() { return kMaxG; }
 
+// A launch that may overlap the end of the kernel before it in the stream
+// (programmatic stream serialization): the kernel's grid_dep_wait() orders
+// its reads of that kernel's results.
+// its reads of that kernel's results.  dep = false: an ordinary launch.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_dep(bool dep, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args &&...args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = dep ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // The five launches of one decode step; pages.table == nullptr: dense caches.
+// Each launch after the first may start while the one before it finishes; the
+// first (the landmark pass, or the top-k when there is none) is an ordinary
+// launch, so the step's inputs are complete before any of its kernels runs.
 static cudaError_t decode_run(const DecodeSpec &ds, bool bf16, const void *q, const void *k,
                               const void *v, const PagedKV &pages, const void *lmk, int32_t *sel,
                               float *w, float *lse_lmk, void *out, float *lse, void *ws,
@@ -1152,15 +1185,17 @@ static cudaError_t decode_run(const DecodeSpec &ds, bool bf16, const void *q, co
     const size_t tsmem = (size_t)ds.n_c * sizeof(float);
     const int staged = tsmem <= 160 * 1024 ? 1 : 0;
     if (staged && (e = cudaFuncSetAttribute(decode_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem)) != cudaSuccess) return e;
-    decode_topk_kernel<<<(unsigned)(ds.B * ds.Hq), kTkThreads, staged ? tsmem : 0, st>>>(ds, scores, sel, w, lse_lmk, staged);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_dep(ds.P > 0, decode_topk_kernel, dim3((unsigned)(ds.B * ds.Hq)), dim3(kTkThreads),
+                        staged ? tsmem : 0, st, ds, (const float *)scores, sel, w, lse_lmk, staged)) != cudaSuccess)
+      return e;
   }
   ++*launches;
   {
     const size_t smem = (size_t)G * ds.topk * 8 + (size_t)ds.nwords * 8;
     if ((e = cudaFuncSetAttribute(decode_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
-    decode_union_kernel<<<(unsigned)BK, 256, smem, st>>>(ds, sel, w, u_c, u_mask, u_logit, u_count);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_dep(true, decode_union_kernel, dim3((unsigned)BK), dim3(256), smem, st, ds,
+                        (const int32_t *)sel, (const float *)w, u_c, u_mask, u_logit, u_count)) != cudaSuccess)
+      return e;
     ++*launches;
   }
   {
@@ -1176,7 +1211,11 @@ static cudaError_t decode_run(const DecodeSpec &ds, bool bf16, const void *q, co
     auto kern = decode_attn_kernel<T, DD, GG>;                                                  \
     const size_t smem = DecAttnLayout<T, DD, GG>::total;                                        \
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e; \
-    kern<<<dim3(ds.Q, (unsigned)BK), kAttnThreads, smem, st>>>(tk, ds, (const T *)q, (const T *)k, (const T *)v, pages, u_c, u_mask, u_logit, u_count, part, err); \
+    if ((e = launch_dep(true, kern, dim3(ds.Q, (unsigned)BK), dim3(kAttnThreads), smem, st, tk, ds,   \
+                        (const T *)q, (const T *)k, (const T *)v, pages, (const int32_t *)u_c,   \
+                        (const uint32_t *)u_mask, (const float *)u_logit,                        \
+                        (const int32_t *)u_count, part, err)) != cudaSuccess)                    \
+      return e;                                                                                 \
   } while (0)
 #define HILS_ATTN_G(T, DD)                                                                      \
   do {                                                                                          \
@@ -1194,7 +1233,12 @@ static cudaError_t decode_run(const DecodeSpec &ds, bool bf16, const void *q, co
   }
   {
     const int nh = ds.B * ds.Hq;
-#define HILS_COMB(T, DD) decode_combine_kernel<T, DD><<<nh, DD, 0, st>>>(ds, part, (T *)out, lse)
+#define HILS_COMB(T, DD)                                                                        \
+  do {                                                                                          \
+    if ((e = launch_dep(true, decode_combine_kernel<T, DD>, dim3((unsigned)nh), dim3(DD), 0, st, ds,    \
+                        (const float *)part, (T *)out, lse)) != cudaSuccess)                     \
+      return e;                                                                                 \
+  } while (0)
     if (bf16) { if (ds.d == 64) HILS_COMB(__nv_bfloat16, 64); else HILS_COMB(__nv_bfloat16, 128); }
     else { if (ds.d == 64) HILS_COMB(float, 64); else HILS_COMB(float, 128); }
 #undef HILS_COMB
