@@ -1054,15 +1054,28 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeSpec ds,
   const int h = blockIdx.x;  // b*Hq + hq
   const int b = h / ds.Hq, hq = h % ds.Hq;
   const int bk = b * ds.Hkv + hq / G, g = hq % G;
-  const size_t rec = 2 + D;
+  const size_t rec = 2 + D, stride = (size_t)G * rec;  // partial s of the head at r0 + s * stride
+  __shared__ float m_s;
   grid_dep_wait();  // the chunk attention's partials
-  float M = -INFINITY;
-  for (int s = 0; s < ds.Q; ++s) M = fmaxf(M, part[(((size_t)bk * ds.Q + s) * G + g) * rec]);
+  const float *r0 = part + ((size_t)bk * ds.Q * G + g) * rec;
+  // the partials' maximum: one load per lane of the first warp
+  if (threadIdx.x < 32) {
+    float m = -INFINITY;
+    for (int s = threadIdx.x; s < ds.Q; s += 32) m = fmaxf(m, r0[s * stride]);
+#pragma unroll
+    for (int o2 = 16; o2; o2 >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o2));
+    if (threadIdx.x == 0) m_s = m;
+  }
+  __syncthreads();
+  const float M = m_s;
+  // one pass over the partials in order, their loads independent of each other
   float L = 0.0f, o = 0.0f;
+#pragma unroll 8
   for (int s = 0; s < ds.Q; ++s) {
-    const float *r = part + (((size_t)bk * ds.Q + s) * G + g) * rec;
-    if (r[0] == -INFINITY) continue;
-    const float w = __expf(r[0] - M);
+    const float *r = r0 + s * stride;
+    const float m = r[0];
+    if (m == -INFINITY) continue;
+    const float w = __expf(m - M);
     L += w * r[1];
     o += w * r[2 + threadIdx.x];
   }
