@@ -58,14 +58,4 @@ __device__ __forceinline__ void report(uint32_t *err, uint32_t code) {
   if (err) atomicCAS(err, DEV_OK, code);
 }
 
-// Programmatic dependent launch.  A kernel launched with the programmatic
-// stream-serialization attribute may start while the kernel before it in the
-// stream is still running; grid_dep_wait() returns once that kernel has
-// completed and its writes are visible (at once for an ordinary launch), so
-// everything before it may only read inputs no kernel in flight writes.
-// grid_dep_launch() lets the next such kernel start launching once every
-// block of this grid has called it or exited.
-__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
 }  // namespace hils
