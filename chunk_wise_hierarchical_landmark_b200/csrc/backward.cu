@@ -21,8 +21,9 @@
 //                     dq with the D-dependent part factored out; then D and
 //                     the per-(row, slot) records (lse_c, w_c, g_c, ds_c).
 //   transposed selection: per (b, kv head, chunk) the (row, slot) pairs that
-//                     select it (count, exclusive scan, fill; the order inside
-//                     a chunk's list follows the atomic fill).
+//                     select it (counted by the row pass, exclusive scan,
+//                     fill; the order inside a chunk's list follows the atomic
+//                     fill).
 //   bwd_chunks_kernel one CTA per (b, kv head, chunk): a thread per (key,
 //                     quarter of the head dimension), that quarter of the
 //                     key's K and V rows in registers, accumulating dk and dv
@@ -119,7 +120,8 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)  // three CTAs per SM: a la
                     const int32_t *__restrict__ sel, const float *__restrict__ chunk_w,
                     const float *__restrict__ lse, const T *__restrict__ dout,
                     const float *__restrict__ dlse, float4 *__restrict__ rec,
-                    float *__restrict__ dq, uint32_t *__restrict__ err) {
+                    float *__restrict__ dq, uint32_t *__restrict__ cnt,
+                    uint32_t *__restrict__ err) {
   constexpr int DL = D / 8;  // dimensions per lane
   const int lane = threadIdx.x & 31, sub = lane & 7, grp = lane >> 3;
   const int wi = threadIdx.x >> 5;
@@ -252,12 +254,15 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)  // three CTAs per SM: a la
           make_float4((acc[u] - Dsum * accd[u]) * bs.scale, (acc[u + 1] - Dsum * accd[u + 1]) * bs.scale,
                       (acc[u + 2] - Dsum * accd[u + 2]) * bs.scale, (acc[u + 3] - Dsum * accd[u + 3]) * bs.scale);
   }
-  // ds_c = w_c (g_c - D + dlse) into the records of the attended slots
+  // ds_c = w_c (g_c - D + dlse) into the records of the attended slots, and
+  // the count of the (row, slot) pairs that select each chunk (the
+  // transposed selection's first step)
   __syncwarp();
   for (int slot = lane; slot <= K; slot += 32) {
     if (slot < K) {
       const int c = srow[slot];
       if (c < 0 || c >= own) continue;
+      atomicAdd(&cnt[((size_t)b * bs.Hkv + hkv) * bs.nch + c], 1u);
     }
     float4 r4 = rrow[slot];
     r4.w = r4.y * (r4.z - Dsum + dl);
@@ -265,20 +270,8 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)  // three CTAs per SM: a la
   }
 }
 
-// the (row, slot) pairs that select each (b, kv head, chunk): count ...
-__global__ void bwd_count_kernel(BwdSpec bs, const int32_t *__restrict__ sel,
-                                 uint32_t *__restrict__ cnt) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long n = (long long)bs.B * bs.Hq * bs.L * bs.topk;
-  if (i >= n) return;
-  const int c = sel[i];
-  const long long row = i / bs.topk;
-  const int t = (int)(row % bs.L), bh = (int)(row / bs.L);
-  if (c < 0 || c >= t / kC) return;
-  const int b = bh / bs.Hq, hkv = (bh % bs.Hq) / (bs.Hq / bs.Hkv);
-  atomicAdd(&cnt[((size_t)b * bs.Hkv + hkv) * bs.nch + c], 1u);
-}
-
+// the (row, slot) pairs that select each (b, kv head, chunk): counted by
+// the row pass ...
 // ... exclusive scan (one CTA; the counts become the fill cursors, zeroed) ...
 __global__ void __launch_bounds__(1024) bwd_scan_kernel(uint32_t *__restrict__ cnt,
                                                         uint32_t *__restrict__ off, int n) {
@@ -545,19 +538,19 @@ cudaError_t bwd_run(const BwdSpec &bs, bool bf16, const void *q, const void *k, 
   int32_t *ent_row = reinterpret_cast<int32_t *>(take(rows * bs.topk * sizeof(int32_t)));
   uint8_t *ent_slot = reinterpret_cast<uint8_t *>(take(rows * bs.topk));
   cudaError_t e;
+  // the row pass counts the (row, slot) pairs per chunk
+  if ((e = cudaMemsetAsync(cnt, 0, nseg * sizeof(uint32_t), st)) != cudaSuccess) return e;
   const unsigned rgrid = (unsigned)((rows + kRowWarps - 1) / kRowWarps);
 #define HILS_BWD_ROWS(T, DD)                                                                     \
   bwd_rows_kernel<T, DD><<<rgrid, kRowWarps * 32, 0, st>>>(                                     \
       bs, (const T *)q, (const T *)k, (const T *)v, (const T *)lmk, sel, chunk_w, lse,           \
-      (const T *)dout, dlse, rec, dq, err)
+      (const T *)dout, dlse, rec, dq, cnt, err)
   if (bf16) { if (bs.d == 64) HILS_BWD_ROWS(__nv_bfloat16, 64); else HILS_BWD_ROWS(__nv_bfloat16, 128); }
   else { if (bs.d == 64) HILS_BWD_ROWS(float, 64); else HILS_BWD_ROWS(float, 128); }
 #undef HILS_BWD_ROWS
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(cnt, 0, nseg * sizeof(uint32_t), st)) != cudaSuccess) return e;
   const long long nsel = (long long)rows * bs.topk;
   const unsigned sgrid = (unsigned)((nsel + 255) / 256);
-  bwd_count_kernel<<<sgrid, 256, 0, st>>>(bs, sel, cnt);
   bwd_scan_kernel<<<1, 1024, 0, st>>>(cnt, off, (int)nseg);
   bwd_fill_kernel<<<sgrid, 256, 0, st>>>(bs, sel, off, cnt, ent_row, ent_slot);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -570,7 +563,7 @@ cudaError_t bwd_run(const BwdSpec &bs, bool bf16, const void *q, const void *k, 
   if (bf16) { if (bs.d == 64) HILS_BWD_CHUNKS(__nv_bfloat16, 64); else HILS_BWD_CHUNKS(__nv_bfloat16, 128); }
   else { if (bs.d == 64) HILS_BWD_CHUNKS(float, 64); else HILS_BWD_CHUNKS(float, 128); }
 #undef HILS_BWD_CHUNKS
-  *launches += 5;
+  *launches += 4;
   return cudaGetLastError();
 }
 
