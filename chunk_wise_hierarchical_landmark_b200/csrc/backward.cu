@@ -109,6 +109,37 @@ __device__ __forceinline__ float dot2(const float (&x)[N], const float (&y)[N]) 
   return a.x + a.y;
 }
 
+// e += a.lo * b.lo, o += a.hi * b.hi for two packed bf16 pairs: the mixed-
+// precision FMA (bf16 operands, fp32 addend and result) rounds once, and a
+// product of two bf16 values is exact in fp32, so this equals widening both
+// operands and an fp32 FMA, without the widening instructions.
+__device__ __forceinline__ void fma_bf16x2(uint32_t a, uint32_t b, float &e, float &o) {
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+      "mov.b32 {al, ah}, %2;\n\t"
+      "mov.b32 {bl, bh}, %3;\n\t"
+      "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
+      "fma.rn.f32.bf16 %1, ah, bh, %1;\n\t}"
+      : "+f"(e), "+f"(o)
+      : "r"(a), "r"(b));
+}
+
+// <row, x> over a lane's N dimensions (16-byte aligned bf16 row, x as packed
+// bf16 pairs): even and odd dimensions summed apart and added at the end, the
+// order dot2 uses
+template <int N>
+__device__ __forceinline__ float dot_bf16(const __nv_bfloat16 *row, const uint32_t (&x)[N / 2]) {
+  float e = 0.0f, o = 0.0f;
+#pragma unroll
+  for (int u = 0; u < N; u += 8) {
+    const uint4 w = *reinterpret_cast<const uint4 *>(row + u);
+    fma_bf16x2(w.x, x[u / 2], e, o);
+    fma_bf16x2(w.y, x[u / 2 + 1], e, o);
+    fma_bf16x2(w.z, x[u / 2 + 2], e, o);
+    fma_bf16x2(w.w, x[u / 2 + 3], e, o);
+  }
+  return e + o;
+}
+
 // A warp per row.  Lane layout: eight lanes per key (sub = lane & 7 holds the
 // head dimensions [sub * DL, sub * DL + DL)), four keys per step (grp =
 // lane >> 3 takes key 4 i + grp at step i), so a 16-byte load of the warp
@@ -135,9 +166,21 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)  // three CTAs per SM: a la
   // per warp: (x, dP) and then (p, p dP) of the chunk's keys
   __shared__ float2 xd_s[kRowWarps][kC], pd_s[kRowWarps][kC];
   float2 *xd = xd_s[wi], *pp = pd_s[wi];
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   float qv[DL], dov[DL];
-  ld_vec<T, DL>(q + (size_t)row * D + sub * DL, qv);
-  ld_vec<T, DL>(dout + (size_t)row * D + sub * DL, dov);
+  uint32_t qp[DL / 2], dop[DL / 2];  // bf16: the lane's q and dO as packed pairs
+  if constexpr (kBf16) {
+#pragma unroll
+    for (int u = 0; u < DL; u += 8) {
+      const uint4 a = *reinterpret_cast<const uint4 *>(q + (size_t)row * D + sub * DL + u);
+      const uint4 c = *reinterpret_cast<const uint4 *>(dout + (size_t)row * D + sub * DL + u);
+      qp[u / 2] = a.x; qp[u / 2 + 1] = a.y; qp[u / 2 + 2] = a.z; qp[u / 2 + 3] = a.w;
+      dop[u / 2] = c.x; dop[u / 2 + 1] = c.y; dop[u / 2 + 2] = c.z; dop[u / 2 + 3] = c.w;
+    }
+  } else {
+    ld_vec<T, DL>(q + (size_t)row * D + sub * DL, qv);
+    ld_vec<T, DL>(dout + (size_t)row * D + sub * DL, dov);
+  }
   const float lse_t = lse[row];
   const float dl = dlse ? dlse[row] : 0.0f;
   const int32_t *srow = sel + (size_t)row * K;
@@ -182,10 +225,17 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3)  // three CTAs per SM: a la
 #pragma unroll 8
     for (int i = 0; i < nsteps; ++i) {
       const int jj = 4 * i + grp, j = min(jj, nkeys - 1);
-      float fk[DL], fv[DL];
-      ld_vec<T, DL>(kc + (size_t)j * D, fk);
-      ld_vec<T, DL>(vc + (size_t)j * D, fv);
-      float a = dot2<DL>(fk, qv), d = dot2<DL>(fv, dov);
+      float a, d;
+      if constexpr (kBf16) {
+        a = dot_bf16<DL>(kc + (size_t)j * D, qp);
+        d = dot_bf16<DL>(vc + (size_t)j * D, dop);
+      } else {
+        float fk[DL], fv[DL];
+        ld_vec<T, DL>(kc + (size_t)j * D, fk);
+        ld_vec<T, DL>(vc + (size_t)j * D, fv);
+        a = dot2<DL>(fk, qv);
+        d = dot2<DL>(fv, dov);
+      }
 #pragma unroll
       for (int o = 1; o < 8; o <<= 1) {
         a += __shfl_xor_sync(0xffffffffu, a, o);
