@@ -1,7 +1,8 @@
 """GPU parity of the backward pass (hils_attn_bwd) against the oracle's
 explicit per-chunk gradient formulas (oracle/backward.py, itself pinned to
 autograd and finite differences): dq, dk, dv and dlmk for the forward's
-selection, on GQA, ragged-length, k >= n_c and fp32 cases."""
+selection, on GQA, ragged-length, k >= n_c, k > 32 and fp32 (d = 64 and 128)
+cases."""
 import numpy as np
 import pytest
 import torch
@@ -21,10 +22,17 @@ CASES = [
     (W.TINY_F32.with_(Hq=2, Hkv=1, L=300, topk=8), 1e-4),
     # bf16, d=64, one query head per KV head, k=3, two sequences
     (W.SMALL_32K.with_(B=2, Hq=2, Hkv=2, L=520, topk=3), 2e-3),
+    # fp32, d=128, k=2 of up to 5 completed chunks (smallest gap at the k-th
+    # logit 8e-4 relative in fp64)
+    (W.TINY_F32.with_(d=128, Hq=2, Hkv=1, L=400, topk=2), 1e-4),
+    # bf16, d=64, k=40: more selected slots than a warp has lanes, ragged
+    # length (smallest gap at the k-th logit 2.6e-4 relative in fp64)
+    (W.SMALL_32K.with_(B=1, Hq=2, Hkv=1, L=64 * 44 + 17, topk=40), 2e-3),
 ]
 
 
-@pytest.mark.parametrize("w,tol", CASES, ids=["bf16_gqa_ragged", "f32_all_selected", "bf16_d64_b2"])
+@pytest.mark.parametrize("w,tol", CASES, ids=["bf16_gqa_ragged", "f32_all_selected", "bf16_d64_b2",
+                                              "f32_d128_k2", "bf16_k40"])
 def test_backward_matches_oracle(w, tol):
     q, k, v, lmk = synth.make_inputs(w, "cpu")
     g = torch.Generator().manual_seed(w.seed + 5)
