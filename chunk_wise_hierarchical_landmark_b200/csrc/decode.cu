@@ -44,6 +44,7 @@
 
 namespace hils {
 namespace {
+
 // Programmatic dependent launch.  A kernel launched with the programmatic
 // stream-serialization attribute may start while the kernel before it in the
 // stream is still running; grid_dep_wait() returns once that kernel has
@@ -1134,7 +1135,6 @@ size_t decode_max_g() { return kMaxG; }
 
 // A launch that may overlap the end of the kernel before it in the stream
 // (programmatic stream serialization): the kernel's grid_dep_wait() orders
-// its reads of that kernel's results.
 // its reads of that kernel's results.  dep = false: an ordinary launch.
 template <typename... KArgs, typename... Args>
 static cudaError_t launch_dep(bool dep, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
