@@ -14,7 +14,8 @@
 //                                                     its log-sum-exp)
 //   dq_t  = scale (sum_cj dx_j k_j + sum_{c selected} ds_c lmk_c)
 //   dk_j += scale dx_j q_t,  dv_j += w_c p_cj dO_t,  dlmk_c += scale ds_c q_t
-// Three stages, all on the CUDA cores in fp32 (bf16 inputs widen exactly):
+// Three stages, all on the CUDA cores with fp32 arithmetic (bf16 inputs widen
+// exactly, or enter a mixed-precision FMA whose products are exact):
 //   bwd_rows_kernel   one warp per row (eight lanes per key, four keys per
 //                     step), one pass over its chunks: per-chunk softmax
 //                     recomputed from q and the chunk's keys, g_c, w_c, and
@@ -24,9 +25,10 @@
 //                     select it (counted by the row pass, exclusive scan,
 //                     fill; the order inside a chunk's list follows the atomic
 //                     fill).
-//   bwd_chunks_kernel one CTA per (b, kv head, chunk): a thread per (key,
-//                     quarter of the head dimension), that quarter of the
-//                     key's K and V rows in registers, accumulating dk and dv
+//   bwd_chunks_kernel one CTA per (b, kv head, chunk): a thread per (keys,
+//                     quarter of the head dimension; two keys at d = 64),
+//                     that quarter of its keys' K and V rows in registers,
+//                     accumulating dk and dv
 //                     over the rows that attend the chunk (its own rows,
 //                     causally, and the rows that selected it; staged in
 //                     shared memory in batches), dlmk over the selecting rows.
