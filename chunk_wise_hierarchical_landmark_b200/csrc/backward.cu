@@ -28,10 +28,10 @@
 //   bwd_chunks_kernel one CTA per (b, kv head, chunk): a thread per (keys,
 //                     quarter of the head dimension; two keys at d = 64),
 //                     that quarter of its keys' K and V rows in registers,
-//                     accumulating dk and dv
-//                     over the rows that attend the chunk (its own rows,
-//                     causally, and the rows that selected it; staged in
-//                     shared memory in batches), dlmk over the selecting rows.
+//                     accumulating dk and dv over the rows that attend the
+//                     chunk (its own rows, causally, and the rows that
+//                     selected it; staged in shared memory in batches), dlmk
+//                     over the selecting rows.
 #include <cuda_bf16.h>
 
 #include <type_traits>
