@@ -147,7 +147,7 @@ __device__ __forceinline__ float dot_bf16(const __nv_bfloat16 *row, const uint32
 // lane >> 3 takes key 4 i + grp at step i), so a 16-byte load of the warp
 // covers four whole key rows and a dot product needs three shuffle levels.
 template <typename T, int D>
-__global__ void __launch_bounds__(kRowWarps * 32, 3)  // three CTAs per SM: a latency-bound loop
+__global__ void __launch_bounds__(kRowWarps * 32, D == 64 ? 3 : 2)  // resident CTAs: a latency-bound loop
     bwd_rows_kernel(BwdSpec bs, const T *__restrict__ q, const T *__restrict__ k,
                     const T *__restrict__ v, const T *__restrict__ lmk,
                     const int32_t *__restrict__ sel, const float *__restrict__ chunk_w,
