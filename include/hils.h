@@ -35,7 +35,11 @@
  *   state other than cached device attributes, a launch counter and the
  *   fixed scratch array of hils_decode_fwd_noalloc (module memory, below).
  *   Streams: every call is asynchronous on `stream` (a cudaStream_t passed as
- *   void*; NULL = legacy default stream).  Argument and shape errors are
+ *   void*; NULL = legacy default stream) and ordered on it as a whole: a
+ *   call's first kernel starts after the work queued before it, and work
+ *   queued after it starts after its last kernel (inside a decode call the
+ *   kernels after the first overlap their predecessors' ends through
+ *   programmatic dependent launch).  Argument and shape errors are
  *   returned before anything is launched.  A launch failure returns
  *   HILS_ERR_CUDA.  With params.debug_checks = 1 the call also validates its
  *   selections on the device and synchronises the stream to report
